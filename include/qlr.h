@@ -1,0 +1,220 @@
+/*
+ * qlr.h -- C ABI of the quantised-base + LoRA linear library for NVIDIA B200 (sm_100a).
+ *
+ * The layer is  Y = X dequant(Wq)^T + s (P(X) A^T) B^T  with a frozen low-bit base
+ * weight Wq and a trainable low-rank adapter (A, B); P is the identity (QLoRA, LQ-LoRA)
+ * or the group mean over L input channels (QA-LoRA).
+ *
+ * Conventions shared by every entry point
+ *   - Return value: QLR_OK (0) or a negative QLR_ERR_* code.  Arguments are validated on the
+ *     host before anything is launched; an invalid call launches nothing and leaves every
+ *     buffer untouched.
+ *   - Pointers are caller-owned DEVICE memory unless stated otherwise; the library keeps no
+ *     allocation of its own.  Scratch space is passed in as `workspace` (device memory of at
+ *     least the size the matching *_workspace_bytes query returns, 256-byte aligned).
+ *   - bf16 and fp16 buffers are passed as uint16_t bit patterns.  Matrices are row-major and
+ *     densely packed (leading dimension = number of columns); every pointer must be 16-byte
+ *     aligned.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).  All work is
+ *     asynchronous on that stream.
+ *   - `status` (optional, may be NULL) is a device int32 that kernels set to a negative
+ *     QLR_ERR_* code when they detect a fault at run time (non-finite weights in a quantiser,
+ *     a pipeline wait that ran past its bound).  The caller zeroes it and reads it after
+ *     synchronising the stream.  Kernels never trap.
+ *   - Shapes: W is [N, K] (out_features x in_features), X is [M, K], Y is [M, N], A is [r, Ka]
+ *     (Ka = K, or K / group for the pooled adapter), B is [N, r].
+ */
+#ifndef QLR_H
+#define QLR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define QLR_API __attribute__((visibility("default")))
+#else
+#define QLR_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  QLR_OK = 0,
+  QLR_ERR_ARG = -1,         /* null pointer, unknown enum value, negative size */
+  QLR_ERR_SHAPE = -2,       /* sizes the kernels do not support (see each call) */
+  QLR_ERR_ALIGN = -3,       /* a pointer is not 16-byte aligned */
+  QLR_ERR_UNSUPPORTED = -4, /* a valid combination this build does not implement */
+  QLR_ERR_NONFINITE = -5,   /* set in *status by a quantiser that met a NaN or infinity */
+  QLR_ERR_TIMEOUT = -6,     /* set in *status by a pipelined kernel whose wait ran out */
+  QLR_ERR_CUDA = -7,        /* a CUDA runtime/driver call failed */
+  QLR_ERR_WORKSPACE = -8    /* workspace missing or smaller than the query's answer */
+};
+
+enum { QLR_FMT_NFK = 1, QLR_FMT_INT4G = 2 };
+
+/* Parts of a quantised weight, for qlr_qweight_part_bytes. */
+enum { QLR_PART_CODES = 0, QLR_PART_C1 = 1, QLR_PART_C1_FP8 = 2, QLR_PART_S2 = 3,
+       QLR_PART_SCALE = 4, QLR_PART_ZERO = 5 };
+
+/*
+ * A quantised base weight.  The struct is plain data owned by the caller; its pointers are
+ * caller-allocated device buffers of the sizes qlr_qweight_part_bytes reports.
+ *
+ * NF-k (fmt = QLR_FMT_NFK; QLoRA explainer, "Innovation 1: 4-bit NormalFloat (NF4)" and
+ * "Innovation 2: Double Quantization"; LQ-LoRA abstract for k = 2, 3 and block 64/128):
+ *   codes   packed k-bit codes of the row-major flattened W.  k=4: two per byte, element 2j in
+ *           the low nibble; k=2: four per byte, element 4j+t at bits 2t..2t+1; k=3: per 32
+ *           codes three little-endian uint32 bit planes (word p holds bit p of code t at bit t).
+ *   c1      fp32 absmax per block of `block` consecutive weights (only when dq_block == 0).
+ *   c1_fp8  E4M3 byte per block: c1 / s2 rounded to nearest even, saturated (dq_block > 0).
+ *   s2      fp32 per group of dq_block blocks: max(c1 in group) / 448 (dq_block > 0).
+ * INT4 group (fmt = QLR_FMT_INT4G; QA-LoRA abstract, group-wise INT4):
+ *   codes   packed like NF-4, row-major [N, K];
+ *   scale   fp16 [N, K / group];  zero  fp16 [N, K / group] (integer before a merge).
+ */
+typedef struct qlr_qweight {
+  int32_t fmt;
+  int32_t bits;
+  int32_t block;
+  int32_t dq_block;
+  int32_t group;
+  int32_t reserved;
+  int64_t N;
+  int64_t K;
+  uint8_t* codes;
+  float* c1;
+  uint8_t* c1_fp8;
+  float* s2;
+  uint16_t* scale;
+  uint16_t* zero;
+} qlr_qweight;
+
+/* Static text for a return code.  Never NULL. */
+QLR_API const char* qlr_error_string(int code);
+
+/* Library ABI version (major * 100 + minor). */
+QLR_API int qlr_version(void);
+
+/* Number of bytes a part of a quantised weight occupies (0 when the format has no such part,
+ * negative QLR_ERR_* for invalid arguments).  Pure host arithmetic. */
+QLR_API int64_t qlr_qweight_part_bytes(int fmt, int64_t N, int64_t K, int bits, int block, int dq_block, int group,
+                               int part);
+
+/* The fp32 NF-k levels the library uses (2^bits values, ascending), derived on the host from
+ * an inverse normal CDF (AS241) by the quantile construction: positive levels at 2^(k-1)
+ * evenly spaced probabilities from delta toward 1/2, negative levels at 2^(k-1)-1, an exact
+ * zero, divided by the quantile at delta, delta = 1 - (1/(2(2^k-1)) + 1/(2^(k+1)))/2.
+ * (QLoRA explainer, "Innovation 1: 4-bit NormalFloat (NF4)": equal share of a normal
+ * distribution per bin.)  `out` is HOST memory of 2^bits floats. */
+QLR_API int qlr_nf_levels(int bits, float* out);
+
+/*
+ * Blockwise NF-k quantisation with optional double quantisation of the constants.
+ * (QLoRA explainer, "Background: what is quantization?", "Innovation 1", the page's code
+ * sketch for absmax / nearest level, "Innovation 2: Double Quantization".)
+ *   W         fp32 [N, K] device, read only.
+ *   bits      2, 3 or 4;  block  64 or 128;  dq_block  256 or 0.
+ *   out       describes the destination buffers (out->fmt/bits/block/dq_block/N/K are checked
+ *             against the arguments); codes, and c1 or (c1_fp8, s2), are written.
+ * Per element: u = fp32(w / absmax) (IEEE division), code = first index minimising
+ * fp32 |u - level|; an all-zero block takes the zero level.  Non-finite W sets
+ * *status = QLR_ERR_NONFINITE (outputs are then unspecified).
+ * Shapes: N*K a multiple of 128 (so blocks, bit-plane groups and bytes never straddle a unit).
+ */
+QLR_API int qlr_quantize_nf4(const float* W, int64_t N, int64_t K, int bits, int block, int dq_block,
+                     const qlr_qweight* out, int32_t* status, void* stream);
+
+/*
+ * Group-wise asymmetric INT4 quantisation (QA-LoRA abstract: group-wise operators, INT4).
+ * Per (row o, group g of `group` consecutive inputs): lo = min(0, min w), hi = max(0, max w),
+ * scale = fp16(fp32(hi - lo) / 15), z = clamp(rne(-lo / scale), 0, 15),
+ * code = clamp(rne(fp32(w / scale) + z), 0, 15); a zero scale gives z = 0 and codes 0.
+ *   W fp32 [N, K] device;  group 32, 64 or 128, dividing K.
+ *   out->codes [N, K/2] bytes, out->scale and out->zero fp16 [N, K/group].
+ */
+QLR_API int qlr_quantize_int4_group(const float* W, int64_t N, int64_t K, int group, const qlr_qweight* out,
+                            int32_t* status, void* stream);
+
+/*
+ * Dequantise a whole weight to bf16 (W_out [N, K] device).  NF-k:
+ * bf16(level[code] * (fp32(E4M3(c1_fp8)) * s2)) (or level * c1 without double
+ * quantisation); INT4 group: bf16(fp32(code - zero) * scale).  Each product is one fp32
+ * multiplication rounded to nearest; the result is the exact value every GEMM of this
+ * library multiplies with.  (QLoRA explainer, "The QLoRA recipe", stage 3: dequantised to
+ * BFloat16.)
+ */
+QLR_API int qlr_dequant(const qlr_qweight* w, uint16_t* W_out, int32_t* status, void* stream);
+
+/*
+ * QA-LoRA merge (QA-LoRA abstract: after fine-tuning the adapter is integrated into the
+ * quantised model without loss of accuracy).  With the pooled adapter, s (B A)[o, g] / L is
+ * added to every weight of group g of row o, which is a shift of the zero point:
+ *   zero'[o, g] = fp16( zero - s * (B A)[o, g] / (group * scale[o, g]) ),  in fp64;
+ * groups with scale == 0 keep their zero.  w->zero is rewritten in place.
+ *   A bf16 [r, K/group], B bf16 [N, r];  w->fmt must be QLR_FMT_INT4G.
+ */
+QLR_API int qlr_qalora_merge(const qlr_qweight* w, const uint16_t* A, const uint16_t* B, int r, float s,
+                     int32_t* status, void* stream);
+
+/*
+ * Forward pass of the layer (QLoRA explainer, "The QLoRA recipe", stage 3 and "The complete
+ * QLoRA forward pass"; QA-LoRA pooled adapter when w->fmt == QLR_FMT_INT4G and pooled != 0):
+ *   T_save = bf16( s * P(X) A^T )                               [M, r]
+ *   Y      = bf16( X dequant(W)^T + T_save B^T )                 [M, N]
+ * The dequantised weight never reaches global memory: the fused kernel streams the packed
+ * codes into shared memory, dequantises them there and feeds tcgen05 tensor-core tiles;
+ * the adapter term is added as r extra reduction columns of the same accumulator.
+ * Token counts M <= 16 with 4-bit NF codes take a memory-streaming decode kernel instead.
+ *   X bf16 [M, K];  A bf16 [r, Ka];  B bf16 [N, r];  Y bf16 [M, N];  T_save bf16 [M, r].
+ *   r in {8, 16, 32, 64};  K a multiple of 64 (and of w->block);  N a multiple of 8.
+ */
+QLR_API size_t qlr_forward_workspace_bytes(const qlr_qweight* w, int64_t M, int r, int pooled);
+QLR_API int qlr_forward(const qlr_qweight* w, const uint16_t* X, int64_t M, const uint16_t* A, const uint16_t* B, int r,
+                float s, int pooled, uint16_t* Y, uint16_t* T_save, void* workspace, size_t workspace_bytes,
+                int32_t* status, void* stream);
+
+/*
+ * Adapter gradients (QLoRA explainer, "Background: how LoRA works" and "The QLoRA recipe":
+ * gradients reach only A and B).  With T_save from qlr_forward:
+ *   dT = bf16( s * dY B )          [M, r]   (written to dT_out, consumed by qlr_backward_dx)
+ *   dB = dY^T T_save               [N, r]   fp32
+ *   dA = dT^T P(X)                 [r, Ka]  fp32  (dT taken in bf16)
+ * Each fp32 reduction over tokens is split across CTAs and summed in a fixed order, so the
+ * results are deterministic.
+ */
+QLR_API size_t qlr_backward_lora_workspace_bytes(const qlr_qweight* w, int64_t M, int r, int pooled);
+QLR_API int qlr_backward_lora(const qlr_qweight* w, const uint16_t* X, const uint16_t* dY, const uint16_t* T_save,
+                      const uint16_t* B, int64_t M, int r, float s, int pooled, float* dA, float* dB,
+                      uint16_t* dT_out, void* workspace, size_t workspace_bytes, int32_t* status, void* stream);
+
+/*
+ * Input gradient through the frozen quantised weight (QLoRA explainer, "The contribution":
+ * backpropagate through the frozen 4-bit weights into the adapters):
+ *   dX = bf16( dY dequant(W) + P^T(dT A) )  [M, K]   (+ the previous dX when accumulate != 0)
+ * P^T spreads each pooled column over its group with weight 1/group.  Same fused
+ * dequant + tcgen05 design as the forward, with the weight tile laid out MN-major.
+ */
+QLR_API size_t qlr_backward_dx_workspace_bytes(const qlr_qweight* w, int64_t M, int r, int pooled);
+QLR_API int qlr_backward_dx(const qlr_qweight* w, const uint16_t* dY, int64_t M, const uint16_t* A, const uint16_t* dT,
+                    int r, int pooled, int accumulate, uint16_t* dX, void* workspace, size_t workspace_bytes,
+                    int32_t* status, void* stream);
+
+/*
+ * SwiGLU between the gate/up and down projections of an MLP block (the LLaMA-7B-shaped
+ * workload): H = silu(G) * U;  backward dG = dH U sig(G) (1 + G (1 - sig(G))), dU = dH silu(G).
+ * All bf16 [n] device buffers, fp32 arithmetic, n >= 0.
+ */
+QLR_API int qlr_swiglu_forward(const uint16_t* G, const uint16_t* U, uint16_t* H, int64_t n, void* stream);
+QLR_API int qlr_swiglu_backward(const uint16_t* dH, const uint16_t* G, const uint16_t* U, uint16_t* dG, uint16_t* dU,
+                        int64_t n, void* stream);
+
+/* Number of SMs of the current device (used to size persistent grids); <= 0 on error. */
+QLR_API int qlr_device_sm_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLR_H */

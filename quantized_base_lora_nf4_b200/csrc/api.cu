@@ -1,0 +1,511 @@
+// C-ABI entry points: argument validation (before any launch), workspace carving, tensor maps,
+// and the launch sequence of each call.  See include/qlr.h for the contract of every function.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "gemm.cuh"
+
+namespace qlr {
+
+__device__ int32_t g_status_sink;
+
+int32_t* status_or_sink(int32_t* status) {
+  if (status) return status;
+  static int32_t* sink = nullptr;
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  int dev = 0;
+  cudaGetDevice(&dev);
+  static int32_t* per_dev[64] = {nullptr};
+  if (dev >= 0 && dev < 64 && !per_dev[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status_sink) == cudaSuccess) per_dev[dev] = static_cast<int32_t*>(p);
+  }
+  sink = (dev >= 0 && dev < 64) ? per_dev[dev] : nullptr;
+  return sink;
+}
+
+Levels levels_for(int bits) {
+  Levels l;
+  for (int i = 0; i < 16; ++i) l.v[i] = 0.f;
+  if (bits >= 2 && bits <= 4) nf_levels_f32(bits, l.v);
+  return l;
+}
+
+int device_sm_count() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!cache[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+}  // namespace qlr
+
+using namespace qlr;
+
+namespace {
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+inline int cuda_rc(cudaError_t e) { return e == cudaSuccess ? QLR_OK : QLR_ERR_CUDA; }
+inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+int check_qweight(const qlr_qweight* w) {
+  if (!w || w->N <= 0 || w->K <= 0 || !w->codes) return QLR_ERR_ARG;
+  if (!aligned16(w->codes)) return QLR_ERR_ALIGN;
+  if (w->fmt == QLR_FMT_NFK) {
+    if (w->bits < 2 || w->bits > 4) return QLR_ERR_ARG;
+    if (w->block != 64 && w->block != 128) return QLR_ERR_ARG;
+    if (w->dq_block != 0 && w->dq_block != 256) return QLR_ERR_ARG;
+    if (w->dq_block ? (!w->c1_fp8 || !w->s2) : !w->c1) return QLR_ERR_ARG;
+    if ((w->N * w->K) % 128) return QLR_ERR_SHAPE;
+    return QLR_OK;
+  }
+  if (w->fmt == QLR_FMT_INT4G) {
+    if (w->group != 32 && w->group != 64 && w->group != 128) return QLR_ERR_ARG;
+    if (!w->scale || !w->zero) return QLR_ERR_ARG;
+    if (w->K % w->group) return QLR_ERR_SHAPE;
+    return QLR_OK;
+  }
+  return QLR_ERR_ARG;
+}
+
+// Shapes the fused tensor-core paths support.
+int check_gemm_weight(const qlr_qweight* w) {
+  int rc = check_qweight(w);
+  if (rc) return rc;
+  if (w->fmt == QLR_FMT_NFK && w->bits != 4) return QLR_ERR_UNSUPPORTED;
+  if (w->K % 64 || w->N % 8) return QLR_ERR_SHAPE;
+  if (w->fmt == QLR_FMT_NFK && w->K % w->block) return QLR_ERR_SHAPE;
+  if (w->N > (int64_t(1) << 30) || w->K > (int64_t(1) << 30)) return QLR_ERR_SHAPE;
+  return QLR_OK;
+}
+
+int check_rank(int r) { return (r == 8 || r == 16 || r == 32 || r == 64) ? QLR_OK : QLR_ERR_SHAPE; }
+
+int adapter_bn(int r) { return r <= 32 ? 32 : 64; }
+
+DqParams dq_params(const qlr_qweight* w) {
+  DqParams d;
+  d.fmt = w->fmt;
+  d.bits = w->bits;
+  d.block = w->block;
+  d.dq_block = w->dq_block;
+  d.group = w->group;
+  d.N = w->N;
+  d.K = w->K;
+  d.c1 = w->c1;
+  d.c1_fp8 = w->c1_fp8;
+  d.s2 = w->s2;
+  d.scale = reinterpret_cast<const __half*>(w->scale);
+  d.zero = reinterpret_cast<const __half*>(w->zero);
+  d.lv = levels_for(w->fmt == QLR_FMT_NFK ? w->bits : 4);
+  return d;
+}
+
+// Splits for a reduction of n_steps 64-wide steps over `tiles` output tiles.
+int pick_splits(int64_t tiles, int64_t n_steps) {
+  const int64_t sms = device_sm_count();
+  int64_t s = cdiv(sms, tiles);
+  const int64_t max_s = n_steps / 2 > 0 ? n_steps / 2 : 1;
+  if (s > max_s) s = max_s;
+  if (s > 16) s = 16;
+  return static_cast<int>(s < 1 ? 1 : s);
+}
+
+size_t partial_bytes(int64_t Mm, int bn, int splits) { return size_t(splits) * cdiv(Mm, 128) * 128 * bn * 4; }
+
+// One adapter GEMM into fp32 partials (split-K), followed by the fixed-order reduction.
+struct AdapterGemm {
+  int a_src, b_src, bn;
+  int64_t Mm, Nn, kred;
+  const void* a_ptr;
+  int64_t a_rows, a_cols;  // row-major extents of the A source matrix
+  const void* b_ptr;
+  int64_t b_rows, b_cols;
+};
+
+int run_adapter_gemm(const AdapterGemm& g, float* part, int splits, int32_t* status, cudaStream_t st) {
+  GemmMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  int rc;
+  if (g.a_src == A_TMA_K)
+    rc = make_tmap(&maps.a, g.a_ptr, 2, g.a_rows, g.a_cols, 128, 64, 128);
+  else
+    rc = make_tmap(&maps.a, g.a_ptr, 2, g.a_rows, g.a_cols, 64, 64, 128);
+  if (rc) return rc;
+  const int atom = g.bn >= 64 ? 64 : g.bn;
+  if (g.b_src == B_TMA_K)
+    rc = make_tmap(&maps.b, g.b_ptr, 2, g.b_rows, g.b_cols, g.bn, 64, 128);
+  else
+    rc = make_tmap(&maps.b, g.b_ptr, 2, g.b_rows, g.b_cols, 64, atom, atom * 2);
+  if (rc) return rc;
+  maps.a_tail = maps.a;
+  maps.b_tail = maps.b;
+  maps.codes = maps.a;
+  GemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.Mm = static_cast<int>(g.Mm);
+  p.Nn = static_cast<int>(g.Nn);
+  p.n_main = static_cast<int>(cdiv(g.kred, 64));
+  p.splits = splits;
+  p.n_tail = 0;
+  p.r_tail = 0;
+  p.m_tiles = static_cast<int>(cdiv(g.Mm, 128));
+  p.n_tiles = 1;
+  p.b_atom = atom;
+  p.out = part;
+  p.ldo = g.bn;
+  p.accumulate = 0;
+  p.status = status;
+  return cuda_rc(launch_gemm(g.a_src, g.b_src, g.bn, OUT_F32_D, 0, p, maps, st));
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* qlr_error_string(int code) {
+  switch (code) {
+    case QLR_OK: return "ok";
+    case QLR_ERR_ARG: return "invalid argument";
+    case QLR_ERR_SHAPE: return "unsupported shape";
+    case QLR_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case QLR_ERR_UNSUPPORTED: return "unsupported combination";
+    case QLR_ERR_NONFINITE: return "non-finite input";
+    case QLR_ERR_TIMEOUT: return "pipeline wait timed out";
+    case QLR_ERR_CUDA: return "CUDA error";
+    case QLR_ERR_WORKSPACE: return "workspace missing or too small";
+    default: return "unknown error";
+  }
+}
+
+int qlr_version(void) { return 100; }
+
+int qlr_device_sm_count(void) { return device_sm_count(); }
+
+int qlr_nf_levels(int bits, float* out) {
+  if (!out || bits < 2 || bits > 4) return QLR_ERR_ARG;
+  nf_levels_f32(bits, out);
+  return QLR_OK;
+}
+
+int64_t qlr_qweight_part_bytes(int fmt, int64_t N, int64_t K, int bits, int block, int dq_block, int group,
+                               int part) {
+  if (N <= 0 || K <= 0) return QLR_ERR_ARG;
+  const int64_t n = N * K;
+  if (fmt == QLR_FMT_NFK) {
+    if (bits < 2 || bits > 4 || (block != 64 && block != 128) || (dq_block != 0 && dq_block != 256))
+      return QLR_ERR_ARG;
+    const int64_t nb = cdiv(n, block);
+    switch (part) {
+      case QLR_PART_CODES: return nb * block * bits / 8;
+      case QLR_PART_C1: return dq_block ? 0 : 4 * nb;
+      case QLR_PART_C1_FP8: return dq_block ? nb : 0;
+      case QLR_PART_S2: return dq_block ? 4 * cdiv(nb, dq_block) : 0;
+      case QLR_PART_SCALE:
+      case QLR_PART_ZERO: return 0;
+      default: return QLR_ERR_ARG;
+    }
+  }
+  if (fmt == QLR_FMT_INT4G) {
+    if (group <= 0 || K % group) return QLR_ERR_ARG;
+    switch (part) {
+      case QLR_PART_CODES: return n / 2;
+      case QLR_PART_SCALE:
+      case QLR_PART_ZERO: return 2 * N * (K / group);
+      case QLR_PART_C1:
+      case QLR_PART_C1_FP8:
+      case QLR_PART_S2: return 0;
+      default: return QLR_ERR_ARG;
+    }
+  }
+  return QLR_ERR_ARG;
+}
+
+int qlr_quantize_nf4(const float* W, int64_t N, int64_t K, int bits, int block, int dq_block,
+                     const qlr_qweight* out, int32_t* status, void* stream) {
+  if (!W || !out) return QLR_ERR_ARG;
+  if (out->fmt != QLR_FMT_NFK || out->bits != bits || out->block != block || out->dq_block != dq_block ||
+      out->N != N || out->K != K)
+    return QLR_ERR_ARG;
+  const int rc = check_qweight(out);
+  if (rc) return rc;
+  if (!aligned16(W)) return QLR_ERR_ALIGN;
+  return cuda_rc(launch_quantize_nfk(W, N * K, bits, block, dq_block, out, status_or_sink(status), as_stream(stream)));
+}
+
+int qlr_quantize_int4_group(const float* W, int64_t N, int64_t K, int group, const qlr_qweight* out,
+                            int32_t* status, void* stream) {
+  if (!W || !out) return QLR_ERR_ARG;
+  if (out->fmt != QLR_FMT_INT4G || out->group != group || out->N != N || out->K != K) return QLR_ERR_ARG;
+  const int rc = check_qweight(out);
+  if (rc) return rc;
+  if (!aligned16(W)) return QLR_ERR_ALIGN;
+  return cuda_rc(launch_quantize_int4g(W, N, K, group, out, status_or_sink(status), as_stream(stream)));
+}
+
+int qlr_dequant(const qlr_qweight* w, uint16_t* W_out, int32_t* status, void* stream) {
+  (void)status;
+  int rc = check_qweight(w);
+  if (rc) return rc;
+  if (!W_out) return QLR_ERR_ARG;
+  if (!aligned16(W_out)) return QLR_ERR_ALIGN;
+  if ((w->N * w->K) % 32) return QLR_ERR_SHAPE;
+  return cuda_rc(launch_dequant(w, W_out, as_stream(stream)));
+}
+
+int qlr_qalora_merge(const qlr_qweight* w, const uint16_t* A, const uint16_t* B, int r, float s, int32_t* status,
+                     void* stream) {
+  (void)status;
+  int rc = check_qweight(w);
+  if (rc) return rc;
+  if (w->fmt != QLR_FMT_INT4G) return QLR_ERR_ARG;
+  if (!A || !B || r <= 0 || r > 1024) return QLR_ERR_ARG;
+  return cuda_rc(launch_merge(w, A, B, r, s, as_stream(stream)));
+}
+
+// ---- forward -------------------------------------------------------------------------------------
+
+size_t qlr_forward_workspace_bytes(const qlr_qweight* w, int64_t M, int r, int pooled) {
+  if (check_qweight(w) || M <= 0 || check_rank(r)) return 0;
+  const int64_t Ka = pooled ? w->K / w->group : w->K;
+  size_t bytes = 0;
+  if (pooled) bytes += align256(size_t(M) * Ka * 2);
+  const int bn = adapter_bn(r);
+  const int splits = pick_splits(cdiv(M, 128), cdiv(Ka, 64));
+  bytes += align256(partial_bytes(M, bn, splits));
+  return bytes;
+}
+
+int qlr_forward(const qlr_qweight* w, const uint16_t* X, int64_t M, const uint16_t* A, const uint16_t* B, int r,
+                float s, int pooled, uint16_t* Y, uint16_t* T_save, void* workspace, size_t workspace_bytes,
+                int32_t* status, void* stream) {
+  int rc = check_gemm_weight(w);
+  if (rc) return rc;
+  if ((rc = check_rank(r))) return rc;
+  if (M < 0) return QLR_ERR_ARG;
+  if (M == 0) return QLR_OK;
+  if (!X || !A || !B || !Y || !T_save) return QLR_ERR_ARG;
+  if (!aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(Y) || !aligned16(T_save)) return QLR_ERR_ALIGN;
+  if (pooled && w->fmt != QLR_FMT_INT4G) return QLR_ERR_UNSUPPORTED;
+  if (pooled && (w->K / w->group) % 8) return QLR_ERR_SHAPE;
+  if (M == 0) return QLR_OK;
+  if (M > (int64_t(1) << 30)) return QLR_ERR_SHAPE;
+  const size_t need = qlr_forward_workspace_bytes(w, M, r, pooled);
+  if (!workspace || workspace_bytes < need) return QLR_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return QLR_ERR_ALIGN;
+  cudaStream_t st = as_stream(stream);
+  int32_t* stat = status_or_sink(status);
+  const int64_t N = w->N, K = w->K;
+  const int64_t Ka = pooled ? K / w->group : K;
+
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const uint16_t* Xa = X;
+  if (pooled) {
+    uint16_t* Xp = reinterpret_cast<uint16_t*>(ws);
+    ws += align256(size_t(M) * Ka * 2);
+    if ((rc = cuda_rc(launch_pool(X, M, K, w->group, Xp, st)))) return rc;
+    Xa = Xp;
+  }
+  // T_save = bf16(s * P(X) A^T): split-K tensor-core GEMM into fp32 partials, then a fixed-order sum
+  const int bn = adapter_bn(r);
+  const int splits = pick_splits(cdiv(M, 128), cdiv(Ka, 64));
+  float* part = reinterpret_cast<float*>(ws);
+  AdapterGemm g{A_TMA_K, B_TMA_K, bn, M, r, Ka, Xa, M, Ka, A, r, Ka};
+  if ((rc = run_adapter_gemm(g, part, splits, stat, st))) return rc;
+  if ((rc = cuda_rc(launch_reduce_splits(part, splits, M, r, bn, s, 0, 1, T_save, r, st)))) return rc;
+
+  // Y = X dequant(W)^T + T_save B^T: fused dequant + tcgen05, computed as Y^T tiles (W rows on TMEM lanes)
+  const int bn_tok = M >= 192 ? 256 : 64;
+  GemmMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  if ((rc = make_tmap(&maps.codes, w->codes, 1, N, K / 2, 128, 32, 0))) return rc;
+  if ((rc = make_tmap(&maps.b, X, 2, M, K, bn_tok, 64, 128))) return rc;
+  if ((rc = make_tmap(&maps.a_tail, B, 2, N, r, 128, 64, 128))) return rc;
+  if ((rc = make_tmap(&maps.b_tail, T_save, 2, M, r, bn_tok, 64, 128))) return rc;
+  maps.a = maps.a_tail;
+  GemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.Mm = static_cast<int>(N);
+  p.Nn = static_cast<int>(M);
+  p.n_main = static_cast<int>(K / 64);
+  p.splits = 1;
+  p.n_tail = static_cast<int>(cdiv(r, 64));
+  p.r_tail = r;
+  p.m_tiles = static_cast<int>(cdiv(N, 128));
+  p.n_tiles = static_cast<int>(cdiv(M, bn_tok));
+  p.b_atom = 64;
+  p.out = Y;
+  p.ldo = N;
+  p.accumulate = 0;
+  p.dq = dq_params(w);
+  p.status = stat;
+  return cuda_rc(launch_gemm(A_DQ_K, B_TMA_K, bn_tok, OUT_BF16_T, 0, p, maps, st));
+}
+
+// ---- backward: adapter gradients -------------------------------------------------------------------
+
+size_t qlr_backward_lora_workspace_bytes(const qlr_qweight* w, int64_t M, int r, int pooled) {
+  if (check_qweight(w) || M <= 0 || check_rank(r)) return 0;
+  const int64_t N = w->N;
+  const int64_t Ka = pooled ? w->K / w->group : w->K;
+  size_t bytes = 0;
+  if (pooled) bytes += align256(size_t(M) * Ka * 2);
+  const int bn = adapter_bn(r);
+  size_t p1 = partial_bytes(M, bn, pick_splits(cdiv(M, 128), cdiv(N, 64)));
+  size_t p2 = partial_bytes(N, bn, pick_splits(cdiv(N, 128), cdiv(M, 64)));
+  size_t p3 = partial_bytes(Ka, bn, pick_splits(cdiv(Ka, 128), cdiv(M, 64)));
+  size_t mx = p1 > p2 ? p1 : p2;
+  mx = mx > p3 ? mx : p3;
+  return bytes + align256(mx);
+}
+
+int qlr_backward_lora(const qlr_qweight* w, const uint16_t* X, const uint16_t* dY, const uint16_t* T_save,
+                      const uint16_t* B, int64_t M, int r, float s, int pooled, float* dA, float* dB,
+                      uint16_t* dT_out, void* workspace, size_t workspace_bytes, int32_t* status, void* stream) {
+  int rc = check_gemm_weight(w);
+  if (rc) return rc;
+  if ((rc = check_rank(r))) return rc;
+  if (M < 0) return QLR_ERR_ARG;
+  if (!dA || !dB) return QLR_ERR_ARG;
+  if (M > 0 && (!X || !dY || !T_save || !B || !dT_out)) return QLR_ERR_ARG;
+  if (!aligned16(X) || !aligned16(dY) || !aligned16(T_save) || !aligned16(B) || !aligned16(dA) || !aligned16(dB) ||
+      !aligned16(dT_out))
+    return QLR_ERR_ALIGN;
+  if (pooled && w->fmt != QLR_FMT_INT4G) return QLR_ERR_UNSUPPORTED;
+  if (pooled && (w->K / w->group) % 8) return QLR_ERR_SHAPE;
+  cudaStream_t st = as_stream(stream);
+  const int64_t N = w->N, K = w->K;
+  const int64_t Ka = pooled ? K / w->group : K;
+  if (M == 0) {
+    // no tokens: the gradients are zero
+    if (cudaMemsetAsync(dA, 0, size_t(r) * Ka * 4, st) != cudaSuccess) return QLR_ERR_CUDA;
+    return cuda_rc(cudaMemsetAsync(dB, 0, size_t(N) * r * 4, st));
+  }
+  if (M > (int64_t(1) << 30)) return QLR_ERR_SHAPE;
+  const size_t need = qlr_backward_lora_workspace_bytes(w, M, r, pooled);
+  if (!workspace || workspace_bytes < need) return QLR_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return QLR_ERR_ALIGN;
+  int32_t* stat = status_or_sink(status);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const uint16_t* Xa = X;
+  if (pooled) {
+    uint16_t* Xp = reinterpret_cast<uint16_t*>(ws);
+    ws += align256(size_t(M) * Ka * 2);
+    if ((rc = cuda_rc(launch_pool(X, M, K, w->group, Xp, st)))) return rc;
+    Xa = Xp;
+  }
+  float* part = reinterpret_cast<float*>(ws);
+  const int bn = adapter_bn(r);
+  // dT = bf16(s dY B)
+  {
+    const int splits = pick_splits(cdiv(M, 128), cdiv(N, 64));
+    AdapterGemm g{A_TMA_K, B_TMA_MN, bn, M, r, N, dY, M, N, B, N, r};
+    if ((rc = run_adapter_gemm(g, part, splits, stat, st))) return rc;
+    if ((rc = cuda_rc(launch_reduce_splits(part, splits, M, r, bn, s, 0, 1, dT_out, r, st)))) return rc;
+  }
+  // dB = dY^T T_save  (rows of D are output features, reduction over tokens)
+  {
+    const int splits = pick_splits(cdiv(N, 128), cdiv(M, 64));
+    AdapterGemm g{A_TMA_MN, B_TMA_MN, bn, N, r, M, dY, M, N, T_save, M, r};
+    if ((rc = run_adapter_gemm(g, part, splits, stat, st))) return rc;
+    if ((rc = cuda_rc(launch_reduce_splits(part, splits, N, r, bn, 1.0f, 0, 0, dB, r, st)))) return rc;
+  }
+  // dA^T = P(X)^T dT  (rows of D are adapter inputs, reduction over tokens), stored transposed
+  {
+    const int splits = pick_splits(cdiv(Ka, 128), cdiv(M, 64));
+    AdapterGemm g{A_TMA_MN, B_TMA_MN, bn, Ka, r, M, Xa, M, Ka, dT_out, M, r};
+    if ((rc = run_adapter_gemm(g, part, splits, stat, st))) return rc;
+    if ((rc = cuda_rc(launch_reduce_splits(part, splits, Ka, r, bn, 1.0f, 1, 0, dA, Ka, st)))) return rc;
+  }
+  return QLR_OK;
+}
+
+// ---- backward: input gradient --------------------------------------------------------------------
+
+size_t qlr_backward_dx_workspace_bytes(const qlr_qweight* w, int64_t M, int r, int pooled) {
+  if (check_qweight(w) || M <= 0 || check_rank(r)) return 0;
+  return pooled ? align256(size_t(r) * w->K * 2) : 0;
+}
+
+int qlr_backward_dx(const qlr_qweight* w, const uint16_t* dY, int64_t M, const uint16_t* A, const uint16_t* dT,
+                    int r, int pooled, int accumulate, uint16_t* dX, void* workspace, size_t workspace_bytes,
+                    int32_t* status, void* stream) {
+  int rc = check_gemm_weight(w);
+  if (rc) return rc;
+  if ((rc = check_rank(r))) return rc;
+  if (M < 0) return QLR_ERR_ARG;
+  if (M == 0) return QLR_OK;
+  if (!dY || !A || !dT || !dX) return QLR_ERR_ARG;
+  if (!aligned16(dY) || !aligned16(A) || !aligned16(dT) || !aligned16(dX)) return QLR_ERR_ALIGN;
+  if (pooled && w->fmt != QLR_FMT_INT4G) return QLR_ERR_UNSUPPORTED;
+  if (M == 0) return QLR_OK;
+  if (M > (int64_t(1) << 30)) return QLR_ERR_SHAPE;
+  const size_t need = qlr_backward_dx_workspace_bytes(w, M, r, pooled);
+  if (need && (!workspace || workspace_bytes < need)) return QLR_ERR_WORKSPACE;
+  if (need && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return QLR_ERR_ALIGN;
+  cudaStream_t st = as_stream(stream);
+  int32_t* stat = status_or_sink(status);
+  const int64_t N = w->N, K = w->K;
+  const uint16_t* At = A;
+  if (pooled) {
+    uint16_t* Aexp = static_cast<uint16_t*>(workspace);
+    if ((rc = cuda_rc(launch_expand_adapter(A, r, K, w->group, Aexp, st)))) return rc;
+    At = Aexp;
+  }
+  const int bn_tok = M >= 192 ? 256 : 64;
+  GemmMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  if ((rc = make_tmap(&maps.codes, w->codes, 1, N, K / 2, 64, 64, 0))) return rc;
+  if ((rc = make_tmap(&maps.b, dY, 2, M, N, bn_tok, 64, 128))) return rc;
+  if ((rc = make_tmap(&maps.a_tail, At, 2, r, K, 64, 64, 128))) return rc;
+  if ((rc = make_tmap(&maps.b_tail, dT, 2, M, r, bn_tok, 64, 128))) return rc;
+  maps.a = maps.a_tail;
+  GemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.Mm = static_cast<int>(K);
+  p.Nn = static_cast<int>(M);
+  p.n_main = static_cast<int>(cdiv(N, 64));
+  p.splits = 1;
+  p.n_tail = static_cast<int>(cdiv(r, 64));
+  p.r_tail = r;
+  p.m_tiles = static_cast<int>(cdiv(K, 128));
+  p.n_tiles = static_cast<int>(cdiv(M, bn_tok));
+  p.b_atom = 64;
+  p.out = dX;
+  p.ldo = K;
+  p.accumulate = accumulate ? 1 : 0;
+  p.dq = dq_params(w);
+  p.status = stat;
+  return cuda_rc(launch_gemm(A_DQ_MN, B_TMA_K, bn_tok, OUT_BF16_T, 1, p, maps, st));
+}
+
+// ---- SwiGLU ---------------------------------------------------------------------------------------
+
+int qlr_swiglu_forward(const uint16_t* G, const uint16_t* U, uint16_t* H, int64_t n, void* stream) {
+  if (n < 0 || (n && (!G || !U || !H))) return QLR_ERR_ARG;
+  if (n % 8) return QLR_ERR_SHAPE;
+  if (!aligned16(G) || !aligned16(U) || !aligned16(H)) return QLR_ERR_ALIGN;
+  return cuda_rc(launch_swiglu_fwd(G, U, H, n, as_stream(stream)));
+}
+
+int qlr_swiglu_backward(const uint16_t* dH, const uint16_t* G, const uint16_t* U, uint16_t* dG, uint16_t* dU,
+                        int64_t n, void* stream) {
+  if (n < 0 || (n && (!dH || !G || !U || !dG || !dU))) return QLR_ERR_ARG;
+  if (n % 8) return QLR_ERR_SHAPE;
+  if (!aligned16(dH) || !aligned16(G) || !aligned16(U) || !aligned16(dG) || !aligned16(dU)) return QLR_ERR_ALIGN;
+  return cuda_rc(launch_swiglu_bwd(dH, G, U, dG, dU, n, as_stream(stream)));
+}
+
+}  // extern "C"

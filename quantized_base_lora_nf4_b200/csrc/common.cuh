@@ -1,0 +1,43 @@
+// Shared declarations of the library's kernels and host helpers.
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/qlr.h"
+
+namespace qlr {
+
+struct Levels {
+  float v[16];
+};
+
+void nf_levels_f32(int k, float* out);
+Levels levels_for(int bits);
+
+// Status sink used when the caller passes no status word.
+int32_t* status_or_sink(int32_t* status);
+
+__device__ __forceinline__ void report(int32_t* status, int32_t code) { atomicExch(status, code); }
+
+// ---- launch wrappers (quantize.cu) ----
+cudaError_t launch_quantize_nfk(const float* W, int64_t n_elems, int bits, int block, int dq_block,
+                                const qlr_qweight* out, int32_t* status, cudaStream_t st);
+cudaError_t launch_quantize_int4g(const float* W, int64_t N, int64_t K, int group, const qlr_qweight* out,
+                                  int32_t* status, cudaStream_t st);
+cudaError_t launch_dequant(const qlr_qweight* w, uint16_t* out, cudaStream_t st);
+cudaError_t launch_merge(const qlr_qweight* w, const uint16_t* A, const uint16_t* B, int r, float s,
+                         cudaStream_t st);
+
+// ---- elementwise (elementwise.cu) ----
+cudaError_t launch_swiglu_fwd(const uint16_t* G, const uint16_t* U, uint16_t* H, int64_t n, cudaStream_t st);
+cudaError_t launch_swiglu_bwd(const uint16_t* dH, const uint16_t* G, const uint16_t* U, uint16_t* dG,
+                              uint16_t* dU, int64_t n, cudaStream_t st);
+cudaError_t launch_pool(const uint16_t* X, int64_t M, int64_t K, int L, uint16_t* Xp, cudaStream_t st);
+cudaError_t launch_expand_adapter(const uint16_t* A, int r, int64_t K, int L, uint16_t* Aexp, cudaStream_t st);
+cudaError_t launch_reduce_splits(const float* part, int splits, int64_t rows, int64_t cols, int64_t ld_part,
+                                 float scale, int transpose, int out_bf16, void* out, int64_t ld_out,
+                                 cudaStream_t st);
+
+int device_sm_count();
+
+}  // namespace qlr

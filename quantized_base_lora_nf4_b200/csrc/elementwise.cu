@@ -1,0 +1,161 @@
+// Memory-bound helpers: SwiGLU forward/backward, QA-LoRA group pooling of the adapter input,
+// the expanded adapter used by the input gradient, and the fixed-order reduction of split
+// partial sums.  Vectorised 16-byte loads/stores; grids sized in multiples of the SM count.
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace qlr {
+
+namespace {
+
+__device__ __forceinline__ float lo_f(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float hi_f(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+
+__device__ __forceinline__ float sigmoidf_(float g) { return 1.0f / (1.0f + expf(-g)); }
+
+__global__ void swiglu_fwd_kernel(const uint4* __restrict__ G, const uint4* __restrict__ U, uint4* __restrict__ H,
+                                  int64_t n8) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const uint4 g = G[i], u = U[i];
+    const uint32_t gv[4] = {g.x, g.y, g.z, g.w}, uv[4] = {u.x, u.y, u.z, u.w};
+    uint32_t hv[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float g0 = lo_f(gv[j]), g1 = hi_f(gv[j]);
+      const float h0 = g0 * sigmoidf_(g0) * lo_f(uv[j]);
+      const float h1 = g1 * sigmoidf_(g1) * hi_f(uv[j]);
+      hv[j] = pack_bf16x2_rn(h0, h1);
+    }
+    H[i] = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+  }
+}
+
+__global__ void swiglu_bwd_kernel(const uint4* __restrict__ dH, const uint4* __restrict__ G, const uint4* __restrict__ U,
+                                  uint4* __restrict__ dG, uint4* __restrict__ dU, int64_t n8) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const uint4 d = dH[i], g = G[i], u = U[i];
+    const uint32_t dv[4] = {d.x, d.y, d.z, d.w}, gv[4] = {g.x, g.y, g.z, g.w}, uv[4] = {u.x, u.y, u.z, u.w};
+    uint32_t og[4], ou[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float rg[2], ru[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const float dh = h ? hi_f(dv[j]) : lo_f(dv[j]);
+        const float gg = h ? hi_f(gv[j]) : lo_f(gv[j]);
+        const float uu = h ? hi_f(uv[j]) : lo_f(uv[j]);
+        const float sg = sigmoidf_(gg);
+        rg[h] = dh * uu * sg * (1.0f + gg * (1.0f - sg));
+        ru[h] = dh * gg * sg;
+      }
+      og[j] = pack_bf16x2_rn(rg[0], rg[1]);
+      ou[j] = pack_bf16x2_rn(ru[0], ru[1]);
+    }
+    dG[i] = make_uint4(og[0], og[1], og[2], og[3]);
+    dU[i] = make_uint4(ou[0], ou[1], ou[2], ou[3]);
+  }
+}
+
+// Xp[m, g] = bf16( (sum of X[m, gL .. gL+L-1]) / L ): one thread per output, fp32 sum.
+__global__ void pool_kernel(const uint16_t* __restrict__ X, int64_t M, int64_t K, int L, uint16_t* __restrict__ Xp) {
+  const int64_t G = K / L;
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= M * G) return;
+  const int64_t m = i / G, g = i % G;
+  const uint4* src = reinterpret_cast<const uint4*>(X + m * K + g * L);
+  float acc = 0.f;
+  for (int c = 0; c < L / 8; ++c) {
+    const uint4 v = src[c];
+    acc += lo_f(v.x) + hi_f(v.x) + lo_f(v.y) + hi_f(v.y) + lo_f(v.z) + hi_f(v.z) + lo_f(v.w) + hi_f(v.w);
+  }
+  const float mean = acc / static_cast<float>(L);
+  Xp[i] = static_cast<uint16_t>(pack_bf16x2_rn(mean, 0.f) & 0xFFFFu);
+}
+
+// Aexp[j, k] = bf16( A[j, k / L] / L ): the adapter seen by the un-pooled input.
+__global__ void expand_kernel(const uint16_t* __restrict__ A, int r, int64_t K, int L, uint16_t* __restrict__ Aexp) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= r * K) return;
+  const int64_t j = i / K, k = i % K;
+  const float v = bf16_bits_to_f32(A[j * (K / L) + k / L]) / static_cast<float>(L);
+  Aexp[i] = static_cast<uint16_t>(pack_bf16x2_rn(v, 0.f) & 0xFFFFu);
+}
+
+// out[row, col] (or out[col, row] when transposed) = scale * sum_s part[s, row, col], summed in
+// split order so the result does not depend on scheduling.
+__global__ void reduce_splits_kernel(const float* __restrict__ part, int splits, int64_t rows, int64_t cols,
+                                     int64_t ld_part, float scale, int transpose, int out_bf16, void* out,
+                                     int64_t ld_out) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= rows * cols) return;
+  int64_t row, col;
+  if (transpose) {  // consecutive threads walk rows so the transposed store is coalesced
+    col = i / rows;
+    row = i % rows;
+  } else {
+    row = i / cols;
+    col = i % cols;
+  }
+  float acc = 0.f;
+  for (int s = 0; s < splits; ++s) acc += part[(static_cast<int64_t>(s) * rows + row) * ld_part + col];
+  acc *= scale;
+  const int64_t o = transpose ? col * ld_out + row : row * ld_out + col;
+  if (out_bf16)
+    static_cast<uint16_t*>(out)[o] = static_cast<uint16_t>(pack_bf16x2_rn(acc, 0.f) & 0xFFFFu);
+  else
+    static_cast<float*>(out)[o] = acc;
+}
+
+unsigned grid_for(int64_t n_items, int threads) {
+  const int64_t want = (n_items + threads - 1) / threads;
+  const int64_t cap = static_cast<int64_t>(device_sm_count()) * 8;
+  return static_cast<unsigned>(want < 1 ? 1 : (want > cap ? cap : want));
+}
+
+}  // namespace
+
+cudaError_t launch_swiglu_fwd(const uint16_t* G, const uint16_t* U, uint16_t* H, int64_t n, cudaStream_t st) {
+  if (n == 0) return cudaSuccess;
+  const int64_t n8 = n / 8;
+  swiglu_fwd_kernel<<<grid_for(n8, 256), 256, 0, st>>>(reinterpret_cast<const uint4*>(G),
+                                                       reinterpret_cast<const uint4*>(U), reinterpret_cast<uint4*>(H), n8);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_swiglu_bwd(const uint16_t* dH, const uint16_t* G, const uint16_t* U, uint16_t* dG, uint16_t* dU,
+                              int64_t n, cudaStream_t st) {
+  if (n == 0) return cudaSuccess;
+  const int64_t n8 = n / 8;
+  swiglu_bwd_kernel<<<grid_for(n8, 256), 256, 0, st>>>(
+      reinterpret_cast<const uint4*>(dH), reinterpret_cast<const uint4*>(G), reinterpret_cast<const uint4*>(U),
+      reinterpret_cast<uint4*>(dG), reinterpret_cast<uint4*>(dU), n8);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pool(const uint16_t* X, int64_t M, int64_t K, int L, uint16_t* Xp, cudaStream_t st) {
+  const int64_t n = M * (K / L);
+  pool_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(X, M, K, L, Xp);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_expand_adapter(const uint16_t* A, int r, int64_t K, int L, uint16_t* Aexp, cudaStream_t st) {
+  const int64_t n = static_cast<int64_t>(r) * K;
+  expand_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(A, r, K, L, Aexp);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_reduce_splits(const float* part, int splits, int64_t rows, int64_t cols, int64_t ld_part,
+                                 float scale, int transpose, int out_bf16, void* out, int64_t ld_out,
+                                 cudaStream_t st) {
+  const int64_t n = rows * cols;
+  if (n == 0) return cudaSuccess;
+  reduce_splits_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(part, splits, rows, cols, ld_part,
+                                                                                 scale, transpose, out_bf16, out, ld_out);
+  return cudaGetLastError();
+}
+
+}  // namespace qlr

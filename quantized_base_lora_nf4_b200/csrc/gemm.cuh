@@ -1,0 +1,59 @@
+// Host-side description of one tcgen05 GEMM launch (see gemm.cu).
+#pragma once
+#include <cuda.h>
+#include <cuda_fp16.h>
+
+#include "common.cuh"
+
+namespace qlr {
+
+// How the MMA "A" operand (the 128 TMEM-lane side) reaches shared memory.
+enum ASrc : int {
+  A_TMA_K = 0,   // TMA tile of a [Mm, Kred] row-major matrix (K-major)
+  A_TMA_MN = 1,  // TMA tiles of a [Kred, Mm] row-major matrix (MN-major)
+  A_DQ_K = 2,    // dequantised from packed codes of W [Mm = N, Kred = K] (forward)
+  A_DQ_MN = 3    // dequantised from packed codes of W [Kred = N, Mm = K] (input gradient)
+};
+enum BSrc : int { B_TMA_K = 0, B_TMA_MN = 1 };
+enum OutMode : int { OUT_BF16_T = 0, OUT_F32_D = 1 };
+
+struct DqParams {
+  int fmt, bits, block, dq_block, group;
+  int64_t N, K;
+  const float* c1;
+  const uint8_t* c1_fp8;
+  const float* s2;
+  const __half* scale;
+  const __half* zero;
+  Levels lv;
+};
+
+// D[Mm, Nn] = sum_k A[Mm, k] B[k, Nn]  (+ a tail segment of extra reduction columns)
+struct GemmParams {
+  int Mm, Nn;            // extents of D (MMA M side = TMEM lanes, MMA N side = TMEM columns)
+  int n_main;            // 64-wide reduction steps of the main segment (all splits)
+  int splits;            // split-K factor of the main segment (partials go to out[split])
+  int n_tail;            // 64-wide reduction steps of the tail (only with splits == 1)
+  int r_tail;            // reduction extent of the tail (its last step may be partial)
+  int m_tiles, n_tiles;
+  int b_atom;            // MN-major B: elements per swizzle atom row (16, 32 or 64)
+  void* out;             // OUT_BF16_T: bf16 [Nn, ldo] receiving D^T; OUT_F32_D: fp32 [splits][m_tiles*128][ldo]
+  int64_t ldo;
+  int accumulate;        // OUT_BF16_T: add the previous contents of out
+  DqParams dq;
+  int32_t* status;
+};
+
+struct GemmMaps {
+  CUtensorMap a, b, a_tail, b_tail, codes;
+};
+
+// Launches the engine variant for (a_src, b_src, BN, out, tail_a_mn).
+cudaError_t launch_gemm(int a_src, int b_src, int bn, int out_mode, int tail_a_mn, const GemmParams& p,
+                        const GemmMaps& maps, cudaStream_t st);
+
+// Tensor-map helper: 2-D row-major [rows, cols] of elem_bytes elements, box [box_rows, box_cols].
+int make_tmap(CUtensorMap* m, const void* base, int elem_bytes, uint64_t rows, uint64_t cols, uint32_t box_rows,
+              uint32_t box_cols, int swizzle_bytes);
+
+}  // namespace qlr

@@ -1,0 +1,115 @@
+"""GPU parity of the forward / backward entry points against the fp64 oracle
+(relative Frobenius error <= 1e-2, the bound stated for the bf16 paths)."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import layer as OL
+from oracle import quantize as Q
+from synth import LinearSpec, linear_tensors, workload, random_matrix
+from tests.gpu_helpers import DEV, bf16_dev, f32_dev, host
+
+pytestmark = [pytest.mark.gpu, pytest.mark.filterwarnings("ignore::RuntimeWarning")]
+
+TOL = 1e-2
+
+
+def quantize_both(qlr, spec, W):
+    if spec.fmt == "int4g":
+        ref = Q.quantize_int4_group(W, spec.group)
+        return qlr.quantize_int4_group(f32_dev(W), spec.group), Q.dequant_int4_group(ref)
+    ref = Q.quantize_nfk(W, spec.bits, spec.block, spec.dq_block)
+    return qlr.quantize_nf4(f32_dev(W), spec.bits, spec.block, spec.dq_block), Q.dequant_nfk(ref)
+
+
+def run_and_check(qlr, spec, M, seed=0, rows=None, accumulate_check=False):
+    t = linear_tensors(spec, M, seed=seed)
+    q, Wdq = quantize_both(qlr, spec, t["W"])
+    X, A, B, dY = bf16_dev(t["X"]), bf16_dev(t["A"]), bf16_dev(t["B"]), bf16_dev(t["dY"])
+    st = qlr.new_status(DEV)
+    Y, T = qlr.forward(q, X, A, B, spec.s, pooled=spec.pooled, status=st)
+    dA, dB, dT = qlr.backward_lora(q, X, dY, T, B, spec.s, pooled=spec.pooled, status=st)
+    dX = qlr.backward_dx(q, dY, A, dT, pooled=spec.pooled, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    L = spec.group if spec.pooled else None
+    sel = slice(None) if rows is None else rows
+    Xs, dYs = t["X"][sel], t["dY"][sel]
+    f = OL.forward(Xs, Wdq, t["A"], t["B"], spec.s, L)
+    assert OL.rel_fro(host(Y)[sel], f["Y"]) <= TOL
+    assert OL.rel_fro(host(T)[sel], spec.s * f["T"]) <= TOL
+    bsel = OL.backward(dYs, Xs, Wdq, t["A"], t["B"], spec.s, L)
+    assert OL.rel_fro(host(dT)[sel], bsel["dT"]) <= TOL
+    assert OL.rel_fro(host(dX)[sel], bsel["dX"]) <= TOL
+    # adapter gradients reduce over every token: checked in full
+    full = bsel if rows is None else OL.backward(t["dY"], t["X"], Wdq, t["A"], t["B"], spec.s, L)
+    assert OL.rel_fro(host(dA), full["dA"]) <= TOL
+    assert OL.rel_fro(host(dB), full["dB"]) <= TOL
+    if accumulate_check:
+        dX2 = dX.clone()
+        qlr.backward_dx(q, dY, A, dT, pooled=spec.pooled, dX=dX2, accumulate=True)
+        torch.cuda.synchronize()
+        assert OL.rel_fro(host(dX2)[sel], 2 * bsel["dX"]) <= TOL
+    return {"Y": Y, "dX": dX, "dA": dA, "dB": dB}
+
+
+def test_tiny_layer(cuda_lib):
+    wl = workload("tiny")
+    run_and_check(cuda_lib, wl.linears[0], wl.M, accumulate_check=True)
+
+
+@pytest.mark.parametrize("M", [1, 40, 200, 333])
+@pytest.mark.parametrize("r", [8, 16, 32, 64])
+def test_ragged_nf4(cuda_lib, M, r):
+    spec = LinearSpec("w", 320, 384, "nfk", 4, 128, 0, r=r, s=0.5)
+    run_and_check(cuda_lib, spec, M, seed=M + r)
+
+
+@pytest.mark.parametrize("M", [64, 300])
+def test_ragged_int4_pooled(cuda_lib, M):
+    spec = LinearSpec("w", 264, 512, "int4g", group=32, r=16, s=1.0, pooled=True)
+    run_and_check(cuda_lib, spec, M, seed=7)
+
+
+def test_int4_unpooled_and_group64(cuda_lib):
+    run_and_check(cuda_lib, LinearSpec("w", 256, 512, "int4g", group=64, r=8, s=2.0, pooled=False), 96, seed=9)
+
+
+def test_qalora_full_size(cuda_lib):
+    wl = workload("qalora")
+    run_and_check(cuda_lib, wl.linears[0], wl.M)
+
+
+@pytest.mark.parametrize("which", [0, 2])
+def test_mlp7b_full_size_sampled_rows(cuda_lib, which):
+    wl = workload("mlp7b")
+    spec = wl.linears[which]
+    rows = np.sort(np.random.default_rng(which).choice(wl.M, 128, replace=False))
+    run_and_check(cuda_lib, spec, wl.M, rows=rows)
+
+
+def test_swiglu(cuda_lib):
+    qlr = cuda_lib
+    G = random_matrix(31, 0, "X", (64, 1024), 2.0, bf16=True)
+    U = random_matrix(31, 1, "X", (64, 1024), 1.0, bf16=True)
+    dH = random_matrix(31, 2, "X", (64, 1024), 1.0, bf16=True)
+    H = qlr.swiglu_forward(bf16_dev(G), bf16_dev(U))
+    dG, dU = qlr.swiglu_backward(bf16_dev(dH), bf16_dev(G), bf16_dev(U))
+    torch.cuda.synchronize()
+    assert OL.rel_fro(host(H), OL.swiglu_forward(G, U)) <= TOL
+    rg, ru = OL.swiglu_backward(dH, G, U)
+    assert OL.rel_fro(host(dG), rg) <= TOL
+    assert OL.rel_fro(host(dU), ru) <= TOL
+
+
+def test_zero_tokens(cuda_lib):
+    qlr = cuda_lib
+    spec = LinearSpec("w", 128, 256, "nfk", 4, 64, 256, r=8, s=1.0)
+    t = linear_tensors(spec, 4, seed=1)
+    q, _ = quantize_both(qlr, spec, t["W"])
+    X = torch.empty((0, 256), dtype=torch.bfloat16, device=DEV)
+    dY = torch.empty((0, 128), dtype=torch.bfloat16, device=DEV)
+    Y, T = qlr.forward(q, X, bf16_dev(t["A"]), bf16_dev(t["B"]), 1.0)
+    dA, dB, dT = qlr.backward_lora(q, X, dY, T, bf16_dev(t["B"]), 1.0)
+    torch.cuda.synchronize()
+    assert Y.shape == (0, 128) and float(dA.abs().sum()) == 0 and float(dB.abs().sum()) == 0

@@ -1,0 +1,106 @@
+"""GPU parity of the quantisers, dequantiser and merge: bit-exact against the oracle."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import quantize as Q
+from oracle.numerics import bf16_bits
+from synth import random_matrix, linear_tensors, workload
+from tests.gpu_helpers import DEV, bf16_dev, f32_dev, host, host_bytes
+
+pytestmark = [pytest.mark.gpu, pytest.mark.filterwarnings("ignore::RuntimeWarning")]
+
+
+def _compare_nf(q_gpu, q_ref, rows=None):
+    n_codes_bytes = q_ref["packed"].size
+    np.testing.assert_array_equal(host_bytes(q_gpu.codes)[:n_codes_bytes], q_ref["packed"])
+    if q_ref["dq_block"]:
+        nb = q_ref["c1_fp8"].size
+        np.testing.assert_array_equal(host_bytes(q_gpu.c1_fp8)[:nb], q_ref["c1_fp8"])
+        np.testing.assert_array_equal(host(q_gpu.s2)[: q_ref["s2"].size].view(np.uint32), q_ref["s2"].view(np.uint32))
+    else:
+        np.testing.assert_array_equal(host(q_gpu.c1)[: q_ref["c1"].size].view(np.uint32), q_ref["c1"].view(np.uint32))
+
+
+@pytest.mark.parametrize("bits,block,dq", [(4, 64, 256), (4, 128, 256), (4, 64, 0), (3, 64, 256), (3, 128, 0),
+                                           (2, 64, 256), (2, 128, 256)])
+@pytest.mark.parametrize("shape", [(256, 256), (96, 640), (40, 128 * 70)])
+def test_nf_quantize_bit_exact(cuda_lib, bits, block, dq, shape):
+    qlr = cuda_lib
+    W = random_matrix(21, bits * 1000 + block + dq, "W", shape, 0.02)
+    W[3, :block] = 0.0                      # a zero block
+    W[5, 7] = 0.5                           # an outlier
+    ref = Q.quantize_nfk(W, bits, block, dq)
+    q = qlr.quantize_nf4(f32_dev(W), bits, block, dq)
+    torch.cuda.synchronize()
+    _compare_nf(q, ref)
+    Wd = qlr.dequant(q)
+    np.testing.assert_array_equal(bf16_bits(host(Wd)), bf16_bits(Q.dequant_nfk(ref)))
+
+
+def test_nf_quantize_full_size_decode_projection(cuda_lib):
+    """28672 x 8192 (the 70B-like decode projection): codes, constants and dequant checked on
+    whole double-quantisation groups of sampled rows (2 rows per group at K = 8192)."""
+    qlr = cuda_lib
+    spec = workload("decode70b").linears[0]
+    W = random_matrix(0, 0, "W", (spec.N, spec.K), spec.sigma_w)
+    q = qlr.quantize_nf4(f32_dev(W), 4, 64, 256)
+    Wd = qlr.dequant(q)
+    torch.cuda.synchronize()
+    codes = host_bytes(q.codes)
+    c8 = host_bytes(q.c1_fp8)
+    s2 = host(q.s2)
+    wd = Wd.view(torch.int16)
+    rng = np.random.default_rng(5)
+    for r0 in sorted(rng.choice(spec.N // 2, 24, replace=False) * 2):
+        sub = W[r0:r0 + 2]
+        ref = Q.quantize_nfk(sub, 4, 64, 256)
+        b0 = r0 * spec.K // 2
+        np.testing.assert_array_equal(codes[b0:b0 + ref["packed"].size], ref["packed"])
+        blk0 = r0 * spec.K // 64
+        np.testing.assert_array_equal(c8[blk0:blk0 + ref["c1_fp8"].size], ref["c1_fp8"])
+        assert s2[blk0 // 256] == ref["s2"][0]
+        got = wd[r0:r0 + 2].cpu().numpy().view(np.uint16)
+        np.testing.assert_array_equal(got, bf16_bits(Q.dequant_nfk(ref)))
+
+
+def test_nf_quantize_reports_nonfinite(cuda_lib):
+    qlr = cuda_lib
+    W = random_matrix(22, 0, "W", (64, 256), 0.02)
+    W[10, 10] = np.inf
+    st = qlr.new_status(DEV)
+    qlr.quantize_nf4(f32_dev(W), 4, 64, 256, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == -5
+
+
+@pytest.mark.parametrize("group", [32, 64, 128])
+@pytest.mark.parametrize("shape", [(64, 256), (4096, 4096)])
+def test_int4_group_quantize_bit_exact(cuda_lib, group, shape):
+    qlr = cuda_lib
+    W = random_matrix(23, group, "W", shape, 0.02)
+    W[0, :group] = 0.0
+    W[1, group:2 * group] = np.abs(W[1, group:2 * group])
+    ref = Q.quantize_int4_group(W, group)
+    q = qlr.quantize_int4_group(f32_dev(W), group)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(host_bytes(q.codes), ref["packed"])
+    np.testing.assert_array_equal(q.scale.cpu().numpy().view(np.uint16), ref["scale"].view(np.uint16))
+    np.testing.assert_array_equal(q.zero.cpu().numpy().view(np.uint16), ref["zero"].view(np.uint16))
+    Wd = qlr.dequant(q)
+    np.testing.assert_array_equal(bf16_bits(host(Wd)), bf16_bits(Q.dequant_int4_group(ref)))
+
+
+def test_qalora_merge_bit_exact_and_lossless(cuda_lib):
+    qlr = cuda_lib
+    wl = workload("qalora")
+    spec = wl.linears[0]
+    t = linear_tensors(spec, 64, seed=0)
+    ref = Q.quantize_int4_group(t["W"], spec.group)
+    q = qlr.quantize_int4_group(f32_dev(t["W"]), spec.group)
+    qlr.qalora_merge(q, bf16_dev(t["A"]), bf16_dev(t["B"]), spec.s)
+    torch.cuda.synchronize()
+    zp = Q.qalora_merge(ref, t["A"], t["B"], spec.s)
+    np.testing.assert_array_equal(q.zero.cpu().numpy().view(np.uint16), zp.view(np.uint16))
+    Wd = qlr.dequant(q)
+    np.testing.assert_array_equal(bf16_bits(host(Wd)), bf16_bits(Q.dequant_int4_group(ref, zero=zp)))
