@@ -32,7 +32,7 @@ QA-LoRA (abstract: group-wise INT4 quantisation, an adapter with fewer degrees o
 freedom, and a merge "without loss of accuracy") is read as:
   * per (row o, group g of L consecutive inputs): lo = min(0, min w), hi = max(0, max w),
     scale = fp16_rn(fp32(fp32(hi - lo) / 15)), z = clamp(rne(fp32(-lo / scale)), 0, 15)
-    stored as fp16, code = clamp(rne(fp32(fp32(w / scale) + z)), 0, 15); a group whose
+    stored as fp16 (an integer, so a zero is +0), code = clamp(rne(fp32(fp32(w / scale) + z)), 0, 15); a group whose
     fp16 scale is 0 has z = 0 and codes 0;
   * dequant = bf16_rn(fp32(fp32(code - z) * scale));
   * merge: the pooled adapter adds (s / L) (B A)[o, g] to every weight of group g of
@@ -200,7 +200,8 @@ def quantize_int4_group(W: np.ndarray, group: int = 32) -> Dict[str, np.ndarray]
     ok = scale > 0
     with np.errstate(divide="ignore", invalid="ignore"):
         zf = np.rint((-lo / scale).astype(np.float32))
-        z = np.where(ok, np.clip(zf, 0, 15), 0).astype(np.float32)
+        # the zero point is an integer in [0, 15]; adding +0.0 maps a -0.0 (from lo == 0) to +0.0
+        z = (np.where(ok, np.clip(zf, 0, 15), 0).astype(np.float32) + np.float32(0.0)).astype(np.float32)
         t = ((g / scale[..., None]).astype(np.float32) + z[..., None]).astype(np.float32)
         code = np.where(ok[..., None], np.clip(np.rint(t), 0, 15), 0).astype(np.uint8)
     codes = code.reshape(N, K)

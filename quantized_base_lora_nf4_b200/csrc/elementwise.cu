@@ -87,9 +87,9 @@ __global__ void expand_kernel(const uint16_t* __restrict__ A, int r, int64_t K, 
 
 // out[row, col] (or out[col, row] when transposed) = scale * sum_s part[s, row, col], summed in
 // split order so the result does not depend on scheduling.
-__global__ void reduce_splits_kernel(const float* __restrict__ part, int splits, int64_t rows, int64_t cols,
-                                     int64_t ld_part, float scale, int transpose, int out_bf16, void* out,
-                                     int64_t ld_out) {
+__global__ void reduce_splits_kernel(const float* __restrict__ part, int splits, int64_t rows, int64_t split_rows,
+                                     int64_t cols, int64_t ld_part, float scale, int transpose, int out_bf16,
+                                     void* out, int64_t ld_out) {
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i >= rows * cols) return;
   int64_t row, col;
@@ -101,7 +101,7 @@ __global__ void reduce_splits_kernel(const float* __restrict__ part, int splits,
     col = i % cols;
   }
   float acc = 0.f;
-  for (int s = 0; s < splits; ++s) acc += part[(static_cast<int64_t>(s) * rows + row) * ld_part + col];
+  for (int s = 0; s < splits; ++s) acc += part[(static_cast<int64_t>(s) * split_rows + row) * ld_part + col];
   acc *= scale;
   const int64_t o = transpose ? col * ld_out + row : row * ld_out + col;
   if (out_bf16)
@@ -153,8 +153,9 @@ cudaError_t launch_reduce_splits(const float* part, int splits, int64_t rows, in
                                  cudaStream_t st) {
   const int64_t n = rows * cols;
   if (n == 0) return cudaSuccess;
-  reduce_splits_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(part, splits, rows, cols, ld_part,
-                                                                                 scale, transpose, out_bf16, out, ld_out);
+  const int64_t split_rows = (rows + 127) / 128 * 128;  // each split holds whole 128-row tiles
+  reduce_splits_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(
+      part, splits, rows, split_rows, cols, ld_part, scale, transpose, out_bf16, out, ld_out);
   return cudaGetLastError();
 }
 

@@ -163,7 +163,7 @@ __global__ void __launch_bounds__(256) quantize_int4g_kernel(const float* __rest
   const __half sc16 = __float2half_rn(__fdiv_rn(__fsub_rn(hi, lo), 15.0f));
   const float sc = __half2float(sc16);
   float z = 0.f;
-  if (sc > 0.f) z = fminf(fmaxf(rintf(__fdiv_rn(-lo, sc)), 0.f), 15.f);
+  if (sc > 0.f) z = __fadd_rn(fminf(fmaxf(rintf(__fdiv_rn(-lo, sc)), 0.f), 15.f), 0.0f);  // +0, never -0
 #pragma unroll
   for (int e = 0; e < E; ++e) {
     int c = 0;

@@ -188,6 +188,7 @@ def test_int4_group_properties():
     z = q["zero"].astype(np.float32)
     assert sc[0, 0] == 0 and z[0, 0] == 0 and np.all(q["codes"].reshape(16, 256)[0, :32] == 0)
     assert z[1, 1] == 0
+    assert q["zero"].view(np.uint16)[1, 1] == 0          # an integer zero point: +0, not -0
     assert np.all((z >= 0) & (z <= 15) & (z == np.rint(z)))
     codes = q["codes"].reshape(16, 8, 32).astype(np.float64)
     assert codes.max() <= 15
