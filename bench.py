@@ -1,0 +1,439 @@
+#!/usr/bin/env python
+"""Throughput of the quantised-base + LoRA linear on B200: fwd+bwd tokens/s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload qalora|tiny|mlp7b] [--impl ours|reference]
+
+One step = forward (adapter down-projection T = s P(X) A^T, fused dequant + tcgen05 base GEMM with the
+adapter term folded in) + backward (dT, dA, dB; fused input gradient) of every linear of the workload,
+over one batch of synthetic tokens already resident in HBM.  The default workload is the QA-LoRA layer:
+INT4 group-32 weight 4096x4096, pooled adapter r=16, 2048 tokens.  Rank 0 prints one JSON line.
+
+Under torchrun (N > 1) every rank runs the same layer on its own tokens (data parallel, weights
+replicated) and the adapter gradients are summed over ranks with NCCL each step; the time is the
+maximum over ranks.  `--impl reference` times the CPU oracle (test infrastructure) on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "fwd+bwd tokens/s through quant-base+LoRA linears; % of TC peak / HBM GB/s"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="qalora", choices=["qalora", "tiny", "mlp7b"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------------------------------ accounting
+def flops_per_token(spec) -> float:
+    """4NK (forward base GEMM + input gradient; the base weight gets no gradient) plus the six rank-r
+    adapter products (T, T B^T, dT, dT A, dA, dB), with K/L adapter inputs for the pooled adapter."""
+    ka = spec.k_adapter
+    return 4.0 * spec.N * spec.K + 2.0 * spec.r * (3 * spec.N + 3 * ka)
+
+
+def workload_desc(wl):
+    spec = wl.linears[0]
+    if wl.name == "qalora":
+        return (f"qalora: INT4 group-{spec.group} base {spec.N}x{spec.K}, pooled adapter r={spec.r} "
+                f"(s={spec.s}), {wl.M} tokens, fwd+bwd")
+    if wl.name == "mlp7b":
+        return f"mlp7b: LLaMA-7B MLP (gate/up 11008x4096, down 4096x11008) NF4+DQ, r=64, SwiGLU, {wl.M} tokens, fwd+bwd"
+    return f"tiny: NF4+DQ 256x256, r=8, {wl.M} tokens, fwd+bwd"
+
+
+def profile_traffic(kernel_file: str):
+    """Per-launch DRAM bytes of the fused forward kernel from the committed ncu summary, if it was taken
+    on the current source of the GEMM engine (else None)."""
+    p = os.path.join(ROOT, "profiles", kernel_file)
+    if not os.path.exists(p):
+        return None
+    text = open(p).read()
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    h = re.search(r"gemm_source_sha256:\s*([0-9a-f]{64})", text)
+    if not m or not h:
+        return None
+    src = os.path.join(ROOT, "quantized_base_lora_nf4_b200", "csrc", "gemm.cu")
+    if hashlib.sha256(open(src, "rb").read()).hexdigest() != h.group(1):
+        return None
+    return float(m.group(1))
+
+
+# ------------------------------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r for r in csv.reader(io.StringIO(out)) if len(r) >= 9]
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].strip().lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------------------------------ GPU arm
+class Layer:
+    """Device-resident state of one quantised linear (weights, adapters, activations, gradients)."""
+
+    def __init__(self, qlr, spec, M, seed, rank, dev, X=None):
+        import numpy as np
+        import torch
+        from synth import linear_tensors, normal
+
+        self.spec = spec
+        t = linear_tensors(spec, M, seed=seed, matrix_index=0, with_x=X is None, with_dy=False)
+        bf = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev).to(torch.bfloat16).contiguous()  # noqa
+        W = torch.from_numpy(t["W"]).to(dev)
+        if spec.fmt == "int4g":
+            self.q = qlr.quantize_int4_group(W, spec.group)
+        else:
+            self.q = qlr.quantize_nf4(W, spec.bits, spec.block, spec.dq_block)
+        del W
+        self.A, self.B = bf(t["A"]), bf(t["B"])
+        self.X = bf(t["X"]) if X is None else X
+        self.dY = bf(normal(seed + 1000 * rank, 0, "dY", (M, spec.N), 1.0, bf16=True))
+        r = spec.r
+        self.T = torch.empty((M, r), dtype=torch.bfloat16, device=dev)
+        self.Y = torch.empty((M, spec.N), dtype=torch.bfloat16, device=dev)
+        self.dT = torch.empty((M, r), dtype=torch.bfloat16, device=dev)
+        self.dA = torch.empty((r, spec.k_adapter), dtype=torch.float32, device=dev)
+        self.dB = torch.empty((spec.N, r), dtype=torch.float32, device=dev)
+        self.dX = torch.empty((M, spec.K), dtype=torch.bfloat16, device=dev)
+        self.ws = qlr.Workspace(dev)
+        self.ws_b = qlr.Workspace(dev)
+        self.ws_x = qlr.Workspace(dev)
+
+
+def run_ours(args, rank, world, dev):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    from quantized_base_lora_nf4_b200 import qlr
+    from synth import workload, normal
+
+    qlr.lib()
+    wl = workload(args.workload, args.seed)
+    M = wl.M
+    seed = args.seed
+    if wl.kind == "mlp":
+        gate_s, up_s, down_s = wl.linears
+        X = normal(seed + 1000 * rank, 0, "X", (M, gate_s.K), 1.0, bf16=True)
+        Xd = torch.from_numpy(X).to(dev).to(torch.bfloat16).contiguous()
+        gate = Layer(qlr, gate_s, M, seed, rank, dev, X=Xd)
+        up = Layer(qlr, up_s, M, seed + 1, rank, dev, X=Xd)
+        Hm = torch.empty((M, gate_s.N), dtype=torch.bfloat16, device=dev)
+        down = Layer(qlr, down_s, M, seed + 2, rank, dev, X=Hm)
+        layers = [gate, up, down]
+        dHm = torch.empty_like(Hm)
+        dG = torch.empty_like(Hm)
+        dU = torch.empty_like(Hm)
+    else:
+        layers = [Layer(qlr, wl.linears[0], M, seed, rank, dev)]
+    fwd_ev = []
+
+    def fwd_base(L, record):
+        if record:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            qlr.forward_base(L.q, L.X, L.B, L.T, Y=L.Y)
+            e1.record()
+            fwd_ev.append((e0, e1))
+        else:
+            qlr.forward_base(L.q, L.X, L.B, L.T, Y=L.Y)
+
+    def lin_bwd(L, dY, dX, accumulate=False):
+        s, pooled = L.spec.s, L.spec.pooled
+        qlr.backward_lora(L.q, L.X, dY, L.T, L.B, s, pooled=pooled, dA=L.dA, dB=L.dB, dT=L.dT, ws=L.ws_b)
+        qlr.backward_dx(L.q, dY, L.A, L.dT, pooled=pooled, dX=dX, accumulate=accumulate, ws=L.ws_x)
+
+    def step(record=False):
+        if wl.kind == "mlp":
+            gate, up, down = layers
+            qlr.lora_down(gate.q, gate.X, gate.A, gate.spec.s, T_save=gate.T, ws=gate.ws)
+            qlr.lora_down(up.q, up.X, up.A, up.spec.s, T_save=up.T, ws=up.ws)
+            fwd_base(gate, record)
+            fwd_base(up, record)
+            qlr.swiglu_forward(gate.Y, up.Y, H=Hm)
+            qlr.lora_down(down.q, Hm, down.A, down.spec.s, T_save=down.T, ws=down.ws)
+            fwd_base(down, record)
+            lin_bwd(down, down.dY, dHm)
+            qlr.swiglu_backward(dHm, gate.Y, up.Y, dG=dG, dU=dU)
+            lin_bwd(gate, dG, gate.dX)
+            lin_bwd(up, dU, gate.dX, accumulate=True)
+        else:
+            L = layers[0]
+            qlr.lora_down(L.q, L.X, L.A, L.spec.s, pooled=L.spec.pooled, T_save=L.T, ws=L.ws)
+            fwd_base(L, record)
+            lin_bwd(L, L.dY, L.dX)
+        if world > 1:
+            for L in layers:
+                dist.all_reduce(L.dA)
+                dist.all_reduce(L.dB)
+
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)  # > 126 MB L2
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    launches0 = qlr.launch_count()
+    evs = []
+    for _ in range(args.steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        step(record=True)
+        e1.record()
+        evs.append((e0, e1))
+    torch.cuda.synchronize()
+    launches = qlr.launch_count() - launches0
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clk = clocks.stop() if clocks else None
+    ms_steps = [a.elapsed_time(b) for a, b in evs]
+    ms_total = sum(ms_steps)
+    fwd_ms = [a.elapsed_time(b) for a, b in fwd_ev]
+    if world > 1:
+        t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_per_step = ms_total / args.steps
+
+    # end to end: inputs from pinned host memory, gradients read back, every step
+    h_in = [(L.X, torch.empty(L.X.shape, dtype=L.X.dtype, pin_memory=True)) for L in layers if L is layers[0]]
+    h_in += [(L.dY, torch.empty(L.dY.shape, dtype=L.dY.dtype, pin_memory=True)) for L in layers[-1:]]
+    if wl.kind != "mlp":
+        h_in = [(layers[0].X, torch.empty(layers[0].X.shape, dtype=torch.bfloat16, pin_memory=True)),
+                (layers[0].dY, torch.empty(layers[0].dY.shape, dtype=torch.bfloat16, pin_memory=True))]
+    for d, h in h_in:
+        h.copy_(d)
+    h_out = [(L.dA, torch.empty(L.dA.shape, dtype=torch.float32, pin_memory=True)) for L in layers]
+    h_out += [(L.dB, torch.empty(L.dB.shape, dtype=torch.float32, pin_memory=True)) for L in layers]
+    h2d = sum(h.numel() * h.element_size() for _, h in h_in)
+    d2h = sum(h.numel() * h.element_size() for _, h in h_out)
+    e2e_steps = max(3, args.steps // 2)
+    for _ in range(2):
+        for d, h in h_in:
+            d.copy_(h, non_blocking=True)
+        step()
+        for d, h in h_out:
+            h.copy_(d, non_blocking=True)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e_s, e_e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_s.record()
+    for _ in range(e2e_steps):
+        for d, h in h_in:
+            d.copy_(h, non_blocking=True)
+        step()
+        for d, h in h_out:
+            h.copy_(d, non_blocking=True)
+    e_e.record()
+    torch.cuda.synchronize()
+    e2e_ms = e_s.elapsed_time(e_e)
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    if world > 1:
+        dist.barrier()
+    return {"wl": wl, "M": M, "ms_per_step": ms_per_step, "ms_steps": ms_steps, "fwd_ms": fwd_ms,
+            "launches": launches, "clocks": clk, "e2e_ms_per_step": e2e_ms / e2e_steps, "h2d": h2d, "d2h": d2h,
+            "layers": layers}
+
+
+# ------------------------------------------------------------------------------------------ CPU oracle arm
+def oracle_tokens_per_s(wl, seed, budget_s=12.0):
+    """Times the oracle (fp64 numpy, as it stands) on a bounded sample: `m` tokens of the workload
+    through forward + backward of every linear; the dequantised weights are prepared untimed."""
+    import numpy as np
+    from oracle import layer as OL
+    from oracle import quantize as Q
+    from synth import linear_tensors
+
+    m = {"tiny": 16, "qalora": 512, "mlp7b": 32}[wl.name]
+    mats = []
+    for i, spec in enumerate(wl.linears):
+        t = linear_tensors(spec, m, seed=seed + i)
+        if spec.fmt == "int4g":
+            Wdq = Q.dequant_int4_group(Q.quantize_int4_group(t["W"], spec.group))
+        else:
+            Wdq = Q.dequant_nfk(Q.quantize_nfk(t["W"], spec.bits, spec.block, spec.dq_block))
+        mats.append((spec, t, Wdq))
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        if wl.kind == "mlp":
+            (gs, gt, gW), (us, ut, uW), (ds, dt, dW) = mats
+            X = gt["X"]
+            G = OL.forward(X, gW, gt["A"], gt["B"], gs.s)["Y"]
+            U = OL.forward(X, uW, ut["A"], ut["B"], us.s)["Y"]
+            Hm = OL.swiglu_forward(G, U)
+            OL.forward(Hm, dW, dt["A"], dt["B"], ds.s)
+            bd = OL.backward(dt["dY"], Hm, dW, dt["A"], dt["B"], ds.s)
+            dG, dU = OL.swiglu_backward(bd["dX"], G, U)
+            OL.backward(dG, X, gW, gt["A"], gt["B"], gs.s)
+            OL.backward(dU, X, uW, ut["A"], ut["B"], us.s)
+        else:
+            spec, t, Wdq = mats[0]
+            L = spec.group if spec.pooled else None
+            OL.forward(t["X"], Wdq, t["A"], t["B"], spec.s, L)
+            OL.backward(t["dY"], t["X"], Wdq, t["A"], t["B"], spec.s, L)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or reps >= 2000:
+            break
+    cores = len(os.sched_getaffinity(0))
+    return {"value": reps * m / el, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{reps} x {m} tokens of the {wl.name} workload, fwd+bwd in fp64 numpy "
+                      f"({el:.1f} s; dequantised weights prepared untimed)"}
+
+
+# ------------------------------------------------------------------------------------------ main
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    from synth import workload
+
+    wl = workload(args.workload, args.seed)
+    fl_tok = sum(flops_per_token(s) for s in wl.linears)
+    cfg = {"workload": workload_desc(wl), "tokens_per_rank": wl.M,
+           "linears": [{"name": s.name, "N": s.N, "K": s.K, "r": s.r, "format": s.fmt,
+                        "bits": s.bits if s.fmt == "nfk" else 4,
+                        "block": s.block if s.fmt == "nfk" else s.group} for s in wl.linears],
+           "l2": "256 MiB buffer written between timed steps (L2 flushed)", "seed": args.seed,
+           "parallelism": f"dp{world}"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        cb = oracle_tokens_per_s(wl, args.seed)
+        line = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "tokens/s", "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * wl.M / cb["value"],
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "config": cfg, "cpu_baseline": cb,
+                "e2e": {"value": cb["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return 0
+
+    import torch
+    if not torch.cuda.is_available():
+        print(json.dumps({"error": "no CUDA device"}))
+        return 1
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    res = run_ours(args, rank, world, dev)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    peaks, peak_kind = load_peaks()
+    M = res["M"]
+    ms = res["ms_per_step"]
+    tokens_s = world * M / (ms / 1e3)
+    tflops = world * fl_tok * M / (ms / 1e3) / 1e12
+    # dominant kernel: the fused dequant + tcgen05 forward GEMM of the first linear
+    spec0 = wl.linears[0]
+    fwd_ms = res["fwd_ms"]
+    n_fwd = len(wl.linears)
+    per_layer = [statistics.mean(fwd_ms[i::n_fwd]) for i in range(n_fwd)]
+    fwd_launch_ms = per_layer[0]
+    fwd_flops = 2.0 * M * spec0.N * spec0.K + 2.0 * M * spec0.N * spec0.r
+    achieved = fwd_flops / (fwd_launch_ms / 1e3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    traffic = profile_traffic(f"fused_forward_{wl.name}.md")
+    line = {
+        "metric": METRIC, "value": tokens_s, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded numpy, shapes and distributions of the workload)",
+        "config": cfg,
+        "tflops": tflops, "tc_frac_of_measured_burst": tflops / peak,
+        "tc_frac_of_measured_sustained": tflops / float(peaks.get("bf16_tflops_sustained", peak)),
+        "roofline": {"bound": "tensor", "kernel": "gemm_kernel<A_DQ_K> (fused dequant + tcgen05 forward)",
+                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "peak_kind": f"{peak_kind} bf16 burst", "traffic": traffic,
+                     "flops_per_launch": fwd_flops, "launch_ms": fwd_launch_ms},
+        "gpu_launches": res["launches"],
+        "clocks": res["clocks"],
+        "e2e": {"value": world * M / (res["e2e_ms_per_step"] / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"],
+                "ms_per_step": res["e2e_ms_per_step"]},
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = oracle_tokens_per_s(wl, args.seed)
+    print(json.dumps(line))
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -175,6 +175,19 @@ QLR_API int qlr_forward(const qlr_qweight* w, const uint16_t* X, int64_t M, cons
                 float s, int pooled, uint16_t* Y, uint16_t* T_save, void* workspace, size_t workspace_bytes,
                 int32_t* status, void* stream);
 
+/* The two stages of qlr_forward, callable separately (same arguments and buffers):
+ *   qlr_lora_down     T_save = bf16(s * P(X) A^T)      (split-K tensor-core GEMM + fixed-order sum)
+ *   qlr_forward_base  Y = bf16(X dequant(W)^T + T_save B^T)   (the fused dequant + tcgen05 kernel)
+ * qlr_lora_down uses the workspace of qlr_forward_workspace_bytes; qlr_forward_base needs none. */
+QLR_API int qlr_lora_down(const qlr_qweight* w, const uint16_t* X, int64_t M, const uint16_t* A, int r, float s,
+                          int pooled, uint16_t* T_save, void* workspace, size_t workspace_bytes, int32_t* status,
+                          void* stream);
+QLR_API int qlr_forward_base(const qlr_qweight* w, const uint16_t* X, int64_t M, const uint16_t* B, int r,
+                             const uint16_t* T_save, uint16_t* Y, int32_t* status, void* stream);
+
+/* Number of kernels this library has launched in this process (all devices, all streams). */
+QLR_API uint64_t qlr_launch_count(void);
+
 /*
  * Adapter gradients (QLoRA explainer, "Background: how LoRA works" and "The QLoRA recipe":
  * gradients reach only A and B).  With T_save from qlr_forward:

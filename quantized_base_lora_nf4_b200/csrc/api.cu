@@ -3,6 +3,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstring>
 #include <mutex>
 
@@ -12,6 +13,9 @@
 namespace qlr {
 
 __device__ int32_t g_status_sink;
+
+static std::atomic<uint64_t> g_launches{0};
+void count_launch(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed); }
 
 int32_t* status_or_sink(int32_t* status) {
   if (status) return status;
@@ -192,6 +196,8 @@ const char* qlr_error_string(int code) {
 
 int qlr_version(void) { return 100; }
 
+uint64_t qlr_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
 int qlr_device_sm_count(void) { return device_sm_count(); }
 
 int qlr_nf_levels(int bits, float* out) {
@@ -288,28 +294,25 @@ size_t qlr_forward_workspace_bytes(const qlr_qweight* w, int64_t M, int r, int p
   return bytes;
 }
 
-int qlr_forward(const qlr_qweight* w, const uint16_t* X, int64_t M, const uint16_t* A, const uint16_t* B, int r,
-                float s, int pooled, uint16_t* Y, uint16_t* T_save, void* workspace, size_t workspace_bytes,
-                int32_t* status, void* stream) {
+int qlr_lora_down(const qlr_qweight* w, const uint16_t* X, int64_t M, const uint16_t* A, int r, float s, int pooled,
+                  uint16_t* T_save, void* workspace, size_t workspace_bytes, int32_t* status, void* stream) {
   int rc = check_gemm_weight(w);
   if (rc) return rc;
   if ((rc = check_rank(r))) return rc;
   if (M < 0) return QLR_ERR_ARG;
   if (M == 0) return QLR_OK;
-  if (!X || !A || !B || !Y || !T_save) return QLR_ERR_ARG;
-  if (!aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(Y) || !aligned16(T_save)) return QLR_ERR_ALIGN;
+  if (!X || !A || !T_save) return QLR_ERR_ARG;
+  if (!aligned16(X) || !aligned16(A) || !aligned16(T_save)) return QLR_ERR_ALIGN;
   if (pooled && w->fmt != QLR_FMT_INT4G) return QLR_ERR_UNSUPPORTED;
   if (pooled && (w->K / w->group) % 8) return QLR_ERR_SHAPE;
-  if (M == 0) return QLR_OK;
   if (M > (int64_t(1) << 30)) return QLR_ERR_SHAPE;
   const size_t need = qlr_forward_workspace_bytes(w, M, r, pooled);
   if (!workspace || workspace_bytes < need) return QLR_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return QLR_ERR_ALIGN;
   cudaStream_t st = as_stream(stream);
   int32_t* stat = status_or_sink(status);
-  const int64_t N = w->N, K = w->K;
+  const int64_t K = w->K;
   const int64_t Ka = pooled ? K / w->group : K;
-
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const uint16_t* Xa = X;
   if (pooled) {
@@ -324,8 +327,22 @@ int qlr_forward(const qlr_qweight* w, const uint16_t* X, int64_t M, const uint16
   float* part = reinterpret_cast<float*>(ws);
   AdapterGemm g{A_TMA_K, B_TMA_K, bn, M, r, Ka, Xa, M, Ka, A, r, Ka};
   if ((rc = run_adapter_gemm(g, part, splits, stat, st))) return rc;
-  if ((rc = cuda_rc(launch_reduce_splits(part, splits, M, r, bn, s, 0, 1, T_save, r, st)))) return rc;
+  return cuda_rc(launch_reduce_splits(part, splits, M, r, bn, s, 0, 1, T_save, r, st));
+}
 
+int qlr_forward_base(const qlr_qweight* w, const uint16_t* X, int64_t M, const uint16_t* B, int r,
+                     const uint16_t* T_save, uint16_t* Y, int32_t* status, void* stream) {
+  int rc = check_gemm_weight(w);
+  if (rc) return rc;
+  if ((rc = check_rank(r))) return rc;
+  if (M < 0) return QLR_ERR_ARG;
+  if (M == 0) return QLR_OK;
+  if (!X || !B || !Y || !T_save) return QLR_ERR_ARG;
+  if (!aligned16(X) || !aligned16(B) || !aligned16(Y) || !aligned16(T_save)) return QLR_ERR_ALIGN;
+  if (M > (int64_t(1) << 30)) return QLR_ERR_SHAPE;
+  cudaStream_t st = as_stream(stream);
+  int32_t* stat = status_or_sink(status);
+  const int64_t N = w->N, K = w->K;
   // Y = X dequant(W)^T + T_save B^T: fused dequant + tcgen05, computed as Y^T tiles (W rows on TMEM lanes)
   const int bn_tok = M >= 192 ? 256 : 64;
   GemmMaps maps;
@@ -352,6 +369,19 @@ int qlr_forward(const qlr_qweight* w, const uint16_t* X, int64_t M, const uint16
   p.dq = dq_params(w);
   p.status = stat;
   return cuda_rc(launch_gemm(A_DQ_K, B_TMA_K, bn_tok, OUT_BF16_T, 0, p, maps, st));
+}
+
+int qlr_forward(const qlr_qweight* w, const uint16_t* X, int64_t M, const uint16_t* A, const uint16_t* B, int r,
+                float s, int pooled, uint16_t* Y, uint16_t* T_save, void* workspace, size_t workspace_bytes,
+                int32_t* status, void* stream) {
+  int rc = check_gemm_weight(w);
+  if (rc) return rc;
+  if ((rc = check_rank(r))) return rc;
+  if (M < 0) return QLR_ERR_ARG;
+  if (M == 0) return QLR_OK;
+  if (!X || !A || !B || !Y || !T_save) return QLR_ERR_ARG;
+  if ((rc = qlr_lora_down(w, X, M, A, r, s, pooled, T_save, workspace, workspace_bytes, status, stream))) return rc;
+  return qlr_forward_base(w, X, M, B, r, T_save, Y, status, stream);
 }
 
 // ---- backward: adapter gradients -------------------------------------------------------------------

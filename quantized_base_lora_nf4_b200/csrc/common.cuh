@@ -40,4 +40,7 @@ cudaError_t launch_reduce_splits(const float* part, int splits, int64_t rows, in
 
 int device_sm_count();
 
+// Counts kernel launches issued by this library (reported by qlr_launch_count).
+void count_launch(int n = 1);
+
 }  // namespace qlr

@@ -121,6 +121,7 @@ unsigned grid_for(int64_t n_items, int threads) {
 cudaError_t launch_swiglu_fwd(const uint16_t* G, const uint16_t* U, uint16_t* H, int64_t n, cudaStream_t st) {
   if (n == 0) return cudaSuccess;
   const int64_t n8 = n / 8;
+  count_launch();
   swiglu_fwd_kernel<<<grid_for(n8, 256), 256, 0, st>>>(reinterpret_cast<const uint4*>(G),
                                                        reinterpret_cast<const uint4*>(U), reinterpret_cast<uint4*>(H), n8);
   return cudaGetLastError();
@@ -130,6 +131,7 @@ cudaError_t launch_swiglu_bwd(const uint16_t* dH, const uint16_t* G, const uint1
                               int64_t n, cudaStream_t st) {
   if (n == 0) return cudaSuccess;
   const int64_t n8 = n / 8;
+  count_launch();
   swiglu_bwd_kernel<<<grid_for(n8, 256), 256, 0, st>>>(
       reinterpret_cast<const uint4*>(dH), reinterpret_cast<const uint4*>(G), reinterpret_cast<const uint4*>(U),
       reinterpret_cast<uint4*>(dG), reinterpret_cast<uint4*>(dU), n8);
@@ -138,12 +140,14 @@ cudaError_t launch_swiglu_bwd(const uint16_t* dH, const uint16_t* G, const uint1
 
 cudaError_t launch_pool(const uint16_t* X, int64_t M, int64_t K, int L, uint16_t* Xp, cudaStream_t st) {
   const int64_t n = M * (K / L);
+  count_launch();
   pool_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(X, M, K, L, Xp);
   return cudaGetLastError();
 }
 
 cudaError_t launch_expand_adapter(const uint16_t* A, int r, int64_t K, int L, uint16_t* Aexp, cudaStream_t st) {
   const int64_t n = static_cast<int64_t>(r) * K;
+  count_launch();
   expand_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(A, r, K, L, Aexp);
   return cudaGetLastError();
 }
@@ -154,6 +158,7 @@ cudaError_t launch_reduce_splits(const float* part, int splits, int64_t rows, in
   const int64_t n = rows * cols;
   if (n == 0) return cudaSuccess;
   const int64_t split_rows = (rows + 127) / 128 * 128;  // each split holds whole 128-row tiles
+  count_launch();
   reduce_splits_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(
       part, splits, rows, split_rows, cols, ld_part, scale, transpose, out_bf16, out, ld_out);
   return cudaGetLastError();

@@ -461,6 +461,7 @@ cudaError_t launch_variant(const GemmParams& p, const GemmMaps& maps, cudaStream
   if (attr_err != cudaSuccess) return attr_err;
   const int tiles = p.m_tiles * p.n_tiles * p.splits;
   const int grid = tiles < device_sm_count() ? tiles : device_sm_count();
+  count_launch();
   kern<<<grid, DQ ? kThreadsDq : kThreadsPlain, C::kSmem + 1024, st>>>(p, maps);
   return cudaGetLastError();
 }

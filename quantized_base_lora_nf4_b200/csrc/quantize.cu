@@ -260,6 +260,7 @@ cudaError_t launch_quantize_nfk(const float* W, int64_t n_elems, int bits, int b
   int zc = 0;
   for (int i = 0; i < (1 << bits); ++i)
     if (lv.v[i] == 0.f) zc = i;
+  count_launch();
   quantize_nfk_kernel<<<static_cast<unsigned>(grid), kQuantThreads, 0, st>>>(
       W, n_blocks, bits, block, dq_block, lv, zc, out->codes, out->c1, out->c1_fp8, out->s2, status);
   return cudaGetLastError();
@@ -272,9 +273,9 @@ cudaError_t launch_quantize_int4g(const float* W, int64_t N, int64_t K, int grou
   __half* sc = reinterpret_cast<__half*>(out->scale);
   __half* z = reinterpret_cast<__half*>(out->zero);
   switch (group) {
-    case 32: quantize_int4g_kernel<32><<<static_cast<unsigned>(grid), 256, 0, st>>>(W, n_groups, out->codes, sc, z, status); break;
-    case 64: quantize_int4g_kernel<64><<<static_cast<unsigned>(grid), 256, 0, st>>>(W, n_groups, out->codes, sc, z, status); break;
-    case 128: quantize_int4g_kernel<128><<<static_cast<unsigned>(grid), 256, 0, st>>>(W, n_groups, out->codes, sc, z, status); break;
+    case 32: count_launch(); quantize_int4g_kernel<32><<<static_cast<unsigned>(grid), 256, 0, st>>>(W, n_groups, out->codes, sc, z, status); break;
+    case 64: count_launch(); quantize_int4g_kernel<64><<<static_cast<unsigned>(grid), 256, 0, st>>>(W, n_groups, out->codes, sc, z, status); break;
+    case 128: count_launch(); quantize_int4g_kernel<128><<<static_cast<unsigned>(grid), 256, 0, st>>>(W, n_groups, out->codes, sc, z, status); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
@@ -284,9 +285,11 @@ cudaError_t launch_dequant(const qlr_qweight* w, uint16_t* out, cudaStream_t st)
   const int64_t n_chunks = w->N * w->K / 32;
   const unsigned grid = static_cast<unsigned>((n_chunks + 255) / 256);
   if (w->fmt == QLR_FMT_NFK) {
+    count_launch();
     dequant_nfk_kernel<<<grid, 256, 0, st>>>(w->codes, w->c1, w->c1_fp8, w->s2, w->bits, w->block, w->dq_block,
                                             levels_for(w->bits), n_chunks, out);
   } else {
+    count_launch();
     dequant_int4g_kernel<<<grid, 256, 0, st>>>(w->codes, reinterpret_cast<const __half*>(w->scale),
                                               reinterpret_cast<const __half*>(w->zero), w->group, n_chunks, out);
   }
@@ -297,6 +300,7 @@ cudaError_t launch_merge(const qlr_qweight* w, const uint16_t* A, const uint16_t
                          cudaStream_t st) {
   const int64_t G = w->K / w->group;
   const int64_t n = w->N * G;
+  count_launch();
   merge_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(
       A, B, r, s, w->N, G, w->group, reinterpret_cast<const __half*>(w->scale), reinterpret_cast<__half*>(w->zero));
   return cudaGetLastError();

@@ -28,7 +28,8 @@ EXPORTED = (
     "qlr_error_string", "qlr_version", "qlr_qweight_part_bytes", "qlr_nf_levels", "qlr_quantize_nf4",
     "qlr_quantize_int4_group", "qlr_dequant", "qlr_qalora_merge", "qlr_forward_workspace_bytes", "qlr_forward",
     "qlr_backward_lora_workspace_bytes", "qlr_backward_lora", "qlr_backward_dx_workspace_bytes",
-    "qlr_backward_dx", "qlr_swiglu_forward", "qlr_swiglu_backward", "qlr_device_sm_count",
+    "qlr_backward_dx", "qlr_swiglu_forward", "qlr_swiglu_backward", "qlr_device_sm_count", "qlr_lora_down",
+    "qlr_forward_base", "qlr_launch_count",
 )
 
 
@@ -76,6 +77,9 @@ def lib() -> ctypes.CDLL:
         "qlr_backward_dx": (I, [QP, P, I64, P, P, I, I, I, P, P, SZ, P, P]),
         "qlr_swiglu_forward": (I, [P, P, P, I64, P]),
         "qlr_swiglu_backward": (I, [P, P, P, P, P, I64, P]),
+        "qlr_lora_down": (I, [QP, P, I64, P, I, F, I, P, P, SZ, P, P]),
+        "qlr_forward_base": (I, [QP, P, I64, P, I, P, P, P, P]),
+        "qlr_launch_count": (ctypes.c_uint64, []),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -240,6 +244,35 @@ def forward(q: QWeight, X: torch.Tensor, A: torch.Tensor, B: torch.Tensor, s: fl
     _check(lib().qlr_forward(ctypes.byref(qs), _ptr(X), M, _ptr(A), _ptr(B), r, float(s), int(pooled), _ptr(Y),
                              _ptr(T_save), _ptr(w), w.numel(), _ptr(status), _stream(stream)), "qlr_forward")
     return Y, T_save
+
+
+def lora_down(q: QWeight, X: torch.Tensor, A: torch.Tensor, s: float, pooled: bool = False,
+              T_save: Optional[torch.Tensor] = None, ws: Optional[Workspace] = None,
+              status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    M = X.shape[0]
+    r = A.shape[0]
+    if T_save is None:
+        T_save = torch.empty((M, r), dtype=torch.bfloat16, device=X.device)
+    qs = q.struct()
+    need = lib().qlr_forward_workspace_bytes(ctypes.byref(qs), M, r, int(pooled))
+    w = (ws or Workspace(X.device)).get(need)
+    _check(lib().qlr_lora_down(ctypes.byref(qs), _ptr(X), M, _ptr(A), r, float(s), int(pooled), _ptr(T_save),
+                               _ptr(w), w.numel(), _ptr(status), _stream(stream)), "qlr_lora_down")
+    return T_save
+
+
+def forward_base(q: QWeight, X: torch.Tensor, B: torch.Tensor, T_save: torch.Tensor, Y: Optional[torch.Tensor] = None,
+                 status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    M = X.shape[0]
+    if Y is None:
+        Y = torch.empty((M, q.N), dtype=torch.bfloat16, device=X.device)
+    _check(lib().qlr_forward_base(q.ref(), _ptr(X), M, _ptr(B), B.shape[1], _ptr(T_save), _ptr(Y), _ptr(status),
+                                  _stream(stream)), "qlr_forward_base")
+    return Y
+
+
+def launch_count() -> int:
+    return int(lib().qlr_launch_count())
 
 
 def backward_lora(q: QWeight, X: torch.Tensor, dY: torch.Tensor, T_save: torch.Tensor, B: torch.Tensor, s: float,
