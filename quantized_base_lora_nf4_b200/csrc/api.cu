@@ -349,9 +349,9 @@ int qlr_forward_base(const qlr_qweight* w, const uint16_t* X, int64_t M, const u
   std::memset(&maps, 0, sizeof(maps));
   if ((rc = make_tmap(&maps.codes, w->codes, 1, N, K / 2, 128, 32, 0))) return rc;
   if ((rc = make_tmap(&maps.b, X, 2, M, K, bn_tok, 64, 128))) return rc;
-  if ((rc = make_tmap(&maps.a_tail, B, 2, N, r, 128, 64, 128))) return rc;
   if ((rc = make_tmap(&maps.b_tail, T_save, 2, M, r, bn_tok, 64, 128))) return rc;
-  maps.a = maps.a_tail;
+  maps.a = maps.b;
+  maps.a_tail = maps.b;
   GemmParams p;
   std::memset(&p, 0, sizeof(p));
   p.Mm = static_cast<int>(N);
@@ -367,6 +367,9 @@ int qlr_forward_base(const qlr_qweight* w, const uint16_t* X, int64_t M, const u
   p.ldo = N;
   p.accumulate = 0;
   p.dq = dq_params(w);
+  p.tail_a = B;
+  p.tail_a_rows = N;
+  p.tail_a_cols = r;
   p.status = stat;
   return cuda_rc(launch_gemm(A_DQ_K, B_TMA_K, bn_tok, OUT_BF16_T, 0, p, maps, st));
 }
@@ -499,9 +502,9 @@ int qlr_backward_dx(const qlr_qweight* w, const uint16_t* dY, int64_t M, const u
   std::memset(&maps, 0, sizeof(maps));
   if ((rc = make_tmap(&maps.codes, w->codes, 1, N, K / 2, 64, 64, 0))) return rc;
   if ((rc = make_tmap(&maps.b, dY, 2, M, N, bn_tok, 64, 128))) return rc;
-  if ((rc = make_tmap(&maps.a_tail, At, 2, r, K, 64, 64, 128))) return rc;
   if ((rc = make_tmap(&maps.b_tail, dT, 2, M, r, bn_tok, 64, 128))) return rc;
-  maps.a = maps.a_tail;
+  maps.a = maps.b;
+  maps.a_tail = maps.b;
   GemmParams p;
   std::memset(&p, 0, sizeof(p));
   p.Mm = static_cast<int>(K);
@@ -517,6 +520,9 @@ int qlr_backward_dx(const qlr_qweight* w, const uint16_t* dY, int64_t M, const u
   p.ldo = K;
   p.accumulate = accumulate ? 1 : 0;
   p.dq = dq_params(w);
+  p.tail_a = At;
+  p.tail_a_rows = r;
+  p.tail_a_cols = K;
   p.status = stat;
   return cuda_rc(launch_gemm(A_DQ_MN, B_TMA_K, bn_tok, OUT_BF16_T, 1, p, maps, st));
 }

@@ -1,0 +1,170 @@
+// Device building blocks shared by the tcgen05 GEMM kernels: the 4-bit dequantiser (16-entry bf16
+// table per block or group, byte-permute lookups) and the epilogue stores.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+
+#include "gemm.cuh"
+#include "ptx.cuh"
+
+namespace qlr {
+namespace eng {
+
+__device__ __forceinline__ float e4m3_to_f32(uint8_t b) {
+  const __half_raw h = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(b), __NV_E4M3);
+  return __half2float(__half(h));
+}
+
+struct Lut {
+  uint32_t l0, l1, l2, l3, h0, h1, h2, h3;
+};
+
+__device__ __forceinline__ Lut make_lut(const float (&v)[16]) {
+  uint32_t p[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) p[j] = pack_bf16x2_rn(v[2 * j], v[2 * j + 1]);
+  Lut t;
+  t.l0 = prmt(p[0], p[1], 0x6420);
+  t.h0 = prmt(p[0], p[1], 0x7531);
+  t.l1 = prmt(p[2], p[3], 0x6420);
+  t.h1 = prmt(p[2], p[3], 0x7531);
+  t.l2 = prmt(p[4], p[5], 0x6420);
+  t.h2 = prmt(p[4], p[5], 0x7531);
+  t.l3 = prmt(p[6], p[7], 0x6420);
+  t.h3 = prmt(p[6], p[7], 0x7531);
+  return t;
+}
+
+// 4 codes (low 16 bits of w, code i at bits 4i..4i+3) -> two bf16x2 words (code 0 in the low half).
+__device__ __forceinline__ void lut4(const Lut& t, uint32_t w, uint32_t& o0, uint32_t& o1) {
+  const uint32_t sel = w & 0x7777u;
+  const uint32_t sel2 = ((w >> 1) & 0x4444u) | 0x3210u;
+  const uint32_t lo = prmt(prmt(t.l0, t.l1, sel), prmt(t.l2, t.l3, sel), sel2);
+  const uint32_t hi = prmt(prmt(t.h0, t.h1, sel), prmt(t.h2, t.h3, sel), sel2);
+  o0 = prmt(lo, hi, 0x5140);
+  o1 = prmt(lo, hi, 0x7362);
+}
+
+__device__ __forceinline__ uint4 lut8(const Lut& t, uint32_t w) {
+  uint4 r;
+  lut4(t, w, r.x, r.y);
+  lut4(t, w >> 16, r.z, r.w);
+  return r;
+}
+
+// Per-thread scale data of one 64-code run, loaded one stage ahead of its use so the global-memory
+// latency overlaps the dequantisation of the previous stage.
+//   NF with double quantisation: a = E4M3 byte of the block, b = bits of its fp32 second-level constant;
+//   NF without:                  a = bits of the fp32 block absmax;
+//   INT4 group:                  a = fp16 scales of the run's group(s), b = fp16 zero points.
+struct DqConst {
+  uint32_t a, b;
+};
+
+__device__ __forceinline__ DqConst load_dq_const(const DqParams& dq, int64_t row, int64_t col, bool valid) {
+  DqConst c{0u, 0u};
+  if (!valid) return c;
+  if (dq.fmt == QLR_FMT_NFK) {
+    const int64_t b = (row * dq.K + col) / dq.block;
+    if (dq.dq_block) {
+      c.a = __ldg(dq.c1_fp8 + b);
+      c.b = __float_as_uint(__ldg(dq.s2 + b / dq.dq_block));
+    } else {
+      c.a = __float_as_uint(__ldg(dq.c1 + b));
+    }
+  } else {
+    const int64_t g0 = row * (dq.K / dq.group) + col / dq.group;
+    if (dq.group == 32) {  // two groups per run; g0 is even, so the pair is one aligned 32-bit word
+      c.a = __ldg(reinterpret_cast<const uint32_t*>(dq.scale + g0));
+      c.b = __ldg(reinterpret_cast<const uint32_t*>(dq.zero + g0));
+    } else {
+      c.a = __ldg(reinterpret_cast<const unsigned short*>(dq.scale + g0));
+      c.b = __ldg(reinterpret_cast<const unsigned short*>(dq.zero + g0));
+    }
+  }
+  return c;
+}
+
+__device__ __forceinline__ Lut nf_lut_c(const DqParams& dq, const DqConst& c) {
+  const float scale = dq.dq_block ? __fmul_rn(e4m3_to_f32(static_cast<uint8_t>(c.a)), __uint_as_float(c.b))
+                                  : __uint_as_float(c.a);
+  float v[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(dq.lv.v[i], scale);
+  return make_lut(v);
+}
+
+__device__ __forceinline__ Lut int4_lut_c(uint32_t sc_bits16, uint32_t z_bits16) {
+  const float sc = __half2float(__ushort_as_half(static_cast<unsigned short>(sc_bits16)));
+  const float z = __half2float(__ushort_as_half(static_cast<unsigned short>(z_bits16)));
+  float v[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(__fsub_rn(static_cast<float>(i), z), sc);
+  return make_lut(v);
+}
+
+// Dequantise 64 consecutive 4-bit codes (one row of W, its scale data in `c`) into the eight 16-byte
+// chunks of one 128-byte swizzled shared-memory row at `dst_row` (`sw` = row index for the swizzle).
+__device__ __forceinline__ void dequant_row64(const DqParams& dq, const uint8_t* codes_smem, const DqConst& c,
+                                              bool valid, uint8_t* dst_row, int sw) {
+  const uint4* src = reinterpret_cast<const uint4*>(codes_smem);
+  const uint4 c0 = src[0], c1 = src[1];
+  const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+  if (!valid) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) *reinterpret_cast<uint4*>(dst_row + ((k ^ sw) << 4)) = make_uint4(0, 0, 0, 0);
+    return;
+  }
+  if (dq.fmt == QLR_FMT_NFK) {
+    const Lut t = nf_lut_c(dq, c);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) *reinterpret_cast<uint4*>(dst_row + ((k ^ sw) << 4)) = lut8(t, w[k]);
+  } else if (dq.group == 32) {
+    const Lut t0 = int4_lut_c(c.a & 0xFFFFu, c.b & 0xFFFFu);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) *reinterpret_cast<uint4*>(dst_row + ((k ^ sw) << 4)) = lut8(t0, w[k]);
+    const Lut t1 = int4_lut_c(c.a >> 16, c.b >> 16);
+#pragma unroll
+    for (int k = 4; k < 8; ++k) *reinterpret_cast<uint4*>(dst_row + ((k ^ sw) << 4)) = lut8(t1, w[k]);
+  } else {
+    const Lut t0 = int4_lut_c(c.a, c.b);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) *reinterpret_cast<uint4*>(dst_row + ((k ^ sw) << 4)) = lut8(t0, w[k]);
+  }
+}
+
+// Writes one 32-column chunk of an fp32 accumulator row as bf16 into out^T (out row = D column),
+// transposing through a per-warp 32x32 staging tile so every global store is 16 bytes wide.
+__device__ __forceinline__ void store_chunk_bf16_t(const uint32_t (&v)[32], uint16_t* stg, int lane, int dcol0,
+                                                   int drow0, const GemmParams& p) {
+#pragma unroll
+  for (int jj = 0; jj < 32; ++jj)
+    stg[jj * 32 + lane] = static_cast<uint16_t>(pack_bf16x2_rn(__uint_as_float(v[jj]), 0.f) & 0xFFFFu);
+  __syncwarp();
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    const int idx = t * 32 + lane;
+    const int jj = idx >> 2, part = idx & 3;
+    const int orow = dcol0 + jj;              // output row (D column)
+    const int ocol = drow0 + part * 8;        // output column (D row)
+    if (orow < p.Nn && ocol < p.Mm) {
+      uint4 val = *reinterpret_cast<const uint4*>(stg + jj * 32 + part * 8);
+      uint16_t* dst = static_cast<uint16_t*>(p.out) + static_cast<int64_t>(orow) * p.ldo + ocol;
+      if (p.accumulate) {
+        const uint4 old = *reinterpret_cast<const uint4*>(dst);
+        uint32_t* nv = reinterpret_cast<uint32_t*>(&val);
+        const uint32_t* ov = reinterpret_cast<const uint32_t*>(&old);
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          nv[e] = pack_bf16x2_rn(bf16_bits_to_f32(nv[e] & 0xFFFFu) + bf16_bits_to_f32(ov[e] & 0xFFFFu),
+                                 bf16_bits_to_f32(nv[e] >> 16) + bf16_bits_to_f32(ov[e] >> 16));
+      }
+      *reinterpret_cast<uint4*>(dst) = val;
+    }
+  }
+  __syncwarp();
+}
+
+}  // namespace eng
+}  // namespace qlr

@@ -1,0 +1,369 @@
+// Fused dequantise + tcgen05 GEMM for sm_100a: the frozen 4-bit weight never reaches global memory
+// in bf16 (QLoRA explainer, "The QLoRA recipe", stage 3: each frozen block is dequantised to bf16 on
+// the fly and multiplied by the input; "Background: how LoRA works": the adapter term is added).
+//
+//   forward         D = Y^T [N, M]:  A = dequant(W) tile, K-major  (W rows on the 128 TMEM lanes)
+//                                    B = X tile [tokens, 64], K-major
+//                   tail (r extra reduction columns): A = B_lora rows, B = T_save = s P(X) A^T
+//   input gradient  D = dX^T [K, M]: A = dequant(W)^T tile, MN-major (W rows are the reduction)
+//                                    B = dY tile, K-major
+//                   tail: A = A_lora (or its group expansion) rows, B = dT
+//
+// Three decoupled shared-memory rings keep the dequantiser off the activation stream's latency:
+//   codes ring (8 x 4 KB)   filled by TMA from a dedicated producer warp, far ahead of use;
+//   A ring     (3-4 x 16 KB) written by the dequantiser warps in the canonical 128-byte-swizzled
+//                            UMMA layout (they also copy the tail's weight-side rows);
+//   B ring     (4-8 stages)  activation tiles by TMA.
+// Warp roles: 0 activation producer, 1 TMEM allocator + MMA issuer, 2..5 epilogue, 6..13 two groups
+// of dequantisers taking alternate reduction steps, 14 codes producer.  Two TMEM accumulators
+// (2 x BN fp32 columns) overlap each tile's epilogue with the next tile's main loop.  Every wait is
+// bounded; a wait that runs out aborts the CTA and reports QLR_ERR_TIMEOUT.
+#include <mutex>
+
+#include "engine.cuh"
+
+namespace qlr {
+
+namespace {
+
+constexpr int kThreadsFused = 480;
+
+template <int BN>
+struct FCfg {
+  static constexpr int kA = 16384;
+  static constexpr int kB = BN * 128;
+  static constexpr int kC = 4096;
+  static constexpr int NSA = BN >= 256 ? 3 : 4;
+  static constexpr int NSC = 8;
+  static constexpr int kStaging = 4 * 32 * 32 * 2;
+  static constexpr int kFixed = kStaging + 2048;
+  static constexpr int kBudget = 227 * 1024 - kFixed - NSA * kA - NSC * kC;
+  static constexpr int NSB = (kBudget / kB) > 8 ? 8 : (kBudget / kB);
+  static constexpr int kOffA = NSB * kB;
+  static constexpr int kOffC = kOffA + NSA * kA;
+  static constexpr int kOffStaging = kOffC + NSC * kC;
+  static constexpr int kOffBars = kOffStaging + kStaging;
+  static constexpr int kSmem = kOffBars + 2048;
+  static constexpr int kTmemCols = (2 * BN <= 128) ? 128 : (2 * BN <= 256) ? 256 : 512;
+  static_assert(NSB >= 2, "not enough shared memory");
+  static_assert(kSmem + 1024 <= 227 * 1024, "shared memory budget");
+};
+
+struct alignas(8) FBars {
+  uint64_t b_full[8], b_empty[8];
+  uint64_t a_full[4], a_empty[4];
+  uint64_t c_full[8], c_empty[8];
+  uint64_t acc_full[2], acc_empty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+// Copies 64 bf16 of one row of the tail's weight-side operand (zero outside the matrix) into one
+// 128-byte swizzled shared-memory row.
+__device__ __forceinline__ void copy_row64(const uint16_t* src_row, bool row_ok, int64_t col0, int64_t ncols,
+                                           uint8_t* dst_row, int sw) {
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (row_ok && col0 + 8 * c < ncols) v = __ldg(reinterpret_cast<const uint4*>(src_row + col0 + 8 * c));
+    *reinterpret_cast<uint4*>(dst_row + ((c ^ sw) << 4)) = v;
+  }
+}
+
+template <int A_SRC, int BN>
+__global__ void __launch_bounds__(kThreadsFused, 1)
+    fused_kernel(const __grid_constant__ GemmParams p, const __grid_constant__ GemmMaps maps) {
+  using C = FCfg<BN>;
+  constexpr bool MN = (A_SRC == A_DQ_MN);
+  constexpr uint32_t kIdesc = idesc_bf16(128, BN, MN ? 1u : 0u, 0u);
+  constexpr int NSA = C::NSA, NSB = C::NSB, NSC = C::NSC;
+
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* ring_b = smem;
+  uint8_t* ring_a = smem + C::kOffA;
+  uint8_t* ring_c = smem + C::kOffC;
+  uint8_t* staging = smem + C::kOffStaging;
+  FBars* bars = reinterpret_cast<FBars*>(smem + C::kOffBars);
+  volatile int* abort_flag = &bars->abort_flag;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NSB; ++s) {
+      mbar_init(&bars->b_full[s], 1);
+      mbar_init(&bars->b_empty[s], 1);
+    }
+    for (int s = 0; s < NSA; ++s) {
+      mbar_init(&bars->a_full[s], 128);
+      mbar_init(&bars->a_empty[s], 1);
+    }
+    for (int s = 0; s < NSC; ++s) {
+      mbar_init(&bars->c_full[s], 1);
+      mbar_init(&bars->c_empty[s], 128);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&bars->acc_full[a], 1);
+      mbar_init(&bars->acc_empty[a], 128);
+    }
+    mbar_init(&bars->drain, 1);
+    bars->abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&maps.b);
+    tma_prefetch_desc(&maps.b_tail);
+  }
+  if (warp == 14 && lane == 0) tma_prefetch_desc(&maps.codes);
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = bars->tmem_base;
+
+  const int n_tiles_total = p.m_tiles * p.n_tiles;
+  const int nmain = p.n_main, ntail = p.n_tail, nsteps = nmain + ntail;
+  auto tile_m0 = [&](int tile) { return (tile / p.n_tiles) * 128; };
+  auto tile_n0 = [&](int tile) { return (tile % p.n_tiles) * BN; };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ activation producer
+    if (lane == 0) {
+      uint32_t j = 0;
+      for (int tile = blockIdx.x; tile < n_tiles_total && !*abort_flag; tile += gridDim.x) {
+        const int n0 = tile_n0(tile);
+        for (int ks = 0; ks < nsteps; ++ks, ++j) {
+          const int s = j % NSB;
+          if (!mbar_wait(&bars->b_empty[s], ((j / NSB) & 1) ^ 1, abort_flag)) break;
+          uint64_t* fb = &bars->b_full[s];
+          mbar_arrive_expect_tx(fb, C::kB);
+          if (ks < nmain)
+            tma_load_2d(ring_b + s * C::kB, &maps.b, ks * 64, n0, fb);
+          else
+            tma_load_2d(ring_b + s * C::kB, &maps.b_tail, (ks - nmain) * 64, n0, fb);
+        }
+      }
+      const uint32_t first = j > NSB ? j - NSB : 0;
+      for (uint32_t q = first; q < j; ++q) {
+        volatile int never = 0;
+        mbar_wait(&bars->b_full[q % NSB], (q / NSB) & 1, &never);
+      }
+    }
+  } else if (warp == 14) {
+    // ------------------------------------------------------------------ codes producer
+    if (lane == 0) {
+      uint32_t jc = 0;
+      for (int tile = blockIdx.x; tile < n_tiles_total && !*abort_flag; tile += gridDim.x) {
+        const int m0 = tile_m0(tile);
+        for (int ks = 0; ks < nmain; ++ks, ++jc) {
+          const int s = jc % NSC;
+          if (!mbar_wait(&bars->c_empty[s], ((jc / NSC) & 1) ^ 1, abort_flag)) break;
+          uint64_t* fb = &bars->c_full[s];
+          mbar_arrive_expect_tx(fb, C::kC);
+          if (!MN)
+            tma_load_2d(ring_c + s * C::kC, &maps.codes, ks * 32, m0, fb);   // [128 W rows][32 bytes]
+          else
+            tma_load_2d(ring_c + s * C::kC, &maps.codes, m0 / 2, ks * 64, fb);  // [64 W rows][64 bytes]
+        }
+      }
+      const uint32_t first = jc > NSC ? jc - NSC : 0;
+      for (uint32_t q = first; q < jc; ++q) {
+        volatile int never = 0;
+        mbar_wait(&bars->c_full[q % NSC], (q / NSC) & 1, &never);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t j = 0;
+      int it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < n_tiles_total && ok; tile += gridDim.x, ++it) {
+        const int acc = it & 1;
+        if (!mbar_wait(&bars->acc_empty[acc], ((it >> 1) & 1) ^ 1, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int ks = 0; ks < nsteps; ++ks, ++j) {
+          const int sb = j % NSB, sa = j % NSA;
+          if (!mbar_wait(&bars->b_full[sb], (j / NSB) & 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(&bars->a_full[sa], (j / NSA) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(ring_a + sa * C::kA);
+          const uint32_t b_addr = smem_u32(ring_b + sb * C::kB);
+          int nsub = 4;
+          if (ks >= nmain) {
+            const int rem = p.r_tail - (ks - nmain) * 64;
+            nsub = rem >= 64 ? 4 : (rem + 15) / 16;
+          }
+          for (int kk = 0; kk < nsub; ++kk) {
+            const uint64_t ad = MN ? smem_desc(a_addr + kk * 2048, 8192, 1024, kSw128)
+                                   : smem_desc(a_addr + kk * 32, 16, 1024, kSw128);
+            const uint64_t bd = smem_desc(b_addr + kk * 32, 16, 1024, kSw128);
+            umma_bf16_ss(d_tmem, ad, bd, kIdesc, (ks > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&bars->b_empty[sb]);
+          umma_commit(&bars->a_empty[sa]);
+        }
+        if (!ok) break;
+        umma_commit(&bars->acc_full[acc]);
+      }
+      umma_commit(&bars->drain);
+      volatile int never = 0;
+      mbar_wait(&bars->drain, 0, &never);
+    }
+  } else if (warp < 6) {
+    // ------------------------------------------------------------------ epilogue
+    const int q = warp & 3;
+    uint16_t* stg = reinterpret_cast<uint16_t*>(staging) + q * 32 * 32;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < n_tiles_total; tile += gridDim.x, ++it) {
+      const int m0 = tile_m0(tile), n0 = tile_n0(tile);
+      const int acc = it & 1;
+      const bool got = mbar_wait(&bars->acc_full[acc], (it >> 1) & 1, abort_flag);
+      __syncwarp();
+      if (!__all_sync(0xffffffffu, got)) break;
+      tc_fence_after();
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem_base + acc * BN + c * 32 + ((q * 32) << 16), v);
+        tmem_ld_wait();
+        eng::store_chunk_bf16_t(v, stg, lane, n0 + c * 32, m0 + q * 32, p);
+      }
+      tc_fence_before();
+      mbar_arrive(&bars->acc_empty[acc]);
+    }
+  } else {
+    // ------------------------------------------------------------------ dequantisers (warps 6..13)
+    const int dt = threadIdx.x - 6 * 32;
+    const int grp = dt >> 7;
+    const int t = dt & 127;
+    auto run_of = [&](int m0, int k0, int64_t& row, int64_t& col, bool& valid) {
+      if (!MN) {  // row t of the W tile: W[m0 + t, k0 .. k0 + 63] -> K-major row t
+        row = m0 + t;
+        col = k0;
+        valid = row < p.dq.N;
+      } else {  // W[k0 + nr, m0 + 64h .. +63] -> MN-major atom h, reduction row nr
+        row = k0 + (t >> 1);
+        col = m0 + 64 * (t & 1);
+        valid = row < p.dq.N && col < p.dq.K;
+      }
+    };
+    // cursor over the CTA's step sequence; j counts every step, jc the main (dequantised) ones
+    int tile = blockIdx.x, ks = 0;
+    uint32_t j = 0, jc = 0;
+    auto seek = [&]() -> bool {  // advance to the next step with (j & 1) == grp
+      while (tile < n_tiles_total) {
+        if (ks >= nsteps) {
+          tile += gridDim.x;
+          ks = 0;
+          continue;
+        }
+        if (static_cast<int>(j & 1) == grp) return true;
+        if (ks < nmain) ++jc;
+        ++ks;
+        ++j;
+      }
+      return false;
+    };
+    auto prefetch = [&]() -> eng::DqConst {
+      eng::DqConst c{0u, 0u};
+      if (ks < nmain) {
+        int64_t row, col;
+        bool valid;
+        run_of(tile_m0(tile), ks * 64, row, col, valid);
+        c = eng::load_dq_const(p.dq, row, col, valid);
+      }
+      return c;
+    };
+    bool have = seek();
+    eng::DqConst cur = have ? prefetch() : eng::DqConst{0u, 0u};
+    while (have) {
+      const int c_m0 = tile_m0(tile), c_ks = ks;
+      const uint32_t c_j = j, c_jc = jc;
+      if (ks < nmain) ++jc;
+      ++ks;
+      ++j;
+      const bool have_next = seek();
+      const eng::DqConst nxt = have_next ? prefetch() : eng::DqConst{0u, 0u};
+
+      const int sa = c_j % NSA;
+      if (!mbar_wait(&bars->a_empty[sa], ((c_j / NSA) & 1) ^ 1, abort_flag)) break;
+      uint8_t* st_a = ring_a + sa * C::kA;
+      if (c_ks < nmain) {
+        const int sc = c_jc % NSC;
+        if (!mbar_wait(&bars->c_full[sc], (c_jc / NSC) & 1, abort_flag)) break;
+        const uint8_t* st_c = ring_c + sc * C::kC;
+        int64_t row, col;
+        bool valid;
+        run_of(c_m0, c_ks * 64, row, col, valid);
+        if (!MN) {
+          eng::dequant_row64(p.dq, st_c + t * 32, cur, valid, st_a + t * 128, t & 7);
+        } else {
+          const int nr = t >> 1, h = t & 1;
+          eng::dequant_row64(p.dq, st_c + nr * 64 + h * 32, cur, valid, st_a + h * 8192 + nr * 128, nr & 7);
+        }
+        mbar_arrive(&bars->c_empty[sc]);
+      } else {
+        const int kt = (c_ks - nmain) * 64;
+        if (!MN) {  // B_lora[m0 + t, kt .. kt + 63]
+          const int64_t row = c_m0 + t;
+          copy_row64(p.tail_a + row * p.tail_a_cols, row < p.tail_a_rows, kt, p.tail_a_cols, st_a + t * 128, t & 7);
+        } else {    // A[kt + nr, m0 + 64h .. +63]
+          const int nr = t >> 1, h = t & 1;
+          const int64_t row = kt + nr;
+          copy_row64(p.tail_a + row * p.tail_a_cols, row < p.tail_a_rows, c_m0 + 64 * h, p.tail_a_cols,
+                     st_a + h * 8192 + nr * 128, nr & 7);
+        }
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&bars->a_full[sa]);
+      cur = nxt;
+      have = have_next;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+  if (threadIdx.x == 0 && bars->abort_flag) report(p.status, QLR_ERR_TIMEOUT);
+}
+
+template <int A_SRC, int BN>
+cudaError_t launch_fused_variant(const GemmParams& p, const GemmMaps& maps, cudaStream_t st) {
+  using C = FCfg<BN>;
+  auto kern = fused_kernel<A_SRC, BN>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [&] {
+    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem + 1024);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  const int tiles = p.m_tiles * p.n_tiles;
+  const int grid = tiles < device_sm_count() ? tiles : device_sm_count();
+  count_launch();
+  kern<<<grid, kThreadsFused, C::kSmem + 1024, st>>>(p, maps);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_fused(int a_src, int bn, const GemmParams& p, const GemmMaps& maps, cudaStream_t st) {
+  if (p.splits != 1) return cudaErrorNotSupported;
+  if (a_src == A_DQ_K && bn == 256) return launch_fused_variant<A_DQ_K, 256>(p, maps, st);
+  if (a_src == A_DQ_K && bn == 64) return launch_fused_variant<A_DQ_K, 64>(p, maps, st);
+  if (a_src == A_DQ_MN && bn == 256) return launch_fused_variant<A_DQ_MN, 256>(p, maps, st);
+  if (a_src == A_DQ_MN && bn == 64) return launch_fused_variant<A_DQ_MN, 64>(p, maps, st);
+  return cudaErrorNotSupported;
+}
+
+}  // namespace qlr

@@ -41,12 +41,19 @@ struct GemmParams {
   int64_t ldo;
   int accumulate;        // OUT_BF16_T: add the previous contents of out
   DqParams dq;
+  // fused kernels: the tail's weight-side operand, copied into the A tile by the dequantiser warps
+  // (forward: B [N, r], row-major; input gradient: A or its group expansion [r, K], row-major)
+  const uint16_t* tail_a;
+  int64_t tail_a_rows, tail_a_cols;
   int32_t* status;
 };
 
 struct GemmMaps {
   CUtensorMap a, b, a_tail, b_tail, codes;
 };
+
+// Launches the fused dequant + tcgen05 kernel (a_src = A_DQ_K forward, A_DQ_MN input gradient).
+cudaError_t launch_fused(int a_src, int bn, const GemmParams& p, const GemmMaps& maps, cudaStream_t st);
 
 // Launches the engine variant for (a_src, b_src, BN, out, tail_a_mn).
 cudaError_t launch_gemm(int a_src, int b_src, int bn, int out_mode, int tail_a_mn, const GemmParams& p,
