@@ -248,9 +248,10 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
         row = m0 + t;
         col = k0;
         valid = row < p.dq.N;
-      } else {  // W[k0 + nr, m0 + 64h .. +63] -> MN-major atom h, reduction row nr
-        row = k0 + (t >> 1);
-        col = m0 + 64 * (t & 1);
+      } else {  // W[k0 + nr, m0 + 64h .. +63] -> MN-major atom h, reduction row nr (nr = t % 64, h = t / 64,
+                // so 8 consecutive threads store 8 consecutive swizzled rows without bank conflicts)
+        row = k0 + (t & 63);
+        col = m0 + 64 * (t >> 6);
         valid = row < p.dq.N && col < p.dq.K;
       }
     };
@@ -305,7 +306,7 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
         if (!MN) {
           eng::dequant_row64(p.dq, st_c + t * 32, cur, valid, st_a + t * 128, t & 7);
         } else {
-          const int nr = t >> 1, h = t & 1;
+          const int nr = t & 63, h = t >> 6;
           eng::dequant_row64(p.dq, st_c + nr * 64 + h * 32, cur, valid, st_a + h * 8192 + nr * 128, nr & 7);
         }
         mbar_arrive(&bars->c_empty[sc]);
@@ -315,7 +316,7 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
           const int64_t row = c_m0 + t;
           copy_row64(p.tail_a + row * p.tail_a_cols, row < p.tail_a_rows, kt, p.tail_a_cols, st_a + t * 128, t & 7);
         } else {    // A[kt + nr, m0 + 64h .. +63]
-          const int nr = t >> 1, h = t & 1;
+          const int nr = t & 63, h = t >> 6;
           const int64_t row = kt + nr;
           copy_row64(p.tail_a + row * p.tail_a_cols, row < p.tail_a_rows, c_m0 + 64 * h, p.tail_a_cols,
                      st_a + h * 8192 + nr * 128, nr & 7);
