@@ -114,6 +114,12 @@ DqParams dq_params(const qlr_qweight* w) {
   d.scale = reinterpret_cast<const __half*>(w->scale);
   d.zero = reinterpret_cast<const __half*>(w->zero);
   d.lv = levels_for(w->fmt == QLR_FMT_NFK ? w->bits : 4);
+  const int unit = w->fmt == QLR_FMT_NFK ? w->block : w->group;
+  d.units_per_row = w->K / unit;
+  d.unit_shift = 0;
+  while ((1 << d.unit_shift) < unit) ++d.unit_shift;
+  d.dq_shift = 0;
+  while (w->dq_block && (1 << d.dq_shift) < w->dq_block) ++d.dq_shift;
   return d;
 }
 

@@ -65,23 +65,20 @@ struct DqConst {
 __device__ __forceinline__ DqConst load_dq_const(const DqParams& dq, int64_t row, int64_t col, bool valid) {
   DqConst c{0u, 0u};
   if (!valid) return c;
+  const int64_t u = row * dq.units_per_row + (col >> dq.unit_shift);  // block (NF) or group (INT4) index
   if (dq.fmt == QLR_FMT_NFK) {
-    const int64_t b = (row * dq.K + col) / dq.block;
     if (dq.dq_block) {
-      c.a = __ldg(dq.c1_fp8 + b);
-      c.b = __float_as_uint(__ldg(dq.s2 + b / dq.dq_block));
+      c.a = __ldg(dq.c1_fp8 + u);
+      c.b = __float_as_uint(__ldg(dq.s2 + (u >> dq.dq_shift)));
     } else {
-      c.a = __float_as_uint(__ldg(dq.c1 + b));
+      c.a = __float_as_uint(__ldg(dq.c1 + u));
     }
+  } else if (dq.group == 32) {  // two groups per run; u is even, so the pair is one aligned 32-bit word
+    c.a = __ldg(reinterpret_cast<const uint32_t*>(dq.scale + u));
+    c.b = __ldg(reinterpret_cast<const uint32_t*>(dq.zero + u));
   } else {
-    const int64_t g0 = row * (dq.K / dq.group) + col / dq.group;
-    if (dq.group == 32) {  // two groups per run; g0 is even, so the pair is one aligned 32-bit word
-      c.a = __ldg(reinterpret_cast<const uint32_t*>(dq.scale + g0));
-      c.b = __ldg(reinterpret_cast<const uint32_t*>(dq.zero + g0));
-    } else {
-      c.a = __ldg(reinterpret_cast<const unsigned short*>(dq.scale + g0));
-      c.b = __ldg(reinterpret_cast<const unsigned short*>(dq.zero + g0));
-    }
+    c.a = __ldg(reinterpret_cast<const unsigned short*>(dq.scale + u));
+    c.b = __ldg(reinterpret_cast<const unsigned short*>(dq.zero + u));
   }
   return c;
 }

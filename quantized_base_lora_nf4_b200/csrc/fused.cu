@@ -257,12 +257,14 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
     };
     // cursor over the CTA's step sequence; j counts every step, jc the main (dequantised) ones
     int tile = blockIdx.x, ks = 0;
+    int tm0 = tile < n_tiles_total ? tile_m0(tile) : 0;
     uint32_t j = 0, jc = 0;
     auto seek = [&]() -> bool {  // advance to the next step with (j & 1) == grp
       while (tile < n_tiles_total) {
         if (ks >= nsteps) {
           tile += gridDim.x;
           ks = 0;
+          if (tile < n_tiles_total) tm0 = tile_m0(tile);
           continue;
         }
         if (static_cast<int>(j & 1) == grp) return true;
@@ -277,7 +279,7 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
       if (ks < nmain) {
         int64_t row, col;
         bool valid;
-        run_of(tile_m0(tile), ks * 64, row, col, valid);
+        run_of(tm0, ks * 64, row, col, valid);
         c = eng::load_dq_const(p.dq, row, col, valid);
       }
       return c;
@@ -285,7 +287,7 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
     bool have = seek();
     eng::DqConst cur = have ? prefetch() : eng::DqConst{0u, 0u};
     while (have) {
-      const int c_m0 = tile_m0(tile), c_ks = ks;
+      const int c_m0 = tm0, c_ks = ks;
       const uint32_t c_j = j, c_jc = jc;
       if (ks < nmain) ++jc;
       ++ks;

@@ -20,6 +20,10 @@ enum OutMode : int { OUT_BF16_T = 0, OUT_F32_D = 1 };
 struct DqParams {
   int fmt, bits, block, dq_block, group;
   int64_t N, K;
+  // index arithmetic without division: blocks (NF) or groups (INT4) per row, and log2 of the
+  // block, group and double-quantisation sizes (all powers of two)
+  int64_t units_per_row;
+  int unit_shift, dq_shift;
   const float* c1;
   const uint8_t* c1_fp8;
   const float* s2;
