@@ -79,11 +79,13 @@ def profile_traffic(kernel_file: str):
         return None
     text = open(p).read()
     m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
-    h = re.search(r"gemm_source_sha256:\s*([0-9a-f]{64})", text)
+    h = re.search(r"fused_source_sha256:\s*([0-9a-f]{64})", text)
     if not m or not h:
         return None
-    src = os.path.join(ROOT, "quantized_base_lora_nf4_b200", "csrc", "gemm.cu")
-    if hashlib.sha256(open(src, "rb").read()).hexdigest() != h.group(1):
+    dig = hashlib.sha256()
+    for f in ("fused.cu", "engine.cuh", "ptx.cuh", "gemm.cuh"):
+        dig.update(open(os.path.join(ROOT, "quantized_base_lora_nf4_b200", "csrc", f), "rb").read())
+    if dig.hexdigest() != h.group(1):
         return None
     return float(m.group(1))
 
@@ -419,7 +421,7 @@ def main():
         "config": cfg,
         "tflops": tflops, "tc_frac_of_measured_burst": tflops / peak,
         "tc_frac_of_measured_sustained": tflops / float(peaks.get("bf16_tflops_sustained", peak)),
-        "roofline": {"bound": "tensor", "kernel": "gemm_kernel<A_DQ_K> (fused dequant + tcgen05 forward)",
+        "roofline": {"bound": "tensor", "kernel": "fused_kernel<A_DQ_K> (fused dequant + tcgen05 forward)",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                      "peak_kind": f"{peak_kind} bf16 burst", "traffic": traffic,
                      "flops_per_launch": fwd_flops, "launch_ms": fwd_launch_ms},
