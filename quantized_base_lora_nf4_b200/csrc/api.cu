@@ -123,29 +123,27 @@ DqParams dq_params(const qlr_qweight* w) {
   return d;
 }
 
-// Splits for a reduction of n_steps 64-wide steps over `tiles` output tiles.
+// Cluster size (CTAs reducing one output tile): the largest power of two <= 8 that keeps the grid
+// within one wave of SMs and gives every CTA at least two 64-wide reduction steps.
 int pick_splits(int64_t tiles, int64_t n_steps) {
   const int64_t sms = device_sm_count();
-  int64_t s = cdiv(sms, tiles);
-  const int64_t max_s = n_steps / 2 > 0 ? n_steps / 2 : 1;
-  if (s > max_s) s = max_s;
-  if (s > 16) s = 16;
-  return static_cast<int>(s < 1 ? 1 : s);
+  int s = 1;
+  while (s < 8 && tiles * (2 * s) <= sms && n_steps >= 2 * (2 * s)) s *= 2;
+  return s;
 }
 
-size_t partial_bytes(int64_t Mm, int bn, int splits) { return size_t(splits) * cdiv(Mm, 128) * 128 * bn * 4; }
-
-// One adapter GEMM into fp32 partials (split-K), followed by the fixed-order reduction.
+// One adapter GEMM: D[Mm, r] over n_red reduction elements, A and B from row-major matrices.
 struct AdapterGemm {
   int a_src, b_src, bn;
-  int64_t Mm, Nn, kred;
+  int64_t Mm, n_red;
   const void* a_ptr;
   int64_t a_rows, a_cols;  // row-major extents of the A source matrix
   const void* b_ptr;
   int64_t b_rows, b_cols;
 };
 
-int run_adapter_gemm(const AdapterGemm& g, float* part, int splits, int32_t* status, cudaStream_t st) {
+int run_adapter(const AdapterGemm& g, int r, int out_mode, float scale, int pool_L, void* out, int64_t ld_out,
+                int32_t* status, cudaStream_t st) {
   GemmMaps maps;
   std::memset(&maps, 0, sizeof(maps));
   int rc;
@@ -163,22 +161,21 @@ int run_adapter_gemm(const AdapterGemm& g, float* part, int splits, int32_t* sta
   maps.a_tail = maps.a;
   maps.b_tail = maps.b;
   maps.codes = maps.a;
-  GemmParams p;
+  AdapterParams p;
   std::memset(&p, 0, sizeof(p));
   p.Mm = static_cast<int>(g.Mm);
-  p.Nn = static_cast<int>(g.Nn);
-  p.n_main = static_cast<int>(cdiv(g.kred, 64));
-  p.splits = splits;
-  p.n_tail = 0;
-  p.r_tail = 0;
+  p.r = r;
+  p.n_steps = static_cast<int>(cdiv(g.n_red, 64));
   p.m_tiles = static_cast<int>(cdiv(g.Mm, 128));
-  p.n_tiles = 1;
+  p.splits = pick_splits(p.m_tiles, p.n_steps);
   p.b_atom = atom;
-  p.out = part;
-  p.ldo = g.bn;
-  p.accumulate = 0;
+  p.out_mode = out_mode;
+  p.scale = scale;
+  p.pool_L = pool_L;
+  p.out = out;
+  p.ld_out = ld_out;
   p.status = status;
-  return cuda_rc(launch_gemm(g.a_src, g.b_src, g.bn, OUT_F32_D, 0, p, maps, st));
+  return cuda_rc(launch_adapter(g.a_src, g.b_src, g.bn, p, maps, st));
 }
 
 }  // namespace
@@ -291,13 +288,7 @@ int qlr_qalora_merge(const qlr_qweight* w, const uint16_t* A, const uint16_t* B,
 
 size_t qlr_forward_workspace_bytes(const qlr_qweight* w, int64_t M, int r, int pooled) {
   if (check_qweight(w) || M <= 0 || check_rank(r)) return 0;
-  const int64_t Ka = pooled ? w->K / w->group : w->K;
-  size_t bytes = 0;
-  if (pooled) bytes += align256(size_t(M) * Ka * 2);
-  const int bn = adapter_bn(r);
-  const int splits = pick_splits(cdiv(M, 128), cdiv(Ka, 64));
-  bytes += align256(partial_bytes(M, bn, splits));
-  return bytes;
+  return pooled ? align256(size_t(r) * w->K * 2) : 0;  // the group expansion of A
 }
 
 int qlr_lora_down(const qlr_qweight* w, const uint16_t* X, int64_t M, const uint16_t* A, int r, float s, int pooled,
@@ -313,27 +304,20 @@ int qlr_lora_down(const qlr_qweight* w, const uint16_t* X, int64_t M, const uint
   if (pooled && (w->K / w->group) % 8) return QLR_ERR_SHAPE;
   if (M > (int64_t(1) << 30)) return QLR_ERR_SHAPE;
   const size_t need = qlr_forward_workspace_bytes(w, M, r, pooled);
-  if (!workspace || workspace_bytes < need) return QLR_ERR_WORKSPACE;
-  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return QLR_ERR_ALIGN;
+  if (need && (!workspace || workspace_bytes < need)) return QLR_ERR_WORKSPACE;
+  if (need && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return QLR_ERR_ALIGN;
   cudaStream_t st = as_stream(stream);
   int32_t* stat = status_or_sink(status);
   const int64_t K = w->K;
-  const int64_t Ka = pooled ? K / w->group : K;
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  const uint16_t* Xa = X;
+  // T_save = bf16(s * P(X) A^T) = bf16(s * X Aexp^T), Aexp[j, k] = A[j, k / L] / L for the pooled adapter
+  const uint16_t* Ab = A;
   if (pooled) {
-    uint16_t* Xp = reinterpret_cast<uint16_t*>(ws);
-    ws += align256(size_t(M) * Ka * 2);
-    if ((rc = cuda_rc(launch_pool(X, M, K, w->group, Xp, st)))) return rc;
-    Xa = Xp;
+    uint16_t* Aexp = static_cast<uint16_t*>(workspace);
+    if ((rc = cuda_rc(launch_expand_adapter(A, r, K, w->group, Aexp, st)))) return rc;
+    Ab = Aexp;
   }
-  // T_save = bf16(s * P(X) A^T): split-K tensor-core GEMM into fp32 partials, then a fixed-order sum
-  const int bn = adapter_bn(r);
-  const int splits = pick_splits(cdiv(M, 128), cdiv(Ka, 64));
-  float* part = reinterpret_cast<float*>(ws);
-  AdapterGemm g{A_TMA_K, B_TMA_K, bn, M, r, Ka, Xa, M, Ka, A, r, Ka};
-  if ((rc = run_adapter_gemm(g, part, splits, stat, st))) return rc;
-  return cuda_rc(launch_reduce_splits(part, splits, M, r, bn, s, 0, 1, T_save, r, st));
+  AdapterGemm g{A_TMA_K, B_TMA_K, adapter_bn(r), M, K, X, M, K, Ab, r, K};
+  return run_adapter(g, r, ADAPTER_ROWS_BF16, s, 1, T_save, r, stat, st);
 }
 
 int qlr_forward_base(const qlr_qweight* w, const uint16_t* X, int64_t M, const uint16_t* B, int r,
@@ -396,23 +380,18 @@ int qlr_forward(const qlr_qweight* w, const uint16_t* X, int64_t M, const uint16
 // ---- backward: adapter gradients -------------------------------------------------------------------
 
 size_t qlr_backward_lora_workspace_bytes(const qlr_qweight* w, int64_t M, int r, int pooled) {
-  if (check_qweight(w) || M <= 0 || check_rank(r)) return 0;
-  const int64_t N = w->N;
-  const int64_t Ka = pooled ? w->K / w->group : w->K;
-  size_t bytes = 0;
-  if (pooled) bytes += align256(size_t(M) * Ka * 2);
-  const int bn = adapter_bn(r);
-  size_t p1 = partial_bytes(M, bn, pick_splits(cdiv(M, 128), cdiv(N, 64)));
-  size_t p2 = partial_bytes(N, bn, pick_splits(cdiv(N, 128), cdiv(M, 64)));
-  size_t p3 = partial_bytes(Ka, bn, pick_splits(cdiv(Ka, 128), cdiv(M, 64)));
-  size_t mx = p1 > p2 ? p1 : p2;
-  mx = mx > p3 ? mx : p3;
-  return bytes + align256(mx);
+  (void)w;
+  (void)M;
+  (void)r;
+  (void)pooled;
+  return 0;  // partial sums are reduced inside each cluster through distributed shared memory
 }
 
 int qlr_backward_lora(const qlr_qweight* w, const uint16_t* X, const uint16_t* dY, const uint16_t* T_save,
                       const uint16_t* B, int64_t M, int r, float s, int pooled, float* dA, float* dB,
                       uint16_t* dT_out, void* workspace, size_t workspace_bytes, int32_t* status, void* stream) {
+  (void)workspace;
+  (void)workspace_bytes;
   int rc = check_gemm_weight(w);
   if (rc) return rc;
   if ((rc = check_rank(r))) return rc;
@@ -433,40 +412,22 @@ int qlr_backward_lora(const qlr_qweight* w, const uint16_t* X, const uint16_t* d
     return cuda_rc(cudaMemsetAsync(dB, 0, size_t(N) * r * 4, st));
   }
   if (M > (int64_t(1) << 30)) return QLR_ERR_SHAPE;
-  const size_t need = qlr_backward_lora_workspace_bytes(w, M, r, pooled);
-  if (!workspace || workspace_bytes < need) return QLR_ERR_WORKSPACE;
-  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return QLR_ERR_ALIGN;
   int32_t* stat = status_or_sink(status);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  const uint16_t* Xa = X;
-  if (pooled) {
-    uint16_t* Xp = reinterpret_cast<uint16_t*>(ws);
-    ws += align256(size_t(M) * Ka * 2);
-    if ((rc = cuda_rc(launch_pool(X, M, K, w->group, Xp, st)))) return rc;
-    Xa = Xp;
-  }
-  float* part = reinterpret_cast<float*>(ws);
   const int bn = adapter_bn(r);
   // dT = bf16(s dY B)
   {
-    const int splits = pick_splits(cdiv(M, 128), cdiv(N, 64));
-    AdapterGemm g{A_TMA_K, B_TMA_MN, bn, M, r, N, dY, M, N, B, N, r};
-    if ((rc = run_adapter_gemm(g, part, splits, stat, st))) return rc;
-    if ((rc = cuda_rc(launch_reduce_splits(part, splits, M, r, bn, s, 0, 1, dT_out, r, st)))) return rc;
+    AdapterGemm g{A_TMA_K, B_TMA_MN, bn, M, N, dY, M, N, B, N, r};
+    if ((rc = run_adapter(g, r, ADAPTER_ROWS_BF16, s, 1, dT_out, r, stat, st))) return rc;
   }
   // dB = dY^T T_save  (rows of D are output features, reduction over tokens)
   {
-    const int splits = pick_splits(cdiv(N, 128), cdiv(M, 64));
-    AdapterGemm g{A_TMA_MN, B_TMA_MN, bn, N, r, M, dY, M, N, T_save, M, r};
-    if ((rc = run_adapter_gemm(g, part, splits, stat, st))) return rc;
-    if ((rc = cuda_rc(launch_reduce_splits(part, splits, N, r, bn, 1.0f, 0, 0, dB, r, st)))) return rc;
+    AdapterGemm g{A_TMA_MN, B_TMA_MN, bn, N, M, dY, M, N, T_save, M, r};
+    if ((rc = run_adapter(g, r, ADAPTER_ROWS_F32, 1.0f, 1, dB, r, stat, st))) return rc;
   }
-  // dA^T = P(X)^T dT  (rows of D are adapter inputs, reduction over tokens), stored transposed
+  // dA^T = X^T dT over all K inputs; the pooled adapter sums each group of L inputs and divides by L
   {
-    const int splits = pick_splits(cdiv(Ka, 128), cdiv(M, 64));
-    AdapterGemm g{A_TMA_MN, B_TMA_MN, bn, Ka, r, M, Xa, M, Ka, dT_out, M, r};
-    if ((rc = run_adapter_gemm(g, part, splits, stat, st))) return rc;
-    if ((rc = cuda_rc(launch_reduce_splits(part, splits, Ka, r, bn, 1.0f, 1, 0, dA, Ka, st)))) return rc;
+    AdapterGemm g{A_TMA_MN, B_TMA_MN, bn, K, M, X, M, K, dT_out, M, r};
+    if ((rc = run_adapter(g, r, ADAPTER_COLS_F32, 1.0f, pooled ? w->group : 1, dA, Ka, stat, st))) return rc;
   }
   return QLR_OK;
 }
@@ -474,8 +435,11 @@ int qlr_backward_lora(const qlr_qweight* w, const uint16_t* X, const uint16_t* d
 // ---- backward: input gradient --------------------------------------------------------------------
 
 size_t qlr_backward_dx_workspace_bytes(const qlr_qweight* w, int64_t M, int r, int pooled) {
-  if (check_qweight(w) || M <= 0 || check_rank(r)) return 0;
-  return pooled ? align256(size_t(r) * w->K * 2) : 0;
+  (void)w;
+  (void)M;
+  (void)r;
+  (void)pooled;
+  return 0;  // the pooled adapter's group expansion is formed while the tail rows are copied
 }
 
 int qlr_backward_dx(const qlr_qweight* w, const uint16_t* dY, int64_t M, const uint16_t* A, const uint16_t* dT,
@@ -491,18 +455,12 @@ int qlr_backward_dx(const qlr_qweight* w, const uint16_t* dY, int64_t M, const u
   if (pooled && w->fmt != QLR_FMT_INT4G) return QLR_ERR_UNSUPPORTED;
   if (M == 0) return QLR_OK;
   if (M > (int64_t(1) << 30)) return QLR_ERR_SHAPE;
-  const size_t need = qlr_backward_dx_workspace_bytes(w, M, r, pooled);
-  if (need && (!workspace || workspace_bytes < need)) return QLR_ERR_WORKSPACE;
-  if (need && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return QLR_ERR_ALIGN;
+  (void)workspace;
+  (void)workspace_bytes;
   cudaStream_t st = as_stream(stream);
   int32_t* stat = status_or_sink(status);
   const int64_t N = w->N, K = w->K;
   const uint16_t* At = A;
-  if (pooled) {
-    uint16_t* Aexp = static_cast<uint16_t*>(workspace);
-    if ((rc = cuda_rc(launch_expand_adapter(A, r, K, w->group, Aexp, st)))) return rc;
-    At = Aexp;
-  }
   const int bn_tok = M >= 192 ? 256 : 64;
   GemmMaps maps;
   std::memset(&maps, 0, sizeof(maps));
@@ -528,7 +486,8 @@ int qlr_backward_dx(const qlr_qweight* w, const uint16_t* dY, int64_t M, const u
   p.dq = dq_params(w);
   p.tail_a = At;
   p.tail_a_rows = r;
-  p.tail_a_cols = K;
+  p.tail_a_cols = pooled ? K / w->group : K;
+  p.tail_pool_L = pooled ? w->group : 0;
   p.status = stat;
   return cuda_rc(launch_gemm(A_DQ_MN, B_TMA_K, bn_tok, OUT_BF16_T, 1, p, maps, st));
 }

@@ -71,6 +71,22 @@ __device__ __forceinline__ void copy_row64(const uint16_t* src_row, bool row_ok,
   }
 }
 
+// As copy_row64 for the input gradient's pooled adapter: column k of the row is bf16(A[j, k / L] / L).
+__device__ __forceinline__ void copy_row64_pooled(const uint16_t* src_row, bool row_ok, int64_t col0, int64_t ncols,
+                                                  int L, uint8_t* dst_row, int sw) {
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    uint4 v = make_uint4(0, 0, 0, 0);
+    const int64_t k = col0 + 8 * c;
+    if (row_ok && k < ncols) {
+      const float a = __fdiv_rn(bf16_bits_to_f32(src_row[k / L]), static_cast<float>(L));
+      const uint32_t pair = pack_bf16x2_rn(a, a);
+      v = make_uint4(pair, pair, pair, pair);
+    }
+    *reinterpret_cast<uint4*>(dst_row + ((c ^ sw) << 4)) = v;
+  }
+}
+
 template <int A_SRC, int BN>
 __global__ void __launch_bounds__(kThreadsFused, 1)
     fused_kernel(const __grid_constant__ GemmParams p, const __grid_constant__ GemmMaps maps) {
@@ -317,11 +333,15 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
         if (!MN) {  // B_lora[m0 + t, kt .. kt + 63]
           const int64_t row = c_m0 + t;
           copy_row64(p.tail_a + row * p.tail_a_cols, row < p.tail_a_rows, kt, p.tail_a_cols, st_a + t * 128, t & 7);
-        } else {    // A[kt + nr, m0 + 64h .. +63]
+        } else {    // A[kt + nr, m0 + 64h .. +63] (or the group expansion of the pooled adapter)
           const int nr = t & 63, h = t >> 6;
           const int64_t row = kt + nr;
-          copy_row64(p.tail_a + row * p.tail_a_cols, row < p.tail_a_rows, c_m0 + 64 * h, p.tail_a_cols,
-                     st_a + h * 8192 + nr * 128, nr & 7);
+          const uint16_t* src = p.tail_a + row * p.tail_a_cols;
+          if (p.tail_pool_L > 1)
+            copy_row64_pooled(src, row < p.tail_a_rows, c_m0 + 64 * h, p.dq.K, p.tail_pool_L,
+                              st_a + h * 8192 + nr * 128, nr & 7);
+          else
+            copy_row64(src, row < p.tail_a_rows, c_m0 + 64 * h, p.tail_a_cols, st_a + h * 8192 + nr * 128, nr & 7);
         }
       }
       fence_proxy_async_smem();

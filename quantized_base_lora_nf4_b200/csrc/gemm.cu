@@ -1,16 +1,17 @@
-// tcgen05 GEMM engine for sm_100a: both operands by TMA (the adapter GEMMs of the layer).
+// tcgen05 GEMM engine for sm_100a: the rank-r adapter GEMMs of the layer (both operands by TMA).
 //
-// One persistent CTA per SM walks a static list of output tiles (128 x BN, optionally split along
-// the reduction).  Warp roles:
-//   warp 0        TMA producer: fills a ring of shared-memory stages (A tile + B tile);
-//   warp 1        allocates TMEM and issues tcgen05.mma (one elected lane), committing each stage
-//                 back to the producer and each finished tile to the epilogue;
-//   warps 2..5    epilogue: TMEM -> registers -> global (fp32 partials, or bf16 through a
-//                 transposing shared-memory tile).
-// Operands may be K-major or MN-major (128/64/32-byte swizzle), so the same kernel computes
-// T = X A^T, dT = dY B, dB = dY^T T and dA^T = X^T dT straight from the row-major tensors.
-// Two TMEM accumulators let the epilogue of one tile overlap the main loop of the next.
-// The fused dequantising kernels live in fused.cu.
+//   T   = s P(X) A^T   D[M, r]  = X [M, K]  (K-major)  x  A (or its group expansion) [r, K] (K-major)
+//   dT  = s dY B       D[M, r]  = dY [M, N] (K-major)  x  B [N, r] (MN-major)
+//   dB  = dY^T T       D[N, r]  = dY^T (MN-major)      x  T_save [M, r] (MN-major)
+//   dA^T = X^T dT      D[K, r]  = X^T (MN-major)       x  dT [M, r] (MN-major), pooled by group for QA-LoRA
+//
+// Each output tile (128 rows x r) is computed by one thread-block cluster: CTA `rank` reduces its
+// share of the reduction steps into a TMEM accumulator, the epilogue writes the fp32 partial to its
+// own shared memory, and the cluster leader sums the partials of ranks 0, 1, ..., S-1 through
+// distributed shared memory (a fixed order, so results are deterministic) and applies the output
+// transform.  No partials go through global memory and no separate reduction kernel is launched.
+// Warp roles per CTA: 0 TMA producer, 1 TMEM allocator + MMA issuer, 2..5 epilogue.  All cross-CTA
+// handshakes are mbarrier arrivals with bounded waits.
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -21,59 +22,64 @@ namespace qlr {
 
 namespace {
 
-constexpr int kThreadsPlain = 192;  // producer, MMA, 4 epilogue warps
+constexpr int kThreadsAdapter = 192;
 
 template <int BN>
-struct Cfg {
+struct ACfg {
   static constexpr int kA = 16384;
   static constexpr int kB = BN * 128;
   static constexpr int kStage = ((kA + kB) + 1023) / 1024 * 1024;
-  static constexpr int kStaging = 4 * 32 * 32 * 2;
-  static constexpr int kBudget = 227 * 1024 - kStaging - 2048;
-  static constexpr int kStagesRaw = kBudget / kStage;
-  static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
-  static constexpr int kAcc = (2 * BN <= 512) ? 2 : 1;
-  static constexpr int kTmemCols = (kAcc * BN <= 32) ? 32 : (kAcc * BN <= 64) ? 64 : (kAcc * BN <= 128) ? 128
-                                   : (kAcc * BN <= 256) ? 256 : 512;
-  static constexpr int kSmem = kStages * kStage + kStaging + 2048;
-  static_assert(kStages >= 2, "not enough shared memory for two stages");
+  static constexpr int kStages = 6;
+  static constexpr int kRedStride = BN + 4;  // floats per partial row (padding spreads banks)
+  static constexpr int kRedBytes = 128 * kRedStride * 4;
+  static constexpr int kRing = kStages * kStage;
+  static constexpr int kSmem = (kRing > kRedBytes ? kRing : kRedBytes) + 1024;
+  static constexpr int kTmemCols = BN < 32 ? 32 : BN;
+  static_assert(kRedBytes <= kRing, "partial tile must fit in the stage ring");
 };
 
-struct alignas(8) Bars {
+struct alignas(8) ABars {
   uint64_t full[8];
   uint64_t empty[8];
-  uint64_t acc_full[2];
-  uint64_t acc_empty[2];
+  uint64_t acc_full;
+  uint64_t red_ready;  // leader: one arrival per other CTA of the cluster
+  uint64_t red_done;   // others: the leader has read their partial
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
 };
 
-template <int A_SRC, int B_SRC, int BN, int OUT>
-__global__ void __launch_bounds__(kThreadsPlain, 1)
-    gemm_kernel(const __grid_constant__ GemmParams p, const __grid_constant__ GemmMaps maps) {
-  using C = Cfg<BN>;
+template <int A_SRC, int B_SRC, int BN>
+__global__ void __launch_bounds__(kThreadsAdapter, 1)
+    adapter_kernel(const __grid_constant__ AdapterParams p, const __grid_constant__ GemmMaps maps) {
+  using C = ACfg<BN>;
   constexpr int NS = C::kStages;
   constexpr uint32_t kIdesc = idesc_bf16(128, BN, A_SRC == A_TMA_MN ? 1u : 0u, B_SRC == B_TMA_MN ? 1u : 0u);
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* staging = smem + NS * C::kStage;
-  Bars* bars = reinterpret_cast<Bars*>(staging + C::kStaging);
+  float* red = reinterpret_cast<float*>(smem);  // reuses the ring once the main loop is done
+  ABars* bars = reinterpret_cast<ABars*>(smem + C::kSmem - 1024);
   volatile int* abort_flag = &bars->abort_flag;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const int S = p.splits;
+  const uint32_t rank = S > 1 ? cluster_ctarank() : 0u;
+  const int tile = blockIdx.x / S;
+  const int m0 = tile * 128;
+  const int sps = (p.n_steps + S - 1) / S;
+  const int kb = static_cast<int>(rank) * sps;
+  const int nsteps = max(0, min(p.n_steps, kb + sps) - kb);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(&bars->full[s], 1);
       mbar_init(&bars->empty[s], 1);
     }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(&bars->acc_full[a], 1);
-      mbar_init(&bars->acc_empty[a], 128);
-    }
+    mbar_init(&bars->acc_full, 1);
+    mbar_init(&bars->red_ready, S > 1 ? S - 1 : 1);
+    mbar_init(&bars->red_done, 1);
     mbar_init(&bars->drain, 1);
     bars->abort_flag = 0;
     fence_barrier_init();
@@ -87,139 +93,179 @@ __global__ void __launch_bounds__(kThreadsPlain, 1)
     tmem_relinquish();
   }
   tc_fence_before();
-  __syncthreads();
+  if (S > 1)
+    cluster_sync_all();  // every CTA's barriers exist before any CTA addresses them
+  else
+    __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = bars->tmem_base;
 
-  const int tiles_per_split = p.m_tiles * p.n_tiles;
-  const int n_tiles_total = tiles_per_split * p.splits;
-  const int steps_per_split = (p.n_main + p.splits - 1) / p.splits;
-
-  auto tile_coords = [&](int tile, int& split, int& m0, int& n0, int& kb, int& nmain) {
-    split = tile / tiles_per_split;
-    const int rem = tile % tiles_per_split;
-    m0 = (rem / p.n_tiles) * 128;
-    n0 = (rem % p.n_tiles) * BN;
-    kb = split * steps_per_split;
-    const int ke = min(p.n_main, kb + steps_per_split);
-    nmain = max(0, ke - kb);
-  };
-
   if (warp == 0) {
-    // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      uint32_t j = 0;
-      for (int tile = blockIdx.x; tile < n_tiles_total && !*abort_flag; tile += gridDim.x) {
-        int split, m0, n0, kb, nmain;
-        tile_coords(tile, split, m0, n0, kb, nmain);
-        for (int ks = 0; ks < nmain; ++ks, ++j) {
-          const int s = j % NS;
-          const uint32_t ph = (j / NS) & 1;
-          if (!mbar_wait(&bars->empty[s], ph ^ 1, abort_flag)) break;
-          uint8_t* st_a = smem + s * C::kStage;
-          uint8_t* st_b = st_a + C::kA;
-          uint64_t* fb = &bars->full[s];
-          const int k0 = (kb + ks) * 64;
-          mbar_arrive_expect_tx(fb, C::kA + C::kB);
-          if (A_SRC == A_TMA_K) {
-            tma_load_2d(st_a, &maps.a, k0, m0, fb);
-          } else {
-            tma_load_2d(st_a, &maps.a, m0, k0, fb);
-            tma_load_2d(st_a + 8192, &maps.a, m0 + 64, k0, fb);
-          }
-          if (B_SRC == B_TMA_K) {
-            tma_load_2d(st_b, &maps.b, k0, n0, fb);
-          } else {
-            const int atom_bytes = 64 * p.b_atom * 2;
-            for (int a = 0; a < BN / p.b_atom; ++a) tma_load_2d(st_b + a * atom_bytes, &maps.b, n0 + a * p.b_atom, k0, fb);
-          }
+      for (int ks = 0; ks < nsteps; ++ks) {
+        const int s = ks % NS;
+        if (!mbar_wait(&bars->empty[s], ((ks / NS) & 1) ^ 1, abort_flag)) break;
+        uint8_t* st_a = smem + s * C::kStage;
+        uint8_t* st_b = st_a + C::kA;
+        uint64_t* fb = &bars->full[s];
+        const int k0 = (kb + ks) * 64;
+        mbar_arrive_expect_tx(fb, C::kA + C::kB);
+        if (A_SRC == A_TMA_K) {
+          tma_load_2d(st_a, &maps.a, k0, m0, fb);
+        } else {
+          tma_load_2d(st_a, &maps.a, m0, k0, fb);
+          tma_load_2d(st_a + 8192, &maps.a, m0 + 64, k0, fb);
         }
-      }
-      // drain: wait (bounded, regardless of abort) for the loads of the last NS issued stages
-      const uint32_t first = j > NS ? j - NS : 0;
-      for (uint32_t q = first; q < j; ++q) {
-        volatile int never = 0;
-        mbar_wait(&bars->full[q % NS], (q / NS) & 1, &never);
+        if (B_SRC == B_TMA_K) {
+          tma_load_2d(st_b, &maps.b, k0, 0, fb);
+        } else {
+          const int atom_bytes = 64 * p.b_atom * 2;
+          for (int a = 0; a < BN / p.b_atom; ++a) tma_load_2d(st_b + a * atom_bytes, &maps.b, a * p.b_atom, k0, fb);
+        }
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      uint32_t j = 0;
-      int it = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < n_tiles_total && ok; tile += gridDim.x, ++it) {
-        int split, m0, n0, kb, nmain;
-        tile_coords(tile, split, m0, n0, kb, nmain);
-        const int acc = it % C::kAcc;
-        const uint32_t aph = (it / C::kAcc) & 1;
-        if (!mbar_wait(&bars->acc_empty[acc], aph ^ 1, abort_flag)) break;
+      for (int ks = 0; ks < nsteps; ++ks) {
+        const int s = ks % NS;
+        if (!mbar_wait(&bars->full[s], (ks / NS) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * BN;
-        for (int ks = 0; ks < nmain; ++ks, ++j) {
-          const int s = j % NS;
-          const uint32_t ph = (j / NS) & 1;
-          if (!mbar_wait(&bars->full[s], ph, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t a_addr = smem_u32(smem + s * C::kStage);
-          const uint32_t b_addr = a_addr + C::kA;
+        const uint32_t a_addr = smem_u32(smem + s * C::kStage);
+        const uint32_t b_addr = a_addr + C::kA;
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t ad = (A_SRC == A_TMA_MN) ? smem_desc(a_addr + kk * 2048, 8192, 1024, kSw128)
-                                                    : smem_desc(a_addr + kk * 32, 16, 1024, kSw128);
-            uint64_t bd;
-            if (B_SRC == B_TMA_MN) {
-              const uint32_t rb = p.b_atom * 2;
-              const uint32_t lay = rb == 128 ? kSw128 : (rb == 64 ? kSw64 : kSw32);
-              bd = smem_desc(b_addr + kk * 16 * rb, 64 * rb, 8 * rb, lay);
-            } else {
-              bd = smem_desc(b_addr + kk * 32, 16, 1024, kSw128);
-            }
-            umma_bf16_ss(d_tmem, ad, bd, kIdesc, (ks > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t ad = (A_SRC == A_TMA_MN) ? smem_desc(a_addr + kk * 2048, 8192, 1024, kSw128)
+                                                  : smem_desc(a_addr + kk * 32, 16, 1024, kSw128);
+          uint64_t bd;
+          if (B_SRC == B_TMA_MN) {
+            const uint32_t rb = p.b_atom * 2;
+            bd = smem_desc(b_addr + kk * 16 * rb, 64 * rb, 8 * rb, rb == 128 ? kSw128 : kSw64);
+          } else {
+            bd = smem_desc(b_addr + kk * 32, 16, 1024, kSw128);
           }
-          umma_commit(&bars->empty[s]);
+          umma_bf16_ss(tmem_base, ad, bd, kIdesc, (ks > 0 || kk > 0) ? 1u : 0u);
         }
-        if (!ok) break;
-        umma_commit(&bars->acc_full[acc]);
+        umma_commit(&bars->empty[s]);
       }
-      // make sure every issued MMA has retired before TMEM is released
+      if (ok && nsteps > 0) umma_commit(&bars->acc_full);
+      // every issued MMA retires before TMEM is released, also when a wait above ran out
       umma_commit(&bars->drain);
       volatile int never = 0;
       mbar_wait(&bars->drain, 0, &never);
     }
   } else {
-    // ------------------------------------------------------------------ epilogue
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
-    uint16_t* stg = reinterpret_cast<uint16_t*>(staging) + q * 32 * 32;
-    int it = 0;
-    for (int tile = blockIdx.x; tile < n_tiles_total; tile += gridDim.x, ++it) {
-      int split, m0, n0, kb, nmain;
-      tile_coords(tile, split, m0, n0, kb, nmain);
-      const int acc = it % C::kAcc;
-      const uint32_t aph = (it / C::kAcc) & 1;
-      const bool got = mbar_wait(&bars->acc_full[acc], aph, abort_flag);
+    // ---------------------------------------------------------------- epilogue (warps 2..5)
+    const int q = warp & 3;
+    const int row = q * 32 + lane;  // row of the tile this thread owns
+    float* my = red + row * C::kRedStride;
+    bool ok = true;
+    if (nsteps > 0) {
+      ok = mbar_wait(&bars->acc_full, 0, abort_flag);
       __syncwarp();
-      if (!__all_sync(0xffffffffu, got)) break;
-      tc_fence_after();
-      const int row = m0 + q * 32 + lane;  // D row (MMA M index)
-#pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(tmem_base + acc * BN + c * 32 + ((q * 32) << 16), v);
-        tmem_ld_wait();
-        if (OUT == OUT_F32_D) {
-          float* o = static_cast<float*>(p.out) +
-                     (static_cast<int64_t>(split) * p.m_tiles * 128 + row) * p.ldo + n0 + c * 32;
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    tc_fence_after();
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            reinterpret_cast<float4*>(o)[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                                                          __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
-        } else {
-          eng::store_chunk_bf16_t(v, stg, lane, n0 + c * 32, m0 + q * 32, p);
+    for (int c = 0; c < BN / 32; ++c) {
+      uint32_t v[32];
+      if (nsteps > 0 && ok) {
+        tmem_ld_32x32b_x32(tmem_base + c * 32 + ((q * 32) << 16), v);
+        tmem_ld_wait();
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = 0u;
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        reinterpret_cast<float4*>(my + c * 32)[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                                                __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+    }
+    named_bar_sync(1, 128);
+    bool leader = true;
+    if (S > 1) {
+      if (rank != 0) {
+        leader = false;
+        if (warp == 2 && lane == 0) {
+          mbar_arrive_cluster(mapa_shared(smem_u32(&bars->red_ready), 0));
+          mbar_wait_cluster(&bars->red_done, 0, abort_flag);  // keep this partial alive until it is read
+        }
+      } else {
+        mbar_wait_cluster(&bars->red_ready, 0, abort_flag);
+      }
+    }
+    if (leader) {
+      float acc[BN];
+#pragma unroll
+      for (int i = 0; i < BN / 4; ++i) {
+        const float4 v = reinterpret_cast<const float4*>(my)[i];
+        acc[4 * i] = v.x; acc[4 * i + 1] = v.y; acc[4 * i + 2] = v.z; acc[4 * i + 3] = v.w;
+      }
+      for (int r = 1; r < S; ++r) {  // fixed split order
+        const uint32_t base = mapa_shared(smem_u32(my), static_cast<uint32_t>(r));
+#pragma unroll
+        for (int i = 0; i < BN / 4; ++i) {
+          const float4 v = ld_cluster_f32x4(base + 16 * i);
+          acc[4 * i] += v.x; acc[4 * i + 1] += v.y; acc[4 * i + 2] += v.z; acc[4 * i + 3] += v.w;
         }
       }
-      tc_fence_before();
-      mbar_arrive(&bars->acc_empty[acc]);
+      if (S > 1) {
+        named_bar_sync(1, 128);
+        if (warp == 2 && lane == 0)
+          for (int r = 1; r < S; ++r) mbar_arrive_cluster(mapa_shared(smem_u32(&bars->red_done), static_cast<uint32_t>(r)));
+      }
+      const int grow = m0 + row;
+      if (p.out_mode == ADAPTER_ROWS_BF16) {
+        if (grow < p.Mm) {
+          uint16_t* o = static_cast<uint16_t*>(p.out) + static_cast<int64_t>(grow) * p.ld_out;
+#pragma unroll
+          for (int j = 0; j < BN; j += 8) {
+            if (j < p.r) {
+              uint4 w;
+              w.x = pack_bf16x2_rn(p.scale * acc[j], p.scale * acc[j + 1]);
+              w.y = pack_bf16x2_rn(p.scale * acc[j + 2], p.scale * acc[j + 3]);
+              w.z = pack_bf16x2_rn(p.scale * acc[j + 4], p.scale * acc[j + 5]);
+              w.w = pack_bf16x2_rn(p.scale * acc[j + 6], p.scale * acc[j + 7]);
+              *reinterpret_cast<uint4*>(o + j) = w;
+            }
+          }
+        }
+      } else if (p.out_mode == ADAPTER_ROWS_F32) {
+        if (grow < p.Mm) {
+          float* o = static_cast<float*>(p.out) + static_cast<int64_t>(grow) * p.ld_out;
+#pragma unroll
+          for (int j = 0; j < BN; j += 4)
+            if (j < p.r) *reinterpret_cast<float4*>(o + j) = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+        }
+      } else if (p.pool_L <= 1) {  // ADAPTER_COLS_F32 without pooling: out[j, m]
+        float* o = static_cast<float*>(p.out);
+        if (grow < p.Mm) {
+#pragma unroll
+          for (int j = 0; j < BN; ++j)
+            if (j < p.r) o[static_cast<int64_t>(j) * p.ld_out + grow] = acc[j];
+        }
+      } else {  // ADAPTER_COLS_F32 with group pooling: sum 32-row chunks per warp, then groups of L rows
+        float* chunk = red;  // this CTA's partial is consumed; reuse its space: [4 chunks][BN]
+        named_bar_sync(1, 128);
+#pragma unroll
+        for (int j = 0; j < BN; ++j) {
+          float v = grow < p.Mm ? acc[j] : 0.f;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+          if (lane == 0) chunk[q * BN + j] = v;
+        }
+        named_bar_sync(1, 128);
+        const int per_group = p.pool_L / 32;  // chunks per group (L = 32, 64 or 128)
+        const int n_groups = 128 / p.pool_L;
+        for (int tid = threadIdx.x - 64; tid < n_groups * p.r; tid += 128) {
+          const int g = tid / p.r, j = tid % p.r;
+          float v = 0.f;
+          for (int c = 0; c < per_group; ++c) v += chunk[(g * per_group + c) * BN + j];
+          const int64_t og = (m0 / p.pool_L) + g;
+          if (og * p.pool_L < p.Mm)
+            static_cast<float*>(p.out)[static_cast<int64_t>(j) * p.ld_out + og] = v / static_cast<float>(p.pool_L);
+        }
+      }
     }
   }
 
@@ -233,42 +279,58 @@ __global__ void __launch_bounds__(kThreadsPlain, 1)
   if (threadIdx.x == 0 && bars->abort_flag) report(p.status, QLR_ERR_TIMEOUT);
 }
 
-template <int A_SRC, int B_SRC, int BN, int OUT>
-cudaError_t launch_variant(const GemmParams& p, const GemmMaps& maps, cudaStream_t st) {
-  using C = Cfg<BN>;
-  auto kern = gemm_kernel<A_SRC, B_SRC, BN, OUT>;
+template <int A_SRC, int B_SRC, int BN>
+cudaError_t launch_adapter_variant(const AdapterParams& p, const GemmMaps& maps, cudaStream_t st) {
+  using C = ACfg<BN>;
+  auto kern = adapter_kernel<A_SRC, B_SRC, BN>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [&] {
     attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem + 1024);
   });
   if (attr_err != cudaSuccess) return attr_err;
-  const int tiles = p.m_tiles * p.n_tiles * p.splits;
-  const int grid = tiles < device_sm_count() ? tiles : device_sm_count();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(p.m_tiles * p.splits), 1, 1);
+  cfg.blockDim = dim3(kThreadsAdapter, 1, 1);
+  cfg.dynamicSmemBytes = C::kSmem + 1024;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(p.splits);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   count_launch();
-  kern<<<grid, kThreadsPlain, C::kSmem + 1024, st>>>(p, maps);
-  return cudaGetLastError();
+  return cudaLaunchKernelEx(&cfg, kern, p, maps);
 }
 
 }  // namespace
 
-cudaError_t launch_gemm(int a_src, int b_src, int bn, int out_mode, int tail_a_mn, const GemmParams& p,
-                        const GemmMaps& maps, cudaStream_t st) {
-  (void)tail_a_mn;
-  if (a_src == A_DQ_K || a_src == A_DQ_MN) return launch_fused(a_src, bn, p, maps, st);
-  if (out_mode != OUT_F32_D) return cudaErrorNotSupported;
+cudaError_t launch_adapter(int a_src, int b_src, int bn, const AdapterParams& p, const GemmMaps& maps,
+                           cudaStream_t st) {
+  if (p.splits < 1 || p.splits > 8) return cudaErrorInvalidValue;
   if (a_src == A_TMA_K && b_src == B_TMA_K) {  // T = X A^T
-    if (bn == 32) return launch_variant<A_TMA_K, B_TMA_K, 32, OUT_F32_D>(p, maps, st);
-    if (bn == 64) return launch_variant<A_TMA_K, B_TMA_K, 64, OUT_F32_D>(p, maps, st);
+    if (bn == 32) return launch_adapter_variant<A_TMA_K, B_TMA_K, 32>(p, maps, st);
+    if (bn == 64) return launch_adapter_variant<A_TMA_K, B_TMA_K, 64>(p, maps, st);
   }
   if (a_src == A_TMA_K && b_src == B_TMA_MN) {  // dT = dY B
-    if (bn == 32) return launch_variant<A_TMA_K, B_TMA_MN, 32, OUT_F32_D>(p, maps, st);
-    if (bn == 64) return launch_variant<A_TMA_K, B_TMA_MN, 64, OUT_F32_D>(p, maps, st);
+    if (bn == 32) return launch_adapter_variant<A_TMA_K, B_TMA_MN, 32>(p, maps, st);
+    if (bn == 64) return launch_adapter_variant<A_TMA_K, B_TMA_MN, 64>(p, maps, st);
   }
   if (a_src == A_TMA_MN && b_src == B_TMA_MN) {  // dB = dY^T T, dA^T = X^T dT
-    if (bn == 32) return launch_variant<A_TMA_MN, B_TMA_MN, 32, OUT_F32_D>(p, maps, st);
-    if (bn == 64) return launch_variant<A_TMA_MN, B_TMA_MN, 64, OUT_F32_D>(p, maps, st);
+    if (bn == 32) return launch_adapter_variant<A_TMA_MN, B_TMA_MN, 32>(p, maps, st);
+    if (bn == 64) return launch_adapter_variant<A_TMA_MN, B_TMA_MN, 64>(p, maps, st);
   }
+  return cudaErrorNotSupported;
+}
+
+cudaError_t launch_gemm(int a_src, int b_src, int bn, int out_mode, int tail_a_mn, const GemmParams& p,
+                        const GemmMaps& maps, cudaStream_t st) {
+  (void)b_src;
+  (void)out_mode;
+  (void)tail_a_mn;
+  if (a_src == A_DQ_K || a_src == A_DQ_MN) return launch_fused(a_src, bn, p, maps, st);
   return cudaErrorNotSupported;
 }
 

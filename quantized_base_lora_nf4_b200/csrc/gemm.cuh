@@ -49,12 +49,38 @@ struct GemmParams {
   // (forward: B [N, r], row-major; input gradient: A or its group expansion [r, K], row-major)
   const uint16_t* tail_a;
   int64_t tail_a_rows, tail_a_cols;
+  int tail_pool_L;       // input gradient with the pooled adapter: tail row j is A[j, k / L] / L
   int32_t* status;
 };
 
 struct GemmMaps {
   CUtensorMap a, b, a_tail, b_tail, codes;
 };
+
+// One adapter GEMM D[Mm, r] = sum_k A[Mm, k] B[k, r] (r <= 64), split along k over the CTAs of a
+// thread-block cluster whose leader sums the fp32 partials (distributed shared memory, split order)
+// and writes the result:
+//   ADAPTER_ROWS_BF16   out[m, j] = bf16(scale * D[m, j])     (T_save, dT; ld_out = r)
+//   ADAPTER_ROWS_F32    out[m, j] = D[m, j]                   (dB; ld_out = r)
+//   ADAPTER_COLS_F32    out[j, m / L] = sum over m in a group of L of D[m, j] / L   (dA; ld_out = Ka)
+enum AdapterOut : int { ADAPTER_ROWS_BF16 = 0, ADAPTER_ROWS_F32 = 1, ADAPTER_COLS_F32 = 2 };
+
+struct AdapterParams {
+  int Mm, r;
+  int n_steps;   // 64-wide reduction steps
+  int splits;    // CTAs per cluster (1..8), one output tile per cluster
+  int m_tiles;
+  int b_atom;    // MN-major B: elements per swizzle atom row (32 or 64)
+  int out_mode;
+  float scale;
+  int pool_L;    // ADAPTER_COLS_F32: group length (1 = none)
+  void* out;
+  int64_t ld_out;
+  int32_t* status;
+};
+
+cudaError_t launch_adapter(int a_src, int b_src, int bn, const AdapterParams& p, const GemmMaps& maps,
+                           cudaStream_t st);
 
 // Launches the fused dequant + tcgen05 kernel (a_src = A_DQ_K forward, A_DQ_MN input gradient).
 cudaError_t launch_fused(int a_src, int bn, const GemmParams& p, const GemmMaps& maps, cudaStream_t st);

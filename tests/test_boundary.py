@@ -109,8 +109,9 @@ def test_host_validation_rejects_before_launch(L):
     q3 = _fake_qweight(bits=3)
     assert L.qlr_forward(ctypes.byref(q3), P(0x1000), 16, P(0x1000), P(0x1000), 8, 1.0, 0, P(0x1000), P(0x1000),
                          P(0x1000), 1 << 20, None, None) == -4
-    # missing workspace
-    assert L.qlr_forward(ctypes.byref(q), P(0x1000), 16, P(0x1000), P(0x1000), 8, 1.0, 0, P(0x1000), P(0x1000),
+    # missing workspace (the pooled adapter's group expansion needs one)
+    q4 = _fake_qweight(fmt=2, group=32)
+    assert L.qlr_forward(ctypes.byref(q4), P(0x1000), 16, P(0x1000), P(0x1000), 8, 1.0, 1, P(0x1000), P(0x1000),
                          None, 0, None, None) == -8
     # merge needs an INT4 group weight
     assert L.qlr_qalora_merge(ctypes.byref(q), P(0x1000), P(0x1000), 8, 1.0, None, None) == -1
