@@ -95,23 +95,24 @@ QLR_DEV float4 ld_cluster_f32x4(uint32_t cluster_addr) {
 QLR_DEV void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
-QLR_DEV bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+QLR_DEV bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "r"(smem_u32(bar)), "r"(parity)
       : "memory");
   return ok != 0;
 }
-// Bounded wait with acquire at cluster scope (for phases completed by other CTAs' arrivals).
+// Bounded wait with acquire at cluster scope, for phases completed by other CTAs' arrivals.  It
+// polls without a suspend hint: a remote arrival need not wake a suspended thread early.
 QLR_DEV bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
   const long long t0 = clock64();
   for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait_cluster(bar, parity, kSuspendNs)) return true;
-    if ((it & 15) == 0 && clock64() - t0 > kWaitCycles) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if ((it & 63) == 0 && clock64() - t0 > kWaitCycles) {
       *abort_flag = 1;
       return false;
     }
