@@ -123,13 +123,29 @@ DqParams dq_params(const qlr_qweight* w) {
   return d;
 }
 
-// Cluster size (CTAs reducing one output tile): the largest power of two <= 8 that keeps the grid
-// within one wave of SMs and gives every CTA at least two 64-wide reduction steps.
+// Split of a rank-r adapter GEMM's reduction: minimises waves x (steps per split + a fixed cost of
+// two steps per work item) over the SMs.
 int pick_splits(int64_t tiles, int64_t n_steps) {
   const int64_t sms = device_sm_count();
-  int s = 1;
-  while (s < 8 && tiles * (2 * s) <= sms && n_steps >= 2 * (2 * s)) s *= 2;
-  return s;
+  int best = 1;
+  double best_cost = 1e30;
+  for (int s = 1; s <= 32; ++s) {
+    if (s > 1 && n_steps / s < 2) break;
+    const double waves = static_cast<double>(cdiv(tiles * s, sms));
+    const double cost = waves * (static_cast<double>(n_steps) / s + 2.0);
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best = s;
+    }
+  }
+  return best;
+}
+
+size_t adapter_ws_bytes(int64_t Mm, int64_t n_red, int r) {
+  const int64_t m_tiles = cdiv(Mm, 128);
+  const int S = pick_splits(m_tiles, cdiv(n_red, 64));
+  if (S == 1) return 0;
+  return align256(size_t(S) * m_tiles * 128 * adapter_bn(r) * 4) + align256(size_t(m_tiles) * 4);
 }
 
 // One adapter GEMM: D[Mm, r] over n_red reduction elements, A and B from row-major matrices.
@@ -143,7 +159,7 @@ struct AdapterGemm {
 };
 
 int run_adapter(const AdapterGemm& g, int r, int out_mode, float scale, int pool_L, void* out, int64_t ld_out,
-                int32_t* status, cudaStream_t st) {
+                uint8_t* ws, int32_t* status, cudaStream_t st) {
   GemmMaps maps;
   std::memset(&maps, 0, sizeof(maps));
   int rc;
@@ -175,6 +191,11 @@ int run_adapter(const AdapterGemm& g, int r, int out_mode, float scale, int pool
   p.out = out;
   p.ld_out = ld_out;
   p.status = status;
+  if (p.splits > 1) {
+    p.part = reinterpret_cast<float*>(ws);
+    p.counters = reinterpret_cast<int*>(ws + align256(size_t(p.splits) * p.m_tiles * 128 * g.bn * 4));
+    if (cudaMemsetAsync(p.counters, 0, size_t(p.m_tiles) * 4, st) != cudaSuccess) return QLR_ERR_CUDA;
+  }
   return cuda_rc(launch_adapter(g.a_src, g.b_src, g.bn, p, maps, st));
 }
 
@@ -288,7 +309,8 @@ int qlr_qalora_merge(const qlr_qweight* w, const uint16_t* A, const uint16_t* B,
 
 size_t qlr_forward_workspace_bytes(const qlr_qweight* w, int64_t M, int r, int pooled) {
   if (check_qweight(w) || M <= 0 || check_rank(r)) return 0;
-  return pooled ? align256(size_t(r) * w->K * 2) : 0;  // the group expansion of A
+  // the group expansion of A (pooled adapter), then the split partial sums and tile counters
+  return (pooled ? align256(size_t(r) * w->K * 2) : 0) + adapter_ws_bytes(M, w->K, r);
 }
 
 int qlr_lora_down(const qlr_qweight* w, const uint16_t* X, int64_t M, const uint16_t* A, int r, float s, int pooled,
@@ -311,13 +333,15 @@ int qlr_lora_down(const qlr_qweight* w, const uint16_t* X, int64_t M, const uint
   const int64_t K = w->K;
   // T_save = bf16(s * P(X) A^T) = bf16(s * X Aexp^T), Aexp[j, k] = A[j, k / L] / L for the pooled adapter
   const uint16_t* Ab = A;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
   if (pooled) {
-    uint16_t* Aexp = static_cast<uint16_t*>(workspace);
+    uint16_t* Aexp = reinterpret_cast<uint16_t*>(ws);
+    ws += align256(size_t(r) * K * 2);
     if ((rc = cuda_rc(launch_expand_adapter(A, r, K, w->group, Aexp, st)))) return rc;
     Ab = Aexp;
   }
   AdapterGemm g{A_TMA_K, B_TMA_K, adapter_bn(r), M, K, X, M, K, Ab, r, K};
-  return run_adapter(g, r, ADAPTER_ROWS_BF16, s, 1, T_save, r, stat, st);
+  return run_adapter(g, r, ADAPTER_ROWS_BF16, s, 1, T_save, r, ws, stat, st);
 }
 
 int qlr_forward_base(const qlr_qweight* w, const uint16_t* X, int64_t M, const uint16_t* B, int r,
@@ -380,18 +404,18 @@ int qlr_forward(const qlr_qweight* w, const uint16_t* X, int64_t M, const uint16
 // ---- backward: adapter gradients -------------------------------------------------------------------
 
 size_t qlr_backward_lora_workspace_bytes(const qlr_qweight* w, int64_t M, int r, int pooled) {
-  (void)w;
-  (void)M;
-  (void)r;
   (void)pooled;
-  return 0;  // partial sums are reduced inside each cluster through distributed shared memory
+  if (check_qweight(w) || M <= 0 || check_rank(r)) return 0;
+  // split partial sums and tile counters of the three GEMMs, which run one after another
+  const size_t a = adapter_ws_bytes(M, w->N, r);
+  const size_t b = adapter_ws_bytes(w->N, M, r);
+  const size_t c = adapter_ws_bytes(w->K, M, r);
+  return a > b ? (a > c ? a : c) : (b > c ? b : c);
 }
 
 int qlr_backward_lora(const qlr_qweight* w, const uint16_t* X, const uint16_t* dY, const uint16_t* T_save,
                       const uint16_t* B, int64_t M, int r, float s, int pooled, float* dA, float* dB,
                       uint16_t* dT_out, void* workspace, size_t workspace_bytes, int32_t* status, void* stream) {
-  (void)workspace;
-  (void)workspace_bytes;
   int rc = check_gemm_weight(w);
   if (rc) return rc;
   if ((rc = check_rank(r))) return rc;
@@ -412,22 +436,26 @@ int qlr_backward_lora(const qlr_qweight* w, const uint16_t* X, const uint16_t* d
     return cuda_rc(cudaMemsetAsync(dB, 0, size_t(N) * r * 4, st));
   }
   if (M > (int64_t(1) << 30)) return QLR_ERR_SHAPE;
+  const size_t need = qlr_backward_lora_workspace_bytes(w, M, r, pooled);
+  if (need && (!workspace || workspace_bytes < need)) return QLR_ERR_WORKSPACE;
+  if (need && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return QLR_ERR_ALIGN;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
   int32_t* stat = status_or_sink(status);
   const int bn = adapter_bn(r);
   // dT = bf16(s dY B)
   {
     AdapterGemm g{A_TMA_K, B_TMA_MN, bn, M, N, dY, M, N, B, N, r};
-    if ((rc = run_adapter(g, r, ADAPTER_ROWS_BF16, s, 1, dT_out, r, stat, st))) return rc;
+    if ((rc = run_adapter(g, r, ADAPTER_ROWS_BF16, s, 1, dT_out, r, ws, stat, st))) return rc;
   }
   // dB = dY^T T_save  (rows of D are output features, reduction over tokens)
   {
     AdapterGemm g{A_TMA_MN, B_TMA_MN, bn, N, M, dY, M, N, T_save, M, r};
-    if ((rc = run_adapter(g, r, ADAPTER_ROWS_F32, 1.0f, 1, dB, r, stat, st))) return rc;
+    if ((rc = run_adapter(g, r, ADAPTER_ROWS_F32, 1.0f, 1, dB, r, ws, stat, st))) return rc;
   }
   // dA^T = X^T dT over all K inputs; the pooled adapter sums each group of L inputs and divides by L
   {
     AdapterGemm g{A_TMA_MN, B_TMA_MN, bn, K, M, X, M, K, dT_out, M, r};
-    if ((rc = run_adapter(g, r, ADAPTER_COLS_F32, 1.0f, pooled ? w->group : 1, dA, Ka, stat, st))) return rc;
+    if ((rc = run_adapter(g, r, ADAPTER_COLS_F32, 1.0f, pooled ? w->group : 1, dA, Ka, ws, stat, st))) return rc;
   }
   return QLR_OK;
 }

@@ -5,13 +5,12 @@
 //   dB  = dY^T T       D[N, r]  = dY^T (MN-major)      x  T_save [M, r] (MN-major)
 //   dA^T = X^T dT      D[K, r]  = X^T (MN-major)       x  dT [M, r] (MN-major), pooled by group for QA-LoRA
 //
-// Each output tile (128 rows x r) is computed by one thread-block cluster: CTA `rank` reduces its
-// share of the reduction steps into a TMEM accumulator, the epilogue writes the fp32 partial to its
-// own shared memory, and the cluster leader sums the partials of ranks 0, 1, ..., S-1 through
-// distributed shared memory (a fixed order, so results are deterministic) and applies the output
-// transform.  No partials go through global memory and no separate reduction kernel is launched.
-// Warp roles per CTA: 0 TMA producer, 1 TMEM allocator + MMA issuer, 2..5 epilogue.  All cross-CTA
-// handshakes are mbarrier arrivals with bounded waits.
+// One persistent CTA per SM walks a static list of (tile, split) work items; a tile is 128 rows x BN.
+// Warp roles: 0 TMA producer (ring of A+B stages), 1 TMEM allocator + single-thread tcgen05.mma
+// issuer, 2..5 epilogue.  Two TMEM accumulators overlap an item's epilogue with the next item's main
+// loop.  With a split reduction each item's fp32 tile is stored to the workspace; the CTA that
+// finishes a tile last (per-tile atomic counter) sums all parts in split order -- deterministic --
+// and applies the output transform, so no separate reduction kernel is launched.
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -29,25 +28,80 @@ struct ACfg {
   static constexpr int kA = 16384;
   static constexpr int kB = BN * 128;
   static constexpr int kStage = ((kA + kB) + 1023) / 1024 * 1024;
-  static constexpr int kStages = 6;
-  static constexpr int kRedStride = BN + 4;  // floats per partial row (padding spreads banks)
-  static constexpr int kRedBytes = 128 * kRedStride * 4;
-  static constexpr int kRing = kStages * kStage;
-  static constexpr int kSmem = (kRing > kRedBytes ? kRing : kRedBytes) + 1024;
-  static constexpr int kTmemCols = BN < 32 ? 32 : BN;
-  static_assert(kRedBytes <= kRing, "partial tile must fit in the stage ring");
+  static constexpr int kStages = 8;
+  static constexpr int kScratch = 4 * BN * 4 + 64;  // per-warp chunk sums + flags
+  static constexpr int kSmem = kStages * kStage + 2048;
+  static constexpr int kTmemCols = (2 * BN <= 64) ? 64 : 128;
 };
 
 struct alignas(8) ABars {
   uint64_t full[8];
   uint64_t empty[8];
-  uint64_t acc_full;
-  uint64_t red_ready;  // leader: one arrival per other CTA of the cluster
-  uint64_t red_done;   // others: the leader has read their partial
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
+  int is_last;
+  float chunk[4 * 64];
 };
+
+// Output transform of one finished row (`acc` = the BN fp32 values of D row m0 + row).
+template <int BN>
+__device__ __forceinline__ void adapter_store(const AdapterParams& p, float (&acc)[BN], int m0, int row, int lane,
+                                              int q, ABars* bars) {
+  const int grow = m0 + row;
+  if (p.out_mode == ADAPTER_ROWS_BF16) {
+    if (grow < p.Mm) {
+      uint16_t* o = static_cast<uint16_t*>(p.out) + static_cast<int64_t>(grow) * p.ld_out;
+#pragma unroll
+      for (int j = 0; j < BN; j += 8) {
+        if (j < p.r) {
+          uint4 w;
+          w.x = pack_bf16x2_rn(p.scale * acc[j], p.scale * acc[j + 1]);
+          w.y = pack_bf16x2_rn(p.scale * acc[j + 2], p.scale * acc[j + 3]);
+          w.z = pack_bf16x2_rn(p.scale * acc[j + 4], p.scale * acc[j + 5]);
+          w.w = pack_bf16x2_rn(p.scale * acc[j + 6], p.scale * acc[j + 7]);
+          *reinterpret_cast<uint4*>(o + j) = w;
+        }
+      }
+    }
+  } else if (p.out_mode == ADAPTER_ROWS_F32) {
+    if (grow < p.Mm) {
+      float* o = static_cast<float*>(p.out) + static_cast<int64_t>(grow) * p.ld_out;
+#pragma unroll
+      for (int j = 0; j < BN; j += 4)
+        if (j < p.r) *reinterpret_cast<float4*>(o + j) = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+    }
+  } else if (p.pool_L <= 1) {  // out[j, m]
+    if (grow < p.Mm) {
+      float* o = static_cast<float*>(p.out);
+#pragma unroll
+      for (int j = 0; j < BN; ++j)
+        if (j < p.r) o[static_cast<int64_t>(j) * p.ld_out + grow] = acc[j];
+    }
+  } else {  // out[j, m / L]: sum 32-row chunks per warp, then groups of L rows
+#pragma unroll
+    for (int j = 0; j < BN; ++j) {
+      float v = grow < p.Mm ? acc[j] : 0.f;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if (lane == 0) bars->chunk[q * BN + j] = v;
+    }
+    named_bar_sync(1, 128);
+    const int per_group = p.pool_L / 32;
+    const int n_groups = 128 / p.pool_L;
+    for (int tid = row; tid < n_groups * p.r; tid += 128) {  // row doubles as a 0..127 thread index
+      const int g = tid / p.r, j = tid % p.r;
+      float v = 0.f;
+      for (int c = 0; c < per_group; ++c) v += bars->chunk[(g * per_group + c) * BN + j];
+      const int64_t og = (m0 / p.pool_L) + g;
+      if (og * p.pool_L < p.Mm)
+        static_cast<float*>(p.out)[static_cast<int64_t>(j) * p.ld_out + og] = v / static_cast<float>(p.pool_L);
+    }
+    named_bar_sync(1, 128);
+  }
+}
 
 template <int A_SRC, int B_SRC, int BN>
 __global__ void __launch_bounds__(kThreadsAdapter, 1)
@@ -58,28 +112,30 @@ __global__ void __launch_bounds__(kThreadsAdapter, 1)
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float* red = reinterpret_cast<float*>(smem);  // reuses the ring once the main loop is done
-  ABars* bars = reinterpret_cast<ABars*>(smem + C::kSmem - 1024);
+  ABars* bars = reinterpret_cast<ABars*>(smem + NS * C::kStage);
   volatile int* abort_flag = &bars->abort_flag;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int S = p.splits;
-  const uint32_t rank = S > 1 ? cluster_ctarank() : 0u;
-  const int tile = blockIdx.x / S;
-  const int m0 = tile * 128;
+  const int n_items = p.m_tiles * S;
   const int sps = (p.n_steps + S - 1) / S;
-  const int kb = static_cast<int>(rank) * sps;
-  const int nsteps = max(0, min(p.n_steps, kb + sps) - kb);
+  auto item_coords = [&](int item, int& tile, int& split, int& kb, int& nsteps) {
+    split = item / p.m_tiles;
+    tile = item % p.m_tiles;
+    kb = split * sps;
+    nsteps = max(0, min(p.n_steps, kb + sps) - kb);
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(&bars->full[s], 1);
       mbar_init(&bars->empty[s], 1);
     }
-    mbar_init(&bars->acc_full, 1);
-    mbar_init(&bars->red_ready, S > 1 ? S - 1 : 1);
-    mbar_init(&bars->red_done, 1);
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&bars->acc_full[a], 1);
+      mbar_init(&bars->acc_empty[a], 128);
+    }
     mbar_init(&bars->drain, 1);
     bars->abort_flag = 0;
     fence_barrier_init();
@@ -93,179 +149,141 @@ __global__ void __launch_bounds__(kThreadsAdapter, 1)
     tmem_relinquish();
   }
   tc_fence_before();
-  if (S > 1)
-    cluster_sync_all();  // every CTA's barriers exist before any CTA addresses them
-  else
-    __syncthreads();
+  __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = bars->tmem_base;
 
   if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      for (int ks = 0; ks < nsteps; ++ks) {
-        const int s = ks % NS;
-        if (!mbar_wait(&bars->empty[s], ((ks / NS) & 1) ^ 1, abort_flag)) break;
-        uint8_t* st_a = smem + s * C::kStage;
-        uint8_t* st_b = st_a + C::kA;
-        uint64_t* fb = &bars->full[s];
-        const int k0 = (kb + ks) * 64;
-        mbar_arrive_expect_tx(fb, C::kA + C::kB);
-        if (A_SRC == A_TMA_K) {
-          tma_load_2d(st_a, &maps.a, k0, m0, fb);
-        } else {
-          tma_load_2d(st_a, &maps.a, m0, k0, fb);
-          tma_load_2d(st_a + 8192, &maps.a, m0 + 64, k0, fb);
+      uint32_t j = 0;
+      for (int item = blockIdx.x; item < n_items && !*abort_flag; item += gridDim.x) {
+        int tile, split, kb, nsteps;
+        item_coords(item, tile, split, kb, nsteps);
+        const int m0 = tile * 128;
+        for (int ks = 0; ks < nsteps; ++ks, ++j) {
+          const int s = j % NS;
+          if (!mbar_wait(&bars->empty[s], ((j / NS) & 1) ^ 1, abort_flag)) break;
+          uint8_t* st_a = smem + s * C::kStage;
+          uint8_t* st_b = st_a + C::kA;
+          uint64_t* fb = &bars->full[s];
+          const int k0 = (kb + ks) * 64;
+          mbar_arrive_expect_tx(fb, C::kA + C::kB);
+          if (A_SRC == A_TMA_K) {
+            tma_load_2d(st_a, &maps.a, k0, m0, fb);
+          } else {
+            tma_load_2d(st_a, &maps.a, m0, k0, fb);
+            tma_load_2d(st_a + 8192, &maps.a, m0 + 64, k0, fb);
+          }
+          if (B_SRC == B_TMA_K) {
+            tma_load_2d(st_b, &maps.b, k0, 0, fb);
+          } else {
+            const int atom_bytes = 64 * p.b_atom * 2;
+            for (int a = 0; a < BN / p.b_atom; ++a) tma_load_2d(st_b + a * atom_bytes, &maps.b, a * p.b_atom, k0, fb);
+          }
         }
-        if (B_SRC == B_TMA_K) {
-          tma_load_2d(st_b, &maps.b, k0, 0, fb);
-        } else {
-          const int atom_bytes = 64 * p.b_atom * 2;
-          for (int a = 0; a < BN / p.b_atom; ++a) tma_load_2d(st_b + a * atom_bytes, &maps.b, a * p.b_atom, k0, fb);
-        }
+      }
+      const uint32_t first = j > NS ? j - NS : 0;
+      for (uint32_t qq = first; qq < j; ++qq) {
+        volatile int never = 0;
+        mbar_wait(&bars->full[qq % NS], (qq / NS) & 1, &never);
       }
     }
   } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
+      uint32_t j = 0;
+      int it = 0;
       bool ok = true;
-      for (int ks = 0; ks < nsteps; ++ks) {
-        const int s = ks % NS;
-        if (!mbar_wait(&bars->full[s], (ks / NS) & 1, abort_flag)) { ok = false; break; }
+      for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++it) {
+        int tile, split, kb, nsteps;
+        item_coords(item, tile, split, kb, nsteps);
+        const int acc = it & 1;
+        if (!mbar_wait(&bars->acc_empty[acc], ((it >> 1) & 1) ^ 1, abort_flag)) break;
         tc_fence_after();
-        const uint32_t a_addr = smem_u32(smem + s * C::kStage);
-        const uint32_t b_addr = a_addr + C::kA;
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int ks = 0; ks < nsteps; ++ks, ++j) {
+          const int s = j % NS;
+          if (!mbar_wait(&bars->full[s], (j / NS) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + s * C::kStage);
+          const uint32_t b_addr = a_addr + C::kA;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t ad = (A_SRC == A_TMA_MN) ? smem_desc(a_addr + kk * 2048, 8192, 1024, kSw128)
-                                                  : smem_desc(a_addr + kk * 32, 16, 1024, kSw128);
-          uint64_t bd;
-          if (B_SRC == B_TMA_MN) {
-            const uint32_t rb = p.b_atom * 2;
-            bd = smem_desc(b_addr + kk * 16 * rb, 64 * rb, 8 * rb, rb == 128 ? kSw128 : kSw64);
-          } else {
-            bd = smem_desc(b_addr + kk * 32, 16, 1024, kSw128);
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ad = (A_SRC == A_TMA_MN) ? smem_desc(a_addr + kk * 2048, 8192, 1024, kSw128)
+                                                    : smem_desc(a_addr + kk * 32, 16, 1024, kSw128);
+            uint64_t bd;
+            if (B_SRC == B_TMA_MN) {
+              const uint32_t rb = p.b_atom * 2;
+              bd = smem_desc(b_addr + kk * 16 * rb, 64 * rb, 8 * rb, rb == 128 ? kSw128 : kSw64);
+            } else {
+              bd = smem_desc(b_addr + kk * 32, 16, 1024, kSw128);
+            }
+            umma_bf16_ss(d_tmem, ad, bd, kIdesc, (ks > 0 || kk > 0) ? 1u : 0u);
           }
-          umma_bf16_ss(tmem_base, ad, bd, kIdesc, (ks > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(&bars->empty[s]);
         }
-        umma_commit(&bars->empty[s]);
+        if (!ok) break;
+        umma_commit(&bars->acc_full[acc]);  // also for an empty item: the epilogue then reads zeros
       }
-      if (ok && nsteps > 0) umma_commit(&bars->acc_full);
-      // every issued MMA retires before TMEM is released, also when a wait above ran out
       umma_commit(&bars->drain);
       volatile int never = 0;
       mbar_wait(&bars->drain, 0, &never);
     }
   } else {
-    // ---------------------------------------------------------------- epilogue (warps 2..5)
+    // ------------------------------------------------------------------ epilogue (warps 2..5)
     const int q = warp & 3;
-    const int row = q * 32 + lane;  // row of the tile this thread owns
-    float* my = red + row * C::kRedStride;
-    bool ok = true;
-    if (nsteps > 0) {
-      ok = mbar_wait(&bars->acc_full, 0, abort_flag);
+    const int row = q * 32 + lane;
+    int it = 0;
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it) {
+      int tile, split, kb, nsteps;
+      item_coords(item, tile, split, kb, nsteps);
+      const int m0 = tile * 128;
+      const int acc = it & 1;
+      const bool got = mbar_wait(&bars->acc_full[acc], (it >> 1) & 1, abort_flag);
       __syncwarp();
-      ok = __all_sync(0xffffffffu, ok);
-    }
-    tc_fence_after();
+      if (!__all_sync(0xffffffffu, got)) break;
+      tc_fence_after();
+      float v[BN];
 #pragma unroll
-    for (int c = 0; c < BN / 32; ++c) {
-      uint32_t v[32];
-      if (nsteps > 0 && ok) {
-        tmem_ld_32x32b_x32(tmem_base + c * 32 + ((q * 32) << 16), v);
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t u[32];
+        tmem_ld_32x32b_x32(tmem_base + acc * BN + c * 32 + ((q * 32) << 16), u);
         tmem_ld_wait();
-      } else {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = 0u;
+        for (int i = 0; i < 32; ++i) v[c * 32 + i] = nsteps > 0 ? __uint_as_float(u[i]) : 0.f;
       }
+      tc_fence_before();
+      mbar_arrive(&bars->acc_empty[acc]);  // the accumulator is free for the next item
+      if (S == 1) {
+        adapter_store<BN>(p, v, m0, row, lane, q, bars);
+        continue;
+      }
+      float* mine = p.part + (static_cast<int64_t>(split) * p.m_tiles * 128 + m0 + row) * BN;
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
-        reinterpret_cast<float4*>(my + c * 32)[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                                                                __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
-    }
-    named_bar_sync(1, 128);
-    bool leader = true;
-    if (S > 1) {
-      if (rank != 0) {
-        leader = false;
-        if (warp == 2 && lane == 0) {
-          mbar_arrive_cluster(mapa_shared(smem_u32(&bars->red_ready), 0));
-          mbar_wait_cluster(&bars->red_done, 0, abort_flag);  // keep this partial alive until it is read
-        }
-      } else {
-        mbar_wait_cluster(&bars->red_ready, 0, abort_flag);
-      }
-    }
-    if (leader) {
-      float acc[BN];
+      for (int i = 0; i < BN / 4; ++i)
+        reinterpret_cast<float4*>(mine)[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+      __threadfence();
+      named_bar_sync(1, 128);
+      if (row == 0) bars->is_last = (atomicAdd(p.counters + tile, 1) == S - 1);
+      named_bar_sync(1, 128);
+      if (bars->is_last) {  // uniform across the 128 epilogue threads
+        __threadfence();
 #pragma unroll
-      for (int i = 0; i < BN / 4; ++i) {
-        const float4 v = reinterpret_cast<const float4*>(my)[i];
-        acc[4 * i] = v.x; acc[4 * i + 1] = v.y; acc[4 * i + 2] = v.z; acc[4 * i + 3] = v.w;
-      }
-      for (int r = 1; r < S; ++r) {  // fixed split order
-        const uint32_t base = mapa_shared(smem_u32(my), static_cast<uint32_t>(r));
+        for (int i = 0; i < BN; ++i) v[i] = 0.f;
+        for (int s = 0; s < S; ++s) {  // fixed split order
+          const float4* src =
+              reinterpret_cast<const float4*>(p.part + (static_cast<int64_t>(s) * p.m_tiles * 128 + m0 + row) * BN);
 #pragma unroll
-        for (int i = 0; i < BN / 4; ++i) {
-          const float4 v = ld_cluster_f32x4(base + 16 * i);
-          acc[4 * i] += v.x; acc[4 * i + 1] += v.y; acc[4 * i + 2] += v.z; acc[4 * i + 3] += v.w;
-        }
-      }
-      if (S > 1) {
-        named_bar_sync(1, 128);
-        if (warp == 2 && lane == 0)
-          for (int r = 1; r < S; ++r) mbar_arrive_cluster(mapa_shared(smem_u32(&bars->red_done), static_cast<uint32_t>(r)));
-      }
-      const int grow = m0 + row;
-      if (p.out_mode == ADAPTER_ROWS_BF16) {
-        if (grow < p.Mm) {
-          uint16_t* o = static_cast<uint16_t*>(p.out) + static_cast<int64_t>(grow) * p.ld_out;
-#pragma unroll
-          for (int j = 0; j < BN; j += 8) {
-            if (j < p.r) {
-              uint4 w;
-              w.x = pack_bf16x2_rn(p.scale * acc[j], p.scale * acc[j + 1]);
-              w.y = pack_bf16x2_rn(p.scale * acc[j + 2], p.scale * acc[j + 3]);
-              w.z = pack_bf16x2_rn(p.scale * acc[j + 4], p.scale * acc[j + 5]);
-              w.w = pack_bf16x2_rn(p.scale * acc[j + 6], p.scale * acc[j + 7]);
-              *reinterpret_cast<uint4*>(o + j) = w;
-            }
+          for (int i = 0; i < BN / 4; ++i) {
+            const float4 w = __ldcg(src + i);
+            v[4 * i] += w.x; v[4 * i + 1] += w.y; v[4 * i + 2] += w.z; v[4 * i + 3] += w.w;
           }
         }
-      } else if (p.out_mode == ADAPTER_ROWS_F32) {
-        if (grow < p.Mm) {
-          float* o = static_cast<float*>(p.out) + static_cast<int64_t>(grow) * p.ld_out;
-#pragma unroll
-          for (int j = 0; j < BN; j += 4)
-            if (j < p.r) *reinterpret_cast<float4*>(o + j) = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
-        }
-      } else if (p.pool_L <= 1) {  // ADAPTER_COLS_F32 without pooling: out[j, m]
-        float* o = static_cast<float*>(p.out);
-        if (grow < p.Mm) {
-#pragma unroll
-          for (int j = 0; j < BN; ++j)
-            if (j < p.r) o[static_cast<int64_t>(j) * p.ld_out + grow] = acc[j];
-        }
-      } else {  // ADAPTER_COLS_F32 with group pooling: sum 32-row chunks per warp, then groups of L rows
-        float* chunk = red;  // this CTA's partial is consumed; reuse its space: [4 chunks][BN]
-        named_bar_sync(1, 128);
-#pragma unroll
-        for (int j = 0; j < BN; ++j) {
-          float v = grow < p.Mm ? acc[j] : 0.f;
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-          if (lane == 0) chunk[q * BN + j] = v;
-        }
-        named_bar_sync(1, 128);
-        const int per_group = p.pool_L / 32;  // chunks per group (L = 32, 64 or 128)
-        const int n_groups = 128 / p.pool_L;
-        for (int tid = threadIdx.x - 64; tid < n_groups * p.r; tid += 128) {
-          const int g = tid / p.r, j = tid % p.r;
-          float v = 0.f;
-          for (int c = 0; c < per_group; ++c) v += chunk[(g * per_group + c) * BN + j];
-          const int64_t og = (m0 / p.pool_L) + g;
-          if (og * p.pool_L < p.Mm)
-            static_cast<float*>(p.out)[static_cast<int64_t>(j) * p.ld_out + og] = v / static_cast<float>(p.pool_L);
-        }
+        adapter_store<BN>(p, v, m0, row, lane, q, bars);
+        if (row == 0) p.counters[tile] = 0;  // leave the counter ready for the next call
       }
+      named_bar_sync(1, 128);
     }
   }
 
@@ -289,27 +307,18 @@ cudaError_t launch_adapter_variant(const AdapterParams& p, const GemmMaps& maps,
     attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem + 1024);
   });
   if (attr_err != cudaSuccess) return attr_err;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(p.m_tiles * p.splits), 1, 1);
-  cfg.blockDim = dim3(kThreadsAdapter, 1, 1);
-  cfg.dynamicSmemBytes = C::kSmem + 1024;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = static_cast<unsigned>(p.splits);
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  const int items = p.m_tiles * p.splits;
+  const int grid = items < device_sm_count() ? items : device_sm_count();
   count_launch();
-  return cudaLaunchKernelEx(&cfg, kern, p, maps);
+  kern<<<grid, kThreadsAdapter, C::kSmem + 1024, st>>>(p, maps);
+  return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_adapter(int a_src, int b_src, int bn, const AdapterParams& p, const GemmMaps& maps,
                            cudaStream_t st) {
-  if (p.splits < 1 || p.splits > 8) return cudaErrorInvalidValue;
+  if (p.splits < 1 || p.splits > 64) return cudaErrorInvalidValue;
   if (a_src == A_TMA_K && b_src == B_TMA_K) {  // T = X A^T
     if (bn == 32) return launch_adapter_variant<A_TMA_K, B_TMA_K, 32>(p, maps, st);
     if (bn == 64) return launch_adapter_variant<A_TMA_K, B_TMA_K, 64>(p, maps, st);

@@ -57,9 +57,10 @@ struct GemmMaps {
   CUtensorMap a, b, a_tail, b_tail, codes;
 };
 
-// One adapter GEMM D[Mm, r] = sum_k A[Mm, k] B[k, r] (r <= 64), split along k over the CTAs of a
-// thread-block cluster whose leader sums the fp32 partials (distributed shared memory, split order)
-// and writes the result:
+// One adapter GEMM D[Mm, r] = sum_k A[Mm, k] B[k, r] (r <= 64).  The reduction is split into
+// `splits` parts for occupancy; each part's fp32 tile goes to `part`, and the last CTA to finish a
+// tile (a per-tile counter in `counters`, zero on entry and left zero on exit) sums the parts in
+// split order and writes the result:
 //   ADAPTER_ROWS_BF16   out[m, j] = bf16(scale * D[m, j])     (T_save, dT; ld_out = r)
 //   ADAPTER_ROWS_F32    out[m, j] = D[m, j]                   (dB; ld_out = r)
 //   ADAPTER_COLS_F32    out[j, m / L] = sum over m in a group of L of D[m, j] / L   (dA; ld_out = Ka)
@@ -68,7 +69,7 @@ enum AdapterOut : int { ADAPTER_ROWS_BF16 = 0, ADAPTER_ROWS_F32 = 1, ADAPTER_COL
 struct AdapterParams {
   int Mm, r;
   int n_steps;   // 64-wide reduction steps
-  int splits;    // CTAs per cluster (1..8), one output tile per cluster
+  int splits;
   int m_tiles;
   int b_atom;    // MN-major B: elements per swizzle atom row (32 or 64)
   int out_mode;
@@ -76,6 +77,8 @@ struct AdapterParams {
   int pool_L;    // ADAPTER_COLS_F32: group length (1 = none)
   void* out;
   int64_t ld_out;
+  float* part;       // [splits][m_tiles * 128][BN] fp32 (splits > 1)
+  int* counters;     // [m_tiles] (splits > 1)
   int32_t* status;
 };
 

@@ -55,13 +55,15 @@ constexpr long long kWaitCycles = 4000000000LL;  // ~2 s at the B200 boost clock
 constexpr uint32_t kSuspendNs = 200000;           // per try_wait
 
 // Waits for the phase with the given parity to complete.  Returns false (and raises
-// *abort) when the bound expires or another role already aborted.
+// *abort) when the bound expires or another role already aborted.  Polls try_wait without a
+// suspend hint: measured on B200, a suspended waiter is not resumed promptly when a TMA
+// transaction or a tcgen05.commit completes the phase, which adds microseconds to every handshake.
 QLR_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait_sleep(bar, parity, kSuspendNs)) return true;
-    if ((it & 15) == 0) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63) == 0) {
       if (*abort_flag) return false;
       if (clock64() - t0 > kWaitCycles) {
         *abort_flag = 1;
