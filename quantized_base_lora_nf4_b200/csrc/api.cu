@@ -145,7 +145,7 @@ size_t adapter_ws_bytes(int64_t Mm, int64_t n_red, int r) {
   const int64_t m_tiles = cdiv(Mm, 128);
   const int S = pick_splits(m_tiles, cdiv(n_red, 64));
   if (S == 1) return 0;
-  return align256(size_t(S) * m_tiles * 128 * adapter_bn(r) * 4) + align256(size_t(m_tiles) * 4);
+  return align256(size_t(S) * m_tiles * 128 * adapter_bn(r) * 4);
 }
 
 // One adapter GEMM: D[Mm, r] over n_red reduction elements, A and B from row-major matrices.
@@ -191,12 +191,10 @@ int run_adapter(const AdapterGemm& g, int r, int out_mode, float scale, int pool
   p.out = out;
   p.ld_out = ld_out;
   p.status = status;
-  if (p.splits > 1) {
-    p.part = reinterpret_cast<float*>(ws);
-    p.counters = reinterpret_cast<int*>(ws + align256(size_t(p.splits) * p.m_tiles * 128 * g.bn * 4));
-    if (cudaMemsetAsync(p.counters, 0, size_t(p.m_tiles) * 4, st) != cudaSuccess) return QLR_ERR_CUDA;
-  }
-  return cuda_rc(launch_adapter(g.a_src, g.b_src, g.bn, p, maps, st));
+  if (p.splits > 1) p.part = reinterpret_cast<float*>(ws);
+  if ((rc = cuda_rc(launch_adapter(g.a_src, g.b_src, g.bn, p, maps, st)))) return rc;
+  if (p.splits > 1) return cuda_rc(launch_adapter_reduce(p, g.bn, st));
+  return QLR_OK;
 }
 
 }  // namespace
@@ -309,7 +307,7 @@ int qlr_qalora_merge(const qlr_qweight* w, const uint16_t* A, const uint16_t* B,
 
 size_t qlr_forward_workspace_bytes(const qlr_qweight* w, int64_t M, int r, int pooled) {
   if (check_qweight(w) || M <= 0 || check_rank(r)) return 0;
-  // the group expansion of A (pooled adapter), then the split partial sums and tile counters
+  // the group expansion of A (pooled adapter), then the split partial sums
   return (pooled ? align256(size_t(r) * w->K * 2) : 0) + adapter_ws_bytes(M, w->K, r);
 }
 
@@ -406,7 +404,7 @@ int qlr_forward(const qlr_qweight* w, const uint16_t* X, int64_t M, const uint16
 size_t qlr_backward_lora_workspace_bytes(const qlr_qweight* w, int64_t M, int r, int pooled) {
   (void)pooled;
   if (check_qweight(w) || M <= 0 || check_rank(r)) return 0;
-  // split partial sums and tile counters of the three GEMMs, which run one after another
+  // split partial sums of the three GEMMs, which run one after another
   const size_t a = adapter_ws_bytes(M, w->N, r);
   const size_t b = adapter_ws_bytes(w->N, M, r);
   const size_t c = adapter_ws_bytes(w->K, M, r);

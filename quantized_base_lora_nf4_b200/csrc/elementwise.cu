@@ -4,6 +4,7 @@
 #include <cuda_bf16.h>
 
 #include "common.cuh"
+#include "gemm.cuh"
 #include "ptx.cuh"
 
 namespace qlr {
@@ -110,6 +111,38 @@ __global__ void reduce_splits_kernel(const float* __restrict__ part, int splits,
     static_cast<float*>(out)[o] = acc;
 }
 
+// Split-order sum of an adapter GEMM's parts + its output transform, one thread per output element
+// (for the pooled transposed output: one thread per (j, group), summing the group's L rows).
+__global__ void adapter_reduce_kernel(const AdapterParams p, int bn) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t split_stride = static_cast<int64_t>(p.m_tiles) * 128 * bn;
+  const int L = (p.out_mode == ADAPTER_COLS_F32 && p.pool_L > 1) ? p.pool_L : 1;
+  const int64_t rows_out = (p.Mm + L - 1) / L;
+  if (i >= rows_out * p.r) return;
+  int64_t orow, j;
+  if (p.out_mode == ADAPTER_COLS_F32) {  // consecutive threads walk output columns (coalesced stores)
+    j = i / rows_out;
+    orow = i % rows_out;
+  } else {
+    orow = i / p.r;
+    j = i % p.r;
+  }
+  float acc = 0.f;
+  for (int64_t m = orow * L; m < (orow + 1) * L && m < p.Mm; ++m) {
+    float sm = 0.f;
+    for (int s = 0; s < p.splits; ++s) sm += p.part[s * split_stride + m * bn + j];
+    acc += sm;
+  }
+  if (p.out_mode == ADAPTER_ROWS_BF16) {
+    static_cast<uint16_t*>(p.out)[orow * p.ld_out + j] =
+        static_cast<uint16_t>(pack_bf16x2_rn(p.scale * acc, 0.f) & 0xFFFFu);
+  } else if (p.out_mode == ADAPTER_ROWS_F32) {
+    static_cast<float*>(p.out)[orow * p.ld_out + j] = acc;
+  } else {
+    static_cast<float*>(p.out)[j * p.ld_out + orow] = L > 1 ? acc / static_cast<float>(L) : acc;
+  }
+}
+
 unsigned grid_for(int64_t n_items, int threads) {
   const int64_t want = (n_items + threads - 1) / threads;
   const int64_t cap = static_cast<int64_t>(device_sm_count()) * 8;
@@ -117,6 +150,15 @@ unsigned grid_for(int64_t n_items, int threads) {
 }
 
 }  // namespace
+
+cudaError_t launch_adapter_reduce(const AdapterParams& p, int bn, cudaStream_t st) {
+  const int L = (p.out_mode == ADAPTER_COLS_F32 && p.pool_L > 1) ? p.pool_L : 1;
+  const int64_t n = (static_cast<int64_t>(p.Mm) + L - 1) / L * p.r;
+  if (n == 0) return cudaSuccess;
+  count_launch();
+  adapter_reduce_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(p, bn);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_swiglu_fwd(const uint16_t* G, const uint16_t* U, uint16_t* H, int64_t n, cudaStream_t st) {
   if (n == 0) return cudaSuccess;

@@ -8,9 +8,9 @@
 // One persistent CTA per SM walks a static list of (tile, split) work items; a tile is 128 rows x BN.
 // Warp roles: 0 TMA producer (ring of A+B stages), 1 TMEM allocator + single-thread tcgen05.mma
 // issuer, 2..5 epilogue.  Two TMEM accumulators overlap an item's epilogue with the next item's main
-// loop.  With a split reduction each item's fp32 tile is stored to the workspace; the CTA that
-// finishes a tile last (per-tile atomic counter) sums all parts in split order -- deterministic --
-// and applies the output transform, so no separate reduction kernel is launched.
+// loop.  Without a split the epilogue applies the output transform directly; with one, each item's
+// fp32 tile goes to the workspace and `adapter_reduce_kernel` (elementwise.cu) sums the parts in
+// split order (deterministic) and applies the transform with one thread per output.
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -42,7 +42,6 @@ struct alignas(8) ABars {
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
-  int is_last;
   float chunk[4 * 64];
 };
 
@@ -263,27 +262,6 @@ __global__ void __launch_bounds__(kThreadsAdapter, 1)
 #pragma unroll
       for (int i = 0; i < BN / 4; ++i)
         reinterpret_cast<float4*>(mine)[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-      __threadfence();
-      named_bar_sync(1, 128);
-      if (row == 0) bars->is_last = (atomicAdd(p.counters + tile, 1) == S - 1);
-      named_bar_sync(1, 128);
-      if (bars->is_last) {  // uniform across the 128 epilogue threads
-        __threadfence();
-#pragma unroll
-        for (int i = 0; i < BN; ++i) v[i] = 0.f;
-        for (int s = 0; s < S; ++s) {  // fixed split order
-          const float4* src =
-              reinterpret_cast<const float4*>(p.part + (static_cast<int64_t>(s) * p.m_tiles * 128 + m0 + row) * BN);
-#pragma unroll
-          for (int i = 0; i < BN / 4; ++i) {
-            const float4 w = __ldcg(src + i);
-            v[4 * i] += w.x; v[4 * i + 1] += w.y; v[4 * i + 2] += w.z; v[4 * i + 3] += w.w;
-          }
-        }
-        adapter_store<BN>(p, v, m0, row, lane, q, bars);
-        if (row == 0) p.counters[tile] = 0;  // leave the counter ready for the next call
-      }
-      named_bar_sync(1, 128);
     }
   }
 

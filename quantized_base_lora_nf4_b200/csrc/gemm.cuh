@@ -57,10 +57,9 @@ struct GemmMaps {
   CUtensorMap a, b, a_tail, b_tail, codes;
 };
 
-// One adapter GEMM D[Mm, r] = sum_k A[Mm, k] B[k, r] (r <= 64).  The reduction is split into
-// `splits` parts for occupancy; each part's fp32 tile goes to `part`, and the last CTA to finish a
-// tile (a per-tile counter in `counters`, zero on entry and left zero on exit) sums the parts in
-// split order and writes the result:
+// One adapter GEMM D[Mm, r] = sum_k A[Mm, k] B[k, r] (r <= 64).  The reduction may be split into
+// `splits` parts for occupancy; each part's fp32 tile then goes to `part` and a reduction kernel
+// sums the parts in split order.  The result is written as:
 //   ADAPTER_ROWS_BF16   out[m, j] = bf16(scale * D[m, j])     (T_save, dT; ld_out = r)
 //   ADAPTER_ROWS_F32    out[m, j] = D[m, j]                   (dB; ld_out = r)
 //   ADAPTER_COLS_F32    out[j, m / L] = sum over m in a group of L of D[m, j] / L   (dA; ld_out = Ka)
@@ -78,12 +77,13 @@ struct AdapterParams {
   void* out;
   int64_t ld_out;
   float* part;       // [splits][m_tiles * 128][BN] fp32 (splits > 1)
-  int* counters;     // [m_tiles] (splits > 1)
   int32_t* status;
 };
 
 cudaError_t launch_adapter(int a_src, int b_src, int bn, const AdapterParams& p, const GemmMaps& maps,
                            cudaStream_t st);
+// Sums the split parts of an adapter GEMM in split order and applies its output transform.
+cudaError_t launch_adapter_reduce(const AdapterParams& p, int bn, cudaStream_t st);
 
 // Launches the fused dequant + tcgen05 kernel (a_src = A_DQ_K forward, A_DQ_MN input gradient).
 cudaError_t launch_fused(int a_src, int bn, const GemmParams& p, const GemmMaps& maps, cudaStream_t st);
