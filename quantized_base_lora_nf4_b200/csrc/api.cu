@@ -356,7 +356,8 @@ int qlr_forward_base(const qlr_qweight* w, const uint16_t* X, int64_t M, const u
   int32_t* stat = status_or_sink(status);
   const int64_t N = w->N, K = w->K;
   // Y = X dequant(W)^T + T_save B^T: fused dequant + tcgen05, computed as Y^T tiles (W rows on TMEM lanes)
-  const int bn_tok = M >= 192 ? 256 : 64;
+  const int tok = M >= 512 ? 512 : (M >= 192 ? 256 : 64);  // tokens per tile
+  const int bn_tok = tok == 512 ? 256 : tok;                // tokens per activation stage
   GemmMaps maps;
   std::memset(&maps, 0, sizeof(maps));
   if ((rc = make_tmap(&maps.codes, w->codes, 1, N, K / 2, 128, 32, 0))) return rc;
@@ -373,7 +374,7 @@ int qlr_forward_base(const qlr_qweight* w, const uint16_t* X, int64_t M, const u
   p.n_tail = static_cast<int>(cdiv(r, 64));
   p.r_tail = r;
   p.m_tiles = static_cast<int>(cdiv(N, 128));
-  p.n_tiles = static_cast<int>(cdiv(M, bn_tok));
+  p.n_tiles = static_cast<int>(cdiv(M, tok));
   p.b_atom = 64;
   p.out = Y;
   p.ldo = N;
@@ -383,7 +384,7 @@ int qlr_forward_base(const qlr_qweight* w, const uint16_t* X, int64_t M, const u
   p.tail_a_rows = N;
   p.tail_a_cols = r;
   p.status = stat;
-  return cuda_rc(launch_gemm(A_DQ_K, B_TMA_K, bn_tok, OUT_BF16_T, 0, p, maps, st));
+  return cuda_rc(launch_gemm(A_DQ_K, B_TMA_K, tok, OUT_BF16_T, 0, p, maps, st));
 }
 
 int qlr_forward(const qlr_qweight* w, const uint16_t* X, int64_t M, const uint16_t* A, const uint16_t* B, int r,
@@ -487,7 +488,8 @@ int qlr_backward_dx(const qlr_qweight* w, const uint16_t* dY, int64_t M, const u
   int32_t* stat = status_or_sink(status);
   const int64_t N = w->N, K = w->K;
   const uint16_t* At = A;
-  const int bn_tok = M >= 192 ? 256 : 64;
+  const int tok = M >= 512 ? 512 : (M >= 192 ? 256 : 64);  // tokens per tile
+  const int bn_tok = tok == 512 ? 256 : tok;                // tokens per activation stage
   GemmMaps maps;
   std::memset(&maps, 0, sizeof(maps));
   if ((rc = make_tmap(&maps.codes, w->codes, 1, N, K / 2, 64, 64, 0))) return rc;
@@ -504,7 +506,7 @@ int qlr_backward_dx(const qlr_qweight* w, const uint16_t* dY, int64_t M, const u
   p.n_tail = static_cast<int>(cdiv(r, 64));
   p.r_tail = r;
   p.m_tiles = static_cast<int>(cdiv(K, 128));
-  p.n_tiles = static_cast<int>(cdiv(M, bn_tok));
+  p.n_tiles = static_cast<int>(cdiv(M, tok));
   p.b_atom = 64;
   p.out = dX;
   p.ldo = K;
@@ -515,7 +517,7 @@ int qlr_backward_dx(const qlr_qweight* w, const uint16_t* dY, int64_t M, const u
   p.tail_a_cols = pooled ? K / w->group : K;
   p.tail_pool_L = pooled ? w->group : 0;
   p.status = stat;
-  return cuda_rc(launch_gemm(A_DQ_MN, B_TMA_K, bn_tok, OUT_BF16_T, 1, p, maps, st));
+  return cuda_rc(launch_gemm(A_DQ_MN, B_TMA_K, tok, OUT_BF16_T, 1, p, maps, st));
 }
 
 // ---- SwiGLU ---------------------------------------------------------------------------------------

@@ -111,35 +111,51 @@ __global__ void reduce_splits_kernel(const float* __restrict__ part, int splits,
     static_cast<float*>(out)[o] = acc;
 }
 
-// Split-order sum of an adapter GEMM's parts + its output transform, one thread per output element
-// (for the pooled transposed output: one thread per (j, group), summing the group's L rows).
+// Split-order sum of an adapter GEMM's parts + its output transform, one thread per output element.
 __global__ void adapter_reduce_kernel(const AdapterParams p, int bn) {
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t split_stride = static_cast<int64_t>(p.m_tiles) * 128 * bn;
-  const int L = (p.out_mode == ADAPTER_COLS_F32 && p.pool_L > 1) ? p.pool_L : 1;
-  const int64_t rows_out = (p.Mm + L - 1) / L;
-  if (i >= rows_out * p.r) return;
-  int64_t orow, j;
+  if (i >= static_cast<int64_t>(p.Mm) * p.r) return;
+  int64_t m, j;
   if (p.out_mode == ADAPTER_COLS_F32) {  // consecutive threads walk output columns (coalesced stores)
-    j = i / rows_out;
-    orow = i % rows_out;
+    j = i / p.Mm;
+    m = i % p.Mm;
   } else {
-    orow = i / p.r;
+    m = i / p.r;
     j = i % p.r;
   }
   float acc = 0.f;
-  for (int64_t m = orow * L; m < (orow + 1) * L && m < p.Mm; ++m) {
-    float sm = 0.f;
-    for (int s = 0; s < p.splits; ++s) sm += p.part[s * split_stride + m * bn + j];
-    acc += sm;
-  }
-  if (p.out_mode == ADAPTER_ROWS_BF16) {
-    static_cast<uint16_t*>(p.out)[orow * p.ld_out + j] =
-        static_cast<uint16_t>(pack_bf16x2_rn(p.scale * acc, 0.f) & 0xFFFFu);
-  } else if (p.out_mode == ADAPTER_ROWS_F32) {
-    static_cast<float*>(p.out)[orow * p.ld_out + j] = acc;
-  } else {
-    static_cast<float*>(p.out)[j * p.ld_out + orow] = L > 1 ? acc / static_cast<float>(L) : acc;
+  for (int s = 0; s < p.splits; ++s) acc += p.part[s * split_stride + m * bn + j];
+  if (p.out_mode == ADAPTER_ROWS_BF16)
+    static_cast<uint16_t*>(p.out)[m * p.ld_out + j] = static_cast<uint16_t>(pack_bf16x2_rn(p.scale * acc, 0.f) & 0xFFFFu);
+  else if (p.out_mode == ADAPTER_ROWS_F32)
+    static_cast<float*>(p.out)[m * p.ld_out + j] = acc;
+  else
+    static_cast<float*>(p.out)[j * p.ld_out + m] = acc;
+}
+
+// The pooled transposed output out[j, g] = (sum of the L rows of group g) / L: a block of 256 threads
+// covers 256 consecutive rows of one column j; each thread sums its row's splits, warps add their 32
+// rows by shuffles, and the group totals combine the warp sums (L = 32, 64 or 128 divides 256).
+__global__ void adapter_reduce_pooled_kernel(const AdapterParams p, int bn) {
+  __shared__ float warp_sum[8];
+  const int64_t split_stride = static_cast<int64_t>(p.m_tiles) * 128 * bn;
+  const int64_t blocks_per_col = (p.Mm + 255) / 256;
+  const int64_t j = blockIdx.x / blocks_per_col;
+  const int64_t m = (blockIdx.x % blocks_per_col) * 256 + threadIdx.x;
+  float v = 0.f;
+  if (m < p.Mm)
+    for (int s = 0; s < p.splits; ++s) v += p.part[s * split_stride + m * bn + j];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if ((threadIdx.x & 31) == 0) warp_sum[threadIdx.x >> 5] = v;
+  __syncthreads();
+  const int L = p.pool_L, wpg = L / 32;
+  if (threadIdx.x < 256 / L) {
+    float g = 0.f;
+    for (int w = 0; w < wpg; ++w) g += warp_sum[threadIdx.x * wpg + w];
+    const int64_t og = ((blockIdx.x % blocks_per_col) * 256) / L + threadIdx.x;
+    if (og * L < p.Mm) static_cast<float*>(p.out)[j * p.ld_out + og] = g / static_cast<float>(L);
   }
 }
 
@@ -152,8 +168,13 @@ unsigned grid_for(int64_t n_items, int threads) {
 }  // namespace
 
 cudaError_t launch_adapter_reduce(const AdapterParams& p, int bn, cudaStream_t st) {
-  const int L = (p.out_mode == ADAPTER_COLS_F32 && p.pool_L > 1) ? p.pool_L : 1;
-  const int64_t n = (static_cast<int64_t>(p.Mm) + L - 1) / L * p.r;
+  if (p.out_mode == ADAPTER_COLS_F32 && p.pool_L > 1) {
+    const int64_t blocks = (static_cast<int64_t>(p.Mm) + 255) / 256 * p.r;
+    count_launch();
+    adapter_reduce_pooled_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(p, bn);
+    return cudaGetLastError();
+  }
+  const int64_t n = static_cast<int64_t>(p.Mm) * p.r;
   if (n == 0) return cudaSuccess;
   count_launch();
   adapter_reduce_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(p, bn);

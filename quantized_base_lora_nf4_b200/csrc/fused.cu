@@ -87,10 +87,14 @@ __device__ __forceinline__ void copy_row64_pooled(const uint16_t* src_row, bool 
   }
 }
 
-template <int A_SRC, int BN>
+// PAIR: one tile covers 2 x BN tokens with both TMEM accumulators, so every dequantised weight
+// stage feeds twice the MMA work (the epilogue then does not overlap the next tile's main loop).
+template <int A_SRC, int BN, bool PAIR>
 __global__ void __launch_bounds__(kThreadsFused, 1)
     fused_kernel(const __grid_constant__ GemmParams p, const __grid_constant__ GemmMaps maps) {
   using C = FCfg<BN>;
+  constexpr int TOK = PAIR ? 2 * BN : BN;    // tokens per tile
+  constexpr int HALVES = PAIR ? 2 : 1;      // activation stages per reduction step
   constexpr bool MN = (A_SRC == A_DQ_MN);
   constexpr uint32_t kIdesc = idesc_bf16(128, BN, MN ? 1u : 0u, 0u);
   constexpr int NSA = C::NSA, NSB = C::NSB, NSC = C::NSC;
@@ -145,7 +149,7 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
   const int n_tiles_total = p.m_tiles * p.n_tiles;
   const int nmain = p.n_main, ntail = p.n_tail, nsteps = nmain + ntail;
   auto tile_m0 = [&](int tile) { return (tile / p.n_tiles) * 128; };
-  auto tile_n0 = [&](int tile) { return (tile % p.n_tiles) * BN; };
+  auto tile_n0 = [&](int tile) { return (tile % p.n_tiles) * TOK; };
 
   if (warp == 0) {
     // ------------------------------------------------------------------ activation producer
@@ -153,15 +157,18 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
       uint32_t j = 0;
       for (int tile = blockIdx.x; tile < n_tiles_total && !*abort_flag; tile += gridDim.x) {
         const int n0 = tile_n0(tile);
-        for (int ks = 0; ks < nsteps; ++ks, ++j) {
-          const int s = j % NSB;
-          if (!mbar_wait(&bars->b_empty[s], ((j / NSB) & 1) ^ 1, abort_flag)) break;
-          uint64_t* fb = &bars->b_full[s];
-          mbar_arrive_expect_tx(fb, C::kB);
-          if (ks < nmain)
-            tma_load_2d(ring_b + s * C::kB, &maps.b, ks * 64, n0, fb);
-          else
-            tma_load_2d(ring_b + s * C::kB, &maps.b_tail, (ks - nmain) * 64, n0, fb);
+        bool ok = true;
+        for (int ks = 0; ks < nsteps && ok; ++ks) {
+          for (int h = 0; h < HALVES; ++h, ++j) {
+            const int s = j % NSB;
+            if (!mbar_wait(&bars->b_empty[s], ((j / NSB) & 1) ^ 1, abort_flag)) { ok = false; break; }
+            uint64_t* fb = &bars->b_full[s];
+            mbar_arrive_expect_tx(fb, C::kB);
+            if (ks < nmain)
+              tma_load_2d(ring_b + s * C::kB, &maps.b, ks * 64, n0 + h * BN, fb);
+            else
+              tma_load_2d(ring_b + s * C::kB, &maps.b_tail, (ks - nmain) * 64, n0 + h * BN, fb);
+          }
         }
       }
       const uint32_t first = j > NSB ? j - NSB : 0;
@@ -196,33 +203,38 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      uint32_t j = 0;
+      uint32_t j = 0, jb = 0;  // A-ring steps, B-ring stages
       int it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < n_tiles_total && ok; tile += gridDim.x, ++it) {
-        const int acc = it & 1;
-        if (!mbar_wait(&bars->acc_empty[acc], ((it >> 1) & 1) ^ 1, abort_flag)) break;
+        const int acc = PAIR ? 0 : (it & 1);
+        const uint32_t acc_par = PAIR ? ((it & 1) ^ 1) : (((it >> 1) & 1) ^ 1);
+        if (!mbar_wait(&bars->acc_empty[acc], acc_par, abort_flag)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * BN;
-        for (int ks = 0; ks < nsteps; ++ks, ++j) {
-          const int sb = j % NSB, sa = j % NSA;
-          if (!mbar_wait(&bars->b_full[sb], (j / NSB) & 1, abort_flag)) { ok = false; break; }
+        for (int ks = 0; ks < nsteps && ok; ++ks, ++j) {
+          const int sa = j % NSA;
           if (!mbar_wait(&bars->a_full[sa], (j / NSA) & 1, abort_flag)) { ok = false; break; }
-          tc_fence_after();
           const uint32_t a_addr = smem_u32(ring_a + sa * C::kA);
-          const uint32_t b_addr = smem_u32(ring_b + sb * C::kB);
           int nsub = 4;
           if (ks >= nmain) {
             const int rem = p.r_tail - (ks - nmain) * 64;
             nsub = rem >= 64 ? 4 : (rem + 15) / 16;
           }
-          for (int kk = 0; kk < nsub; ++kk) {
-            const uint64_t ad = MN ? smem_desc(a_addr + kk * 2048, 8192, 1024, kSw128)
-                                   : smem_desc(a_addr + kk * 32, 16, 1024, kSw128);
-            const uint64_t bd = smem_desc(b_addr + kk * 32, 16, 1024, kSw128);
-            umma_bf16_ss(d_tmem, ad, bd, kIdesc, (ks > 0 || kk > 0) ? 1u : 0u);
+          for (int h = 0; h < HALVES; ++h, ++jb) {
+            const int sb = jb % NSB;
+            if (!mbar_wait(&bars->b_full[sb], (jb / NSB) & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t b_addr = smem_u32(ring_b + sb * C::kB);
+            const uint32_t d_tmem = tmem_base + (PAIR ? h : acc) * BN;
+            for (int kk = 0; kk < nsub; ++kk) {
+              const uint64_t ad = MN ? smem_desc(a_addr + kk * 2048, 8192, 1024, kSw128)
+                                     : smem_desc(a_addr + kk * 32, 16, 1024, kSw128);
+              const uint64_t bd = smem_desc(b_addr + kk * 32, 16, 1024, kSw128);
+              umma_bf16_ss(d_tmem, ad, bd, kIdesc, (ks > 0 || kk > 0) ? 1u : 0u);
+            }
+            umma_commit(&bars->b_empty[sb]);
           }
-          umma_commit(&bars->b_empty[sb]);
+          if (!ok) break;
           umma_commit(&bars->a_empty[sa]);
         }
         if (!ok) break;
@@ -239,15 +251,16 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
     int it = 0;
     for (int tile = blockIdx.x; tile < n_tiles_total; tile += gridDim.x, ++it) {
       const int m0 = tile_m0(tile), n0 = tile_n0(tile);
-      const int acc = it & 1;
-      const bool got = mbar_wait(&bars->acc_full[acc], (it >> 1) & 1, abort_flag);
+      const int acc = PAIR ? 0 : (it & 1);
+      const uint32_t acc_par = PAIR ? (it & 1) : ((it >> 1) & 1);
+      const bool got = mbar_wait(&bars->acc_full[acc], acc_par, abort_flag);
       __syncwarp();
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c = 0; c < TOK / 32; ++c) {  // PAIR: accumulator columns 0..2*BN-1 are tokens n0 .. n0+2*BN-1
         uint32_t v[32];
-        tmem_ld_32x32b_x32(tmem_base + acc * BN + c * 32 + ((q * 32) << 16), v);
+        tmem_ld_32x32b_x32(tmem_base + (PAIR ? 0 : acc * BN) + c * 32 + ((q * 32) << 16), v);
         tmem_ld_wait();
         eng::store_chunk_bf16_t(v, stg, lane, n0 + c * 32, m0 + q * 32, p);
       }
@@ -361,10 +374,10 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
   if (threadIdx.x == 0 && bars->abort_flag) report(p.status, QLR_ERR_TIMEOUT);
 }
 
-template <int A_SRC, int BN>
+template <int A_SRC, int BN, bool PAIR>
 cudaError_t launch_fused_variant(const GemmParams& p, const GemmMaps& maps, cudaStream_t st) {
   using C = FCfg<BN>;
-  auto kern = fused_kernel<A_SRC, BN>;
+  auto kern = fused_kernel<A_SRC, BN, PAIR>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [&] {
@@ -380,12 +393,15 @@ cudaError_t launch_fused_variant(const GemmParams& p, const GemmMaps& maps, cuda
 
 }  // namespace
 
+// bn = tokens per tile: 512 (paired 256-column accumulators), 256 or 64.
 cudaError_t launch_fused(int a_src, int bn, const GemmParams& p, const GemmMaps& maps, cudaStream_t st) {
   if (p.splits != 1) return cudaErrorNotSupported;
-  if (a_src == A_DQ_K && bn == 256) return launch_fused_variant<A_DQ_K, 256>(p, maps, st);
-  if (a_src == A_DQ_K && bn == 64) return launch_fused_variant<A_DQ_K, 64>(p, maps, st);
-  if (a_src == A_DQ_MN && bn == 256) return launch_fused_variant<A_DQ_MN, 256>(p, maps, st);
-  if (a_src == A_DQ_MN && bn == 64) return launch_fused_variant<A_DQ_MN, 64>(p, maps, st);
+  if (a_src == A_DQ_K && bn == 512) return launch_fused_variant<A_DQ_K, 256, true>(p, maps, st);
+  if (a_src == A_DQ_K && bn == 256) return launch_fused_variant<A_DQ_K, 256, false>(p, maps, st);
+  if (a_src == A_DQ_K && bn == 64) return launch_fused_variant<A_DQ_K, 64, false>(p, maps, st);
+  if (a_src == A_DQ_MN && bn == 512) return launch_fused_variant<A_DQ_MN, 256, true>(p, maps, st);
+  if (a_src == A_DQ_MN && bn == 256) return launch_fused_variant<A_DQ_MN, 256, false>(p, maps, st);
+  if (a_src == A_DQ_MN && bn == 64) return launch_fused_variant<A_DQ_MN, 64, false>(p, maps, st);
   return cudaErrorNotSupported;
 }
 

@@ -58,14 +58,14 @@ def test_tiny_layer(cuda_lib):
     run_and_check(cuda_lib, wl.linears[0], wl.M, accumulate_check=True)
 
 
-@pytest.mark.parametrize("M", [1, 40, 200, 333])
+@pytest.mark.parametrize("M", [1, 40, 200, 333, 700])
 @pytest.mark.parametrize("r", [8, 16, 32, 64])
 def test_ragged_nf4(cuda_lib, M, r):
     spec = LinearSpec("w", 320, 384, "nfk", 4, 128, 0, r=r, s=0.5)
     run_and_check(cuda_lib, spec, M, seed=M + r)
 
 
-@pytest.mark.parametrize("M", [64, 300])
+@pytest.mark.parametrize("M", [64, 300, 1100])
 def test_ragged_int4_pooled(cuda_lib, M):
     spec = LinearSpec("w", 264, 512, "int4g", group=32, r=16, s=1.0, pooled=True)
     run_and_check(cuda_lib, spec, M, seed=7)
