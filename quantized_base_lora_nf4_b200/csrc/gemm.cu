@@ -29,7 +29,6 @@ struct ACfg {
   static constexpr int kB = BN * 128;
   static constexpr int kStage = ((kA + kB) + 1023) / 1024 * 1024;
   static constexpr int kStages = 8;
-  static constexpr int kScratch = 4 * BN * 4 + 64;  // per-warp chunk sums + flags
   static constexpr int kSmem = kStages * kStage + 2048;
   static constexpr int kTmemCols = (2 * BN <= 64) ? 64 : 128;
 };
