@@ -202,6 +202,30 @@ QLR_API int qlr_backward_lora(const qlr_qweight* w, const uint16_t* X, const uin
                       const uint16_t* B, int64_t M, int r, float s, int pooled, float* dA, float* dB,
                       uint16_t* dT_out, void* workspace, size_t workspace_bytes, int32_t* status, void* stream);
 
+/* Size in bytes of the scratch array built into the library for qlr_backward_lora_noalloc: one per
+ * GPU that loads the library, held until the process exits. */
+#define QLR_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/*
+ * qlr_backward_lora for callers that cannot allocate device memory (the pages have no counterpart:
+ * this is a property of the library's interface, not of the method).  Such callers include a
+ * framework that owns all device memory through its own pool, a runtime with a fixed memory plan,
+ * and latency-critical loops that must not pay cudaMalloc/cudaFree.  Same arguments, results and
+ * errors as qlr_backward_lora, without workspace: the split partial sums go to a scratch array of
+ * QLR_NOALLOC_SCRATCH_BYTES compiled into the library.  It allocates nothing.
+ *   - A problem whose workspace would exceed QLR_NOALLOC_SCRATCH_BYTES is rejected with
+ *     QLR_ERR_WORKSPACE before anything is launched.
+ *   - The array's device address is looked up once per GPU, on the first call made while that GPU
+ *     is current; make that first call outside any stream capture.
+ *   - All calls share the array and leave their partial sums in it (nothing needs to start at zero).
+ *     Calls that can overlap on the GPU -- different streams, or several host threads -- race on it
+ *     and must be serialised by the caller.
+ */
+QLR_API int qlr_backward_lora_noalloc(const qlr_qweight* w, const uint16_t* X, const uint16_t* dY,
+                                      const uint16_t* T_save, const uint16_t* B, int64_t M, int r, float s,
+                                      int pooled, float* dA, float* dB, uint16_t* dT_out, int32_t* status,
+                                      void* stream);
+
 /*
  * Input gradient through the frozen quantised weight (QLoRA explainer, "The contribution":
  * backpropagate through the frozen 4-bit weights into the adapters):

@@ -29,7 +29,7 @@ EXPORTED = (
     "qlr_quantize_int4_group", "qlr_dequant", "qlr_qalora_merge", "qlr_forward_workspace_bytes", "qlr_forward",
     "qlr_backward_lora_workspace_bytes", "qlr_backward_lora", "qlr_backward_dx_workspace_bytes",
     "qlr_backward_dx", "qlr_swiglu_forward", "qlr_swiglu_backward", "qlr_device_sm_count", "qlr_lora_down",
-    "qlr_forward_base", "qlr_launch_count",
+    "qlr_forward_base", "qlr_launch_count", "qlr_backward_lora_noalloc",
 )
 
 
@@ -80,6 +80,7 @@ def lib() -> ctypes.CDLL:
         "qlr_lora_down": (I, [QP, P, I64, P, I, F, I, P, P, SZ, P, P]),
         "qlr_forward_base": (I, [QP, P, I64, P, I, P, P, P, P]),
         "qlr_launch_count": (ctypes.c_uint64, []),
+        "qlr_backward_lora_noalloc": (I, [QP, P, P, P, P, I64, I, F, I, P, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
