@@ -46,7 +46,7 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="qalora", choices=["qalora", "tiny", "mlp7b"])
+    ap.add_argument("--workload", default="qalora", choices=["qalora", "tiny", "mlp7b", "decode70b"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -353,6 +353,55 @@ def oracle_tokens_per_s(wl, seed, budget_s=12.0):
                       f"({el:.1f} s; dequantised weights prepared untimed)"}
 
 
+# ------------------------------------------------------------------------------------------ decode shape
+def run_decode(args, dev):
+    """Forward of the 28672 x 8192 NF4+DQ projection at 1, 4 and 16 tokens: HBM-bound on the codes."""
+    import numpy as np
+    import torch
+    from quantized_base_lora_nf4_b200 import qlr
+    from synth import workload, linear_tensors, normal
+
+    peaks, peak_kind = load_peaks()
+    wl = workload("decode70b", args.seed)
+    spec = wl.linears[0]
+    t = linear_tensors(spec, 16, seed=args.seed, with_dy=False)
+    W = torch.from_numpy(t["W"]).to(dev)
+    q = qlr.quantize_nf4(W, 4, 64, 256)
+    del W
+    bf = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev).to(torch.bfloat16).contiguous()  # noqa
+    A, B = bf(t["A"]), bf(t["B"])
+    code_bytes = spec.N * spec.K // 2
+    all_bytes = code_bytes + spec.N * spec.K // 64 + 4 * spec.N * spec.K // (64 * 256) + 2 * spec.r * (spec.N + spec.K)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    out = {}
+    for M in wl.token_counts:
+        X = bf(t["X"][:M])
+        ws = qlr.Workspace(dev)
+        T = torch.empty((M, spec.r), dtype=torch.bfloat16, device=dev)
+        Y = torch.empty((M, spec.N), dtype=torch.bfloat16, device=dev)
+        def fwd():
+            qlr.lora_down(q, X, A, spec.s, T_save=T, ws=ws)
+            qlr.forward_base(q, X, B, T, Y=Y)
+        for _ in range(args.warmup):
+            fwd()
+        torch.cuda.synchronize()
+        ms = []
+        for _ in range(args.steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fwd()
+            e1.record()
+            ms.append((e0, e1))
+        torch.cuda.synchronize()
+        t_ms = statistics.median(a.elapsed_time(b) for a, b in ms)
+        out[str(M)] = {"ms": t_ms, "code_GBps": code_bytes / t_ms / 1e6, "all_GBps": all_bytes / t_ms / 1e6,
+                       "code_frac_of_hbm": code_bytes / t_ms / 1e6 / float(peaks["hbm_gbs"])}
+    return {"workload": "decode70b: NF4+DQ 28672x8192, r=64, forward at 1/4/16 tokens", "per_tokens": out,
+            "hbm_peak_gbs": float(peaks["hbm_gbs"]), "peak_kind": peak_kind,
+            "code_bytes": code_bytes, "all_bytes": all_bytes}
+
+
 # ------------------------------------------------------------------------------------------ main
 def main():
     args = parse()
@@ -393,6 +442,14 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     dev = torch.device("cuda", local if world > 1 else 0)
     torch.cuda.set_device(dev)
+    if args.workload == "decode70b":
+        if rank == 0:
+            print(json.dumps({"metric": "decode forward time and HBM GB/s on the 4-bit code bytes",
+                              **run_decode(args, dev)}))
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return 0
     res = run_ours(args, rank, world, dev)
     if world > 1:
         import torch.distributed as dist

@@ -113,3 +113,25 @@ def test_zero_tokens(cuda_lib):
     dA, dB, dT = qlr.backward_lora(q, X, dY, T, bf16_dev(t["B"]), 1.0)
     torch.cuda.synchronize()
     assert Y.shape == (0, 128) and float(dA.abs().sum()) == 0 and float(dB.abs().sum()) == 0
+
+
+@pytest.mark.parametrize("M", [1, 4, 16])
+def test_decode_projection_full_size_sampled_rows(cuda_lib, M):
+    """The 28672 x 8192 NF4+DQ projection at decode token counts (the HBM-bound decode kernel):
+    output features checked on whole double-quantisation groups of sampled weight rows."""
+    qlr = cuda_lib
+    wl = workload("decode70b")
+    spec = wl.linears[0]
+    t = linear_tensors(spec, 16, seed=0, with_dy=False)
+    q = qlr.quantize_nf4(f32_dev(t["W"]), 4, 64, 256)
+    X = t["X"][:M]
+    Y, T = qlr.forward(q, bf16_dev(X), bf16_dev(t["A"]), bf16_dev(t["B"]), spec.s)
+    torch.cuda.synchronize()
+    Yh = host(Y)
+    rows = np.sort(np.random.default_rng(M).choice(spec.N // 2, 48, replace=False)) * 2
+    sel = np.concatenate([[r, r + 1] for r in rows])
+    Wdq = np.concatenate([Q.dequant_nfk(Q.quantize_nfk(t["W"][r:r + 2], 4, 64, 256)) for r in rows])
+    ref = OL.forward(X, np.zeros((2 * len(rows), spec.K)), t["A"], t["B"][sel], spec.s)["Y"] + \
+        X.astype(np.float64) @ Wdq.astype(np.float64).T
+    assert OL.rel_fro(Yh[:, sel], ref) <= TOL
+    assert OL.rel_fro(host(T), spec.s * OL.forward(X, np.zeros((1, spec.K)), t["A"], t["B"][:1], spec.s)["T"]) <= TOL
