@@ -356,8 +356,7 @@ int qlr_forward_base(const qlr_qweight* w, const uint16_t* X, int64_t M, const u
   int32_t* stat = status_or_sink(status);
   const int64_t N = w->N, K = w->K;
   // a few tokens of a 4-bit NF weight: the HBM-bound decode kernel
-  if (M <= 16 && w->fmt == QLR_FMT_NFK && w->bits == 4 && K % 128 == 0)
-    return cuda_rc(launch_decode(w, X, M, B, r, T_save, Y, st));
+  if (decode_supported(w, M)) return cuda_rc(launch_decode(w, X, M, B, r, T_save, Y, stat, st));
   // Y = X dequant(W)^T + T_save B^T: fused dequant + tcgen05, computed as Y^T tiles (W rows on TMEM lanes)
   const int tok = M >= 512 ? 512 : (M >= 192 ? 256 : 64);  // tokens per tile
   const int bn_tok = tok == 512 ? 256 : tok;                // tokens per activation stage

@@ -40,9 +40,10 @@ cudaError_t launch_reduce_splits(const float* part, int splits, int64_t rows, in
 
 int device_sm_count();
 
-// Decode-shape forward (1..16 tokens) of a 4-bit NF weight (decode.cu).
+// Decode-shape forward (1..16 tokens) of a 4-bit NF weight with double quantisation (decode.cu).
+bool decode_supported(const qlr_qweight* w, int64_t M);
 cudaError_t launch_decode(const qlr_qweight* w, const uint16_t* X, int64_t M, const uint16_t* B, int r,
-                          const uint16_t* T_save, uint16_t* Y, cudaStream_t st);
+                          const uint16_t* T_save, uint16_t* Y, int32_t* status, cudaStream_t st);
 
 // Counts kernel launches issued by this library (reported by qlr_launch_count).
 void count_launch(int n = 1);

@@ -135,3 +135,11 @@ def test_decode_projection_full_size_sampled_rows(cuda_lib, M):
         X.astype(np.float64) @ Wdq.astype(np.float64).T
     assert OL.rel_fro(Yh[:, sel], ref) <= TOL
     assert OL.rel_fro(host(T), spec.s * OL.forward(X, np.zeros((1, spec.K)), t["A"], t["B"][:1], spec.s)["T"]) <= TOL
+
+
+@pytest.mark.parametrize("M", [1, 5, 16])
+@pytest.mark.parametrize("block,r", [(64, 8), (128, 64)])
+def test_decode_ragged(cuda_lib, M, block, r):
+    """Decode kernel on a weight whose rows do not fill the last 64-row CTA."""
+    spec = LinearSpec("w", 320, 384, "nfk", 4, block, 256, r=r, s=0.5)
+    run_and_check(cuda_lib, spec, M, seed=11 + M)
