@@ -2,22 +2,22 @@
 //
 // At a few tokens the layer is a matrix-vector product bound by the HBM read of the packed 4-bit
 // codes (QLoRA explainer, "The complete QLoRA forward pass": each frozen NF4 block is dequantised to
-// bf16 on the fly and multiplied by the input).  A CTA owns 64 weight rows: a producer warp streams
-// every 128-wide reduction step -- the rows' codes (64 x 64 bytes, 64-byte swizzle) and the input
-// tile (16 tokens x 128, 128-byte swizzle) -- by TMA into a ring of 5-6 shared-memory slots, and four
-// compute warps (16 rows each) consume it.  The block constants of the 64 rows are staged in shared
-// memory once.  448 CTAs of 160 threads cover a 28672-row weight in one wave.
+// bf16 on the fly and multiplied by the input).  One persistent CTA per SM owns a contiguous range of
+// 16-row units (about 12 for a 28672-row weight on 148 SMs), one compute warp per unit; a producer
+// warp streams every 128-wide reduction step -- each unit's codes (16 rows x 64 bytes, 64-byte
+// swizzle) and the input tile (tokens x 128, 128-byte swizzle) -- by TMA into a ring of shared-memory
+// slots that all compute warps consume in step.
 //
-// Per step a lane takes, for rows g and g+8 of its warp, 16 codes of each of the step's two 64-code
-// halves.  Codes become bf16 NF4 levels through a byte-permute table lookup and
-// feed mma.sync m16n8k16 (weight rows on the M side, tokens on the N side, fp32 accumulate); the
-// reduction index is permuted consistently for the weight and the input, and every MMA stays inside
-// one block, so each block's partial dot products are scaled by the block's constant
-// fp32(E4M3(c1_8)) * s2 (or c1) once and added to the accumulator.  The effective weight is therefore
-// bf16(level) * scale, rounded once less than the bf16(level * scale) the tensor-core GEMMs use.
+// A code byte (two 4-bit codes) becomes the bf16 pair (level[lo], level[hi]) with one shared-memory
+// load from a 256-entry table replicated per lane (conflict-free), which is exactly one mma.sync
+// m16n8k16 A-register.  The weight rows are the MMA's M side, tokens its N side, fp32 accumulate;
+// the reduction index is permuted consistently for weight and input, every MMA stays inside one
+// block, and each block's partial sums are scaled once by fp32(E4M3(c1_8)) * s2.  The effective weight
+// is bf16(level) * scale: one rounding fewer than the bf16(level * scale) of the tensor-core GEMMs.
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "common.cuh"
@@ -28,8 +28,10 @@ namespace qlr {
 
 namespace {
 
-constexpr int kComputeWarps = 4;                 // 64 weight rows per CTA, 16 per warp
-constexpr int kThreads = (kComputeWarps + 1) * 32;  // + one TMA producer warp
+constexpr int kMaxUnits = 14;                        // 16-row units per CTA
+constexpr int kComputeWarps = 2 * kMaxUnits;         // two per unit, one per 64-wide half of each step
+constexpr int kThreads = (kComputeWarps + 1) * 32;   // + one TMA producer warp
+constexpr int kPartBytes = kMaxUnits * 32 * 8 * 4;   // second-half partial sums, [unit][lane][8] fp32
 
 struct DecodeParams {
   const uint8_t* c1_fp8;
@@ -37,6 +39,8 @@ struct DecodeParams {
   int block_shift;          // log2 of the block (64 or 128)
   int64_t N, K;
   int M;
+  int units;                // ceil(N / 16)
+  int nu_lo;                // every CTA owns nu_lo or nu_lo + 1 (<= kMaxUnits) units
   const uint16_t* B;        // [N, r] bf16
   const uint16_t* T_save;   // [M, r] bf16
   int r;
@@ -46,204 +50,293 @@ struct DecodeParams {
 };
 
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-struct Lut16 {
-  uint32_t l0, l1, l2, l3, h0, h1, h2, h3;
-};
-
-// 4 codes (low 16 bits of w) -> two bf16x2 words, code 0 in the low half of the first.
-__device__ __forceinline__ void lut4(const Lut16& t, uint32_t w, uint32_t& o0, uint32_t& o1) {
-  const uint32_t sel = w & 0x7777u;
-  const uint32_t sel2 = ((w >> 1) & 0x4444u) | 0x3210u;
-  const uint32_t lo = prmt(prmt(t.l0, t.l1, sel), prmt(t.l2, t.l3, sel), sel2);
-  const uint32_t hi = prmt(prmt(t.h0, t.h1, sel), prmt(t.h2, t.h3, sel), sel2);
-  o0 = prmt(lo, hi, 0x5140);
-  o1 = prmt(lo, hi, 0x7362);
-}
-
 template <int NT>
 struct DCfg {
-  static constexpr int kCodes = 64 * 64;            // [64 rows][64 bytes] of codes per step
-  static constexpr int kXHalf = 8 * NT * 128;        // [8 NT tokens][64 bf16] per half step
-  static constexpr int kSlot = kCodes + 2 * kXHalf;  // 1 KB multiple
+  static constexpr int kXHalf = 8 * NT * 128;                   // [8 NT tokens][64 bf16]
+  static constexpr int kSlot = kMaxUnits * 1024 + 2 * kXHalf;   // codes of every unit + input tile
   static constexpr int kSlots = NT == 1 ? 6 : 5;
 };
 
-// Shared-memory bytes after the ring: E4M3 bytes of 64 rows, the s2 values they use, barriers.
-inline int decode_scale_bytes(int64_t bpr) { return static_cast<int>((64 * bpr + 1023) / 1024 * 1024) + 2048; }
+// Shared-memory map, as shared-window addresses.  The dequantisation table sits at 64 KB so that one
+// byte permute of (code word, 4 lane | 64 KB) yields the address of a table entry; the block
+// constants and barriers fill the space below it and the TMA ring starts at 128 KB.
+constexpr uint32_t kLutAddr = 0x10000;   // [256 code bytes][256 B: 32 lanes x bf16x2, 128 B unused]
+constexpr uint32_t kRingAddr = 0x20000;
+constexpr uint32_t kBarBytes = 1024;
 
 struct alignas(8) DBars {
-  uint64_t full[8];
-  uint64_t empty[8];
+  uint64_t full[6];
+  uint64_t empty[6];
   int abort_flag;
 };
 
+// Barriers, s2 values, second-half partial sums, then E4M3 bytes [16 kMaxUnits rows][bpr + 4].
+__host__ __device__ inline uint32_t decode_const_bytes(int64_t bpr) {
+  const uint64_t c8 = 16ull * kMaxUnits * (bpr + 4);
+  const uint64_t s2 = ((16ull * kMaxUnits * bpr) / 256 + 4) * 4;
+  return static_cast<uint32_t>(kBarBytes + (s2 + 1023) / 1024 * 1024 + kPartBytes + c8);
+}
+
+// The dynamic window starts at some address of at most 1 KB (reserved shared memory), so a window of
+// kRingAddr + ring bytes reaches past the ring whatever that start is.
+inline size_t decode_smem_bytes(int nt) {
+  return kRingAddr + static_cast<size_t>(nt == 1 ? DCfg<1>::kSlots * DCfg<1>::kSlot : DCfg<2>::kSlots * DCfg<2>::kSlot);
+}
+
+// The table is written once before the first barrier and only read afterwards, so its loads may be
+// scheduled freely (no volatile); the ring loads stay ordered after their barrier waits.
+__device__ __forceinline__ uint32_t lds_table(uint32_t addr) {
+  uint32_t v;
+  asm("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ uint2 lds_v2(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds_u8(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u8 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ float lds_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+  return v;
+}
+
 // NT: token tiles of 8 (1: M <= 8, 2: M <= 16).
 template <int NT>
-__global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant__ DecodeParams p,
-                                                          const __grid_constant__ CUtensorMap tm_codes,
-                                                          const __grid_constant__ CUtensorMap tm_x) {
+__global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_constant__ DecodeParams p,
+                                                             const __grid_constant__ CUtensorMap tm_codes_lo,
+                                                             const __grid_constant__ CUtensorMap tm_codes_hi,
+                                                             const __grid_constant__ CUtensorMap tm_x) {
   using C = DCfg<NT>;
-  constexpr int NSL = C::kSlots;
+  constexpr int kSlots = C::kSlots;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* ring = smem;
-  const int64_t bpr = p.K >> p.block_shift;      // blocks per row
-  uint8_t* s_c8 = smem + NSL * C::kSlot;        // [64 rows][blocks per row] E4M3 bytes
-  float* s_s2 = reinterpret_cast<float*>(s_c8 + (64 * bpr + 1023) / 1024 * 1024);  // <= 64 bpr / 256 + 2 values
-  DBars* bars = reinterpret_cast<DBars*>(reinterpret_cast<uint8_t*>(s_s2) + 1024);
+  const uint32_t base = smem_u32(smem_raw);
+  const int64_t bpr = p.K >> p.block_shift;  // blocks per row
+  const int c8_stride = static_cast<int>(bpr) + 4;
+  const uint32_t bars_addr = (base + 1023u) & ~1023u;
+  const uint32_t s2_addr = bars_addr + kBarBytes;
+  const uint32_t part_addr = s2_addr + ((16u * kMaxUnits * static_cast<uint32_t>(bpr)) / 256u * 4u + 16u + 1023u) / 1024u * 1024u;
+  const uint32_t c8_addr = part_addr + kPartBytes;
+  if (bars_addr + decode_const_bytes(bpr) > kLutAddr) {  // the window starts higher than assumed
+    if (threadIdx.x == 0) report(p.status, QLR_ERR_UNSUPPORTED);
+    return;
+  }
+  auto gen = [&](uint32_t addr) { return smem_raw + (addr - base); };  // generic pointer of a shared address
+  DBars* bars = reinterpret_cast<DBars*>(gen(bars_addr));
+  uint32_t* lut = reinterpret_cast<uint32_t*>(gen(kLutAddr));
+  uint8_t* s_c8 = gen(c8_addr);
+  float* s_s2 = reinterpret_cast<float*>(gen(s2_addr));
   volatile int* abort_flag = &bars->abort_flag;
-
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * 64;
+
+  // this CTA's contiguous range of 16-row units
+  const int u_begin = static_cast<int>((static_cast<int64_t>(blockIdx.x) * p.units) / gridDim.x);
+  const int u_end = static_cast<int>((static_cast<int64_t>(blockIdx.x + 1) * p.units) / gridDim.x);
   const int nsteps = static_cast<int>(p.K / 128);
-  const int64_t s2_first = (row0 * bpr) >> 8;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < NSL; ++s) {
+    for (int s = 0; s < kSlots; ++s) {
       mbar_init(&bars->full[s], 1);
       mbar_init(&bars->empty[s], kComputeWarps);
     }
     bars->abort_flag = 0;
     fence_barrier_init();
   }
-  // block constants of this CTA's 64 rows, once
-  {
-    const int64_t rows = (p.N - row0) < 64 ? (p.N - row0) : 64;
-    const int64_t n8 = rows * bpr;
-    for (int64_t i = threadIdx.x; i < n8; i += kThreads) s_c8[i] = __ldg(p.c1_fp8 + row0 * bpr + i);
-    const int64_t n2 = (((row0 + rows) * bpr - 1) >> 8) - s2_first + 1;
-    for (int64_t i = threadIdx.x; i < n2; i += kThreads) s_s2[i] = __ldg(p.s2 + s2_first + i);
+  // code byte e -> (bf16 level[e & 15], bf16 level[e >> 4]), one copy per lane at 64 KB + 256 e + 4 lane
+  for (int i = threadIdx.x; i < 256 * 32; i += kThreads) {
+    const int e = i >> 5;
+    lut[e * 64 + (i & 31)] = pack_bf16x2_rn(p.lv.v[e & 15], p.lv.v[e >> 4]);
   }
-  __syncthreads();
 
-  if (warp == kComputeWarps) {
-    // ------------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      tma_prefetch_desc(&tm_codes);
-      tma_prefetch_desc(&tm_x);
-      int s = 0;
-      for (; s < nsteps; ++s) {
-        const int sl = s % NSL;
-        if (!mbar_wait(&bars->empty[sl], ((s / NSL) & 1) ^ 1, abort_flag)) break;
-        uint8_t* slot = ring + sl * C::kSlot;
-        mbar_arrive_expect_tx(&bars->full[sl], C::kSlot);
-        tma_load_2d(slot, &tm_codes, s * 64, static_cast<int32_t>(row0), &bars->full[sl]);
-        tma_load_2d(slot + C::kCodes, &tm_x, s * 128, 0, &bars->full[sl]);
-        tma_load_2d(slot + C::kCodes + C::kXHalf, &tm_x, s * 128 + 64, 0, &bars->full[sl]);
+  __syncthreads();  // barriers and table ready
+
+  {
+    const uint32_t jslot = 0;
+    const int nu = u_end - u_begin;  // nu_lo or nu_lo + 1, at most kMaxUnits (host grid sizing)
+    const int64_t prow0 = static_cast<int64_t>(u_begin) * 16;
+    const int prows = static_cast<int>(static_cast<int64_t>(nu) * 16 < p.N - prow0 ? nu * 16 : p.N - prow0);
+    const int64_t s2_first = (prow0 * bpr) >> 8;
+
+    if (warp == kComputeWarps) {
+      // ---------------------------------------------------------------- TMA producer
+      // one box of all this CTA's rows (16 nu x 64 B of codes) and two input halves per step
+      if (lane == 0) {
+        const CUtensorMap* tm_codes = nu == p.nu_lo ? &tm_codes_lo : &tm_codes_hi;
+        tma_prefetch_desc(tm_codes);
+        tma_prefetch_desc(&tm_x);
+        for (int s = 0; s < nsteps; ++s) {
+          const uint32_t j = jslot + s;
+          const int sl = j % kSlots;
+          if (!mbar_wait(&bars->empty[sl], ((j / kSlots) & 1) ^ 1, abort_flag)) break;
+          uint8_t* slot = gen(kRingAddr + sl * C::kSlot);
+          mbar_arrive_expect_tx(&bars->full[sl], nu * 1024 + 2 * C::kXHalf);
+          tma_load_2d(slot, tm_codes, s * 64, static_cast<int32_t>(prow0), &bars->full[sl]);
+          tma_load_2d(slot + kMaxUnits * 1024, &tm_x, s * 128, 0, &bars->full[sl]);
+          tma_load_2d(slot + kMaxUnits * 1024 + C::kXHalf, &tm_x, s * 128 + 64, 0, &bars->full[sl]);
+        }
       }
-      const int first = s > NSL ? s - NSL : 0;  // drain the loads still in flight
-      for (int q = first; q < s; ++q) {
-        volatile int never = 0;
-        mbar_wait(&bars->full[q % NSL], (q / NSL) & 1, &never);
+    } else {
+      // ---------------------------------------------------------------- compute warps
+      // stage the block constants of this CTA's rows (the compute warps alone, so the producer can start)
+      for (int lr = warp; lr < prows; lr += kComputeWarps)
+        for (int b = lane; b < bpr; b += 32) s_c8[lr * c8_stride + b] = __ldg(p.c1_fp8 + (prow0 + lr) * bpr + b);
+      {
+        const int n2 = static_cast<int>((((prow0 + prows) * bpr - 1) >> 8) - s2_first + 1);
+        for (int i = threadIdx.x; i < n2; i += kComputeWarps * 32) s_s2[i] = __ldg(p.s2 + s2_first + i);
       }
-    }
-  } else {
-    // ------------------------------------------------------------------ compute warps
-    const int g = lane >> 2, t = lane & 3;
-    const int lr_a = warp * 16 + g, lr_b = lr_a + 8;     // local rows 0..63
-    const int64_t ra = row0 + lr_a, rb = row0 + lr_b;
-    const bool va = ra < p.N, vb = rb < p.N;
-    Lut16 lut;
-    {
-      uint32_t pk[8];
+      named_bar_sync(1, kComputeWarps * 32);
+      const int g = lane >> 2, t = lane & 3;
+      const int unit = warp >> 1, hh = warp & 1;  // this warp's unit and half (64 codes) of every step
+      const bool active = unit < nu;
+      // MMA row g reads weight row pi(g) of the unit (bits 1 and 2 of g swapped), which spreads the eight
+      // byte code loads of each half-warp over all 32 banks under the 64-byte swizzle
+      const int pg = (g & 1) | ((g & 2) << 1) | ((g & 4) >> 1);
+      const int lr_a = unit * 16 + pg, lr_b = lr_a + 8;  // rows of this CTA, 0 .. 16 nu - 1
+      const int64_t ra = prow0 + lr_a, rb = prow0 + lr_b;
+      const bool va = active && ra < p.N, vb = active && rb < p.N;
+      const uint32_t lut_lane = kLutAddr | (4u * lane);
+      // per-lane parts of the shared addresses that do not change from step to step
+      // codes: 16-byte chunk 2 hh + t/2 of the row, 64-byte swizzle; input: chunks 2t, 2t+1 of a 128-byte row
+      const uint32_t code_a = unit * 1024 + pg * 64 + 8 * (t & 1), code_b = code_a + 8 * 64;
+      const uint32_t chunk_a = (((2 * hh + (t >> 1)) ^ ((pg >> 1) & 3)) << 4);
+      const uint32_t chunk_b = (((2 * hh + (t >> 1)) ^ (((pg + 8) >> 1) & 3)) << 4);
+      const uint32_t c8_a = c8_addr + lr_a * c8_stride, c8_b = c8_addr + lr_b * c8_stride;
+      const uint32_t s2_off = static_cast<uint32_t>((prow0 * bpr) & 255);
+      const uint32_t s2_a = lr_a * static_cast<uint32_t>(bpr) + s2_off, s2_b = lr_b * static_cast<uint32_t>(bpr) + s2_off;
+      const int bshift = p.block_shift;
+      float acc[NT][4];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) pk[j] = pack_bf16x2_rn(p.lv.v[2 * j], p.lv.v[2 * j + 1]);
-      lut.l0 = prmt(pk[0], pk[1], 0x6420); lut.h0 = prmt(pk[0], pk[1], 0x7531);
-      lut.l1 = prmt(pk[2], pk[3], 0x6420); lut.h1 = prmt(pk[2], pk[3], 0x7531);
-      lut.l2 = prmt(pk[4], pk[5], 0x6420); lut.h2 = prmt(pk[4], pk[5], 0x7531);
-      lut.l3 = prmt(pk[6], pk[7], 0x6420); lut.h3 = prmt(pk[6], pk[7], 0x7531);
-    }
-    auto scale = [&](int lr, int64_t b) -> float {  // fp32(E4M3(c1_8)) * s2 of block b of local row lr
-      const __half_raw hr =
-          __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(s_c8[lr * bpr + b]), __NV_E4M3);
-      return __fmul_rn(__half2float(__half(hr)), s_s2[(((row0 + lr) * bpr + b) >> 8) - s2_first]);
-    };
-    float acc[NT][4];
-#pragma unroll
-    for (int n = 0; n < NT; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
-    for (int s = 0; s < nsteps; ++s) {
-      const int sl = s % NSL;
-      const bool ok = mbar_wait(&bars->full[sl], (s / NSL) & 1, abort_flag);
-      if (!__all_sync(0xffffffffu, ok)) break;
-      const uint8_t* codes = ring + sl * C::kSlot;
-      const uint8_t* xs = codes + C::kCodes;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        // 64-byte swizzled code rows: 16-byte chunk c of row r sits at chunk c ^ ((r >> 1) & 3)
-        const int c = 2 * h + (t >> 1);
-        const uint2 wa = *reinterpret_cast<const uint2*>(codes + lr_a * 64 + ((c ^ ((lr_a >> 1) & 3)) << 4) + 8 * (t & 1));
-        const uint2 wb = *reinterpret_cast<const uint2*>(codes + lr_b * 64 + ((c ^ ((lr_b >> 1) & 3)) << 4) + 8 * (t & 1));
-        const uint8_t* xh = xs + h * C::kXHalf;
-        float part[NT][4];
-#pragma unroll
-        for (int n = 0; n < NT; ++n) part[n][0] = part[n][1] = part[n][2] = part[n][3] = 0.f;
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          // this lane's codes: k = 128 s + 64 h + 16 t + i; MMA m takes i = 4m .. 4m+3
-          uint32_t a[4];
-          lut4(lut, (m < 2 ? wa.x : wa.y) >> (16 * (m & 1)), a[0], a[2]);
-          lut4(lut, (m < 2 ? wb.x : wb.y) >> (16 * (m & 1)), a[1], a[3]);
+      for (int n = 0; n < NT; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+      for (int s = 0; s < nsteps; ++s) {
+        const uint32_t j = jslot + s;
+        const int sl = j % kSlots;
+        const bool ok = mbar_wait(&bars->full[sl], (j / kSlots) & 1, abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        // copy this step's ring data (this half's codes and input) to registers, then free the slot
+        const uint32_t slot = kRingAddr + sl * C::kSlot;  // codes [unit][16 rows][64 B] (64-byte swizzle), then X
+        uint2 wa, wb;
+        uint4 xv[NT][2];
+        if (active) {
+          wa = lds_v2(slot + code_a + chunk_a);
+          wb = lds_v2(slot + code_b + chunk_b);
+          // input X[tok][64 hh + 16 t .. +15]: two 16-byte chunks of a 128-byte swizzled row
 #pragma unroll
           for (int n = 0; n < NT; ++n) {
-            // 128-byte swizzled input rows: X[tok][16 t + 4 m .. +3] at chunk (2t + m/2) ^ (tok & 7)
             const int tok = 8 * n + g;
-            const int ch = (2 * t + (m >> 1)) ^ (tok & 7);
-            const uint2 xv = *reinterpret_cast<const uint2*>(xh + tok * 128 + (ch << 4) + 8 * (m & 1));
-            mma_bf16_16816(part[n], a, xv.x, xv.y);
+            const uint32_t xr = slot + kMaxUnits * 1024 + hh * C::kXHalf + tok * 128;
+            if (tok < p.M) {  // rows past the last token are zero; skipping them saves shared-memory wavefronts
+              xv[n][0] = lds_v4(xr + (((2 * t) ^ (tok & 7)) << 4));
+              xv[n][1] = lds_v4(xr + (((2 * t + 1) ^ (tok & 7)) << 4));
+            } else {
+              xv[n][0] = xv[n][1] = make_uint4(0u, 0u, 0u, 0u);
+            }
           }
         }
-        const int64_t b = (static_cast<int64_t>(s) * 128 + 64 * h) >> p.block_shift;
-        const float sa = va ? scale(lr_a, b) : 0.f;
-        const float sb = vb ? scale(lr_b, b) : 0.f;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->empty[sl]);
+        if (active) {
+          float part[NT][4];
+#pragma unroll
+          for (int n = 0; n < NT; ++n) part[n][0] = part[n][1] = part[n][2] = part[n][3] = 0.f;
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            // this lane's codes: k = 128 s + 64 hh + 16 t + i; MMA m takes i = 4m .. 4m+3 (bytes 2m, 2m+1)
+            const uint32_t qa = m < 2 ? wa.x : wa.y, qb = m < 2 ? wb.x : wb.y;
+            // byte permute: address bytes 0, 2, 3 from (4 lane | 64 KB), byte 1 = the code byte
+            constexpr uint32_t kSelLo[2] = {0x7604u, 0x7624u}, kSelHi[2] = {0x7614u, 0x7634u};
+            uint32_t af[4];
+            af[0] = lds_table(__byte_perm(qa, lut_lane, kSelLo[m & 1]));
+            af[2] = lds_table(__byte_perm(qa, lut_lane, kSelHi[m & 1]));
+            af[1] = lds_table(__byte_perm(qb, lut_lane, kSelLo[m & 1]));
+            af[3] = lds_table(__byte_perm(qb, lut_lane, kSelHi[m & 1]));
+#pragma unroll
+            for (int n = 0; n < NT; ++n) {
+              const uint4 x4 = xv[n][m >> 1];
+              mma_bf16_16816(part[n], af, (m & 1) ? x4.z : x4.x, (m & 1) ? x4.w : x4.y);
+            }
+          }
+          const uint32_t b = static_cast<uint32_t>((s * 128 + 64 * hh) >> bshift);
+          float sa = 0.f, sb = 0.f;
+          if (va) {
+            const __half_raw hr = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(lds_u8(c8_a + b)), __NV_E4M3);
+            sa = __fmul_rn(__half2float(__half(hr)), lds_f32(s2_addr + ((s2_a + b) >> 8) * 4));
+          }
+          if (vb) {
+            const __half_raw hr = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(lds_u8(c8_b + b)), __NV_E4M3);
+            sb = __fmul_rn(__half2float(__half(hr)), lds_f32(s2_addr + ((s2_b + b) >> 8) * 4));
+          }
+#pragma unroll
+          for (int n = 0; n < NT; ++n) {
+            acc[n][0] = fmaf(sa, part[n][0], acc[n][0]);
+            acc[n][1] = fmaf(sa, part[n][1], acc[n][1]);
+            acc[n][2] = fmaf(sb, part[n][2], acc[n][2]);
+            acc[n][3] = fmaf(sb, part[n][3], acc[n][3]);
+          }
+        }
+      }
+      // the second-half warp hands its sums to the first-half warp of the same unit
+      float* s_part = reinterpret_cast<float*>(gen(part_addr)) + (unit * 32 + lane) * 8;
+      if (active && hh == 1) {
+#pragma unroll
+        for (int n = 0; n < NT; ++n)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) s_part[4 * n + e] = acc[n][e];
+      }
+      named_bar_sync(1, kComputeWarps * 32);
+      if (active && hh == 0) {
+#pragma unroll
+        for (int n = 0; n < NT; ++n)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[n][e] += s_part[4 * n + e];
+        // adapter term: rows of B (16 x r) times T_save^T (r x tokens), r/16 more MMAs
+        for (int kr = 0; kr < p.r; kr += 16) {
+          const bool hi_ok = kr + 8 < p.r;  // r = 8: the upper eight slots are zero
+          const uint32_t* ba = reinterpret_cast<const uint32_t*>(p.B + ra * p.r + kr);
+          const uint32_t* bb = reinterpret_cast<const uint32_t*>(p.B + rb * p.r + kr);
+          uint32_t a[4];
+          a[0] = va ? __ldg(ba + t) : 0u;
+          a[1] = vb ? __ldg(bb + t) : 0u;
+          a[2] = (va && hi_ok) ? __ldg(ba + t + 4) : 0u;
+          a[3] = (vb && hi_ok) ? __ldg(bb + t + 4) : 0u;
+#pragma unroll
+          for (int n = 0; n < NT; ++n) {
+            const int tok = 8 * n + g;
+            uint32_t b0 = 0, b1 = 0;
+            if (tok < p.M) {
+              const uint32_t* tp = reinterpret_cast<const uint32_t*>(p.T_save + static_cast<int64_t>(tok) * p.r + kr);
+              b0 = __ldg(tp + t);
+              b1 = hi_ok ? __ldg(tp + t + 4) : 0u;
+            }
+            mma_bf16_16816(acc[n], a, b0, b1);
+          }
+        }
 #pragma unroll
         for (int n = 0; n < NT; ++n) {
-          acc[n][0] = fmaf(sa, part[n][0], acc[n][0]);
-          acc[n][1] = fmaf(sa, part[n][1], acc[n][1]);
-          acc[n][2] = fmaf(sb, part[n][2], acc[n][2]);
-          acc[n][3] = fmaf(sb, part[n][3], acc[n][3]);
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->empty[sl]);
-    }
-
-    // adapter term: rows of B (16 x r) times T_save^T (r x tokens), r/16 more MMAs
-    for (int kr = 0; kr < p.r; kr += 16) {
-      const bool hi_ok = kr + 8 < p.r;  // r = 8: the upper eight slots are zero
-      const uint32_t* ba = reinterpret_cast<const uint32_t*>(p.B + ra * p.r + kr);
-      const uint32_t* bb = reinterpret_cast<const uint32_t*>(p.B + rb * p.r + kr);
-      uint32_t a[4];
-      a[0] = va ? __ldg(ba + t) : 0u;
-      a[1] = vb ? __ldg(bb + t) : 0u;
-      a[2] = (va && hi_ok) ? __ldg(ba + t + 4) : 0u;
-      a[3] = (vb && hi_ok) ? __ldg(bb + t + 4) : 0u;
 #pragma unroll
-      for (int n = 0; n < NT; ++n) {
-        const int tok = 8 * n + g;
-        uint32_t b0 = 0, b1 = 0;
-        if (tok < p.M) {
-          const uint32_t* tp = reinterpret_cast<const uint32_t*>(p.T_save + static_cast<int64_t>(tok) * p.r + kr);
-          b0 = __ldg(tp + t);
-          b1 = hi_ok ? __ldg(tp + t + 4) : 0u;
-        }
-        mma_bf16_16816(acc[n], a, b0, b1);
-      }
-    }
-#pragma unroll
-    for (int n = 0; n < NT; ++n) {
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int tok = 8 * n + 2 * t + e;
-        if (tok < p.M) {
-          if (va) p.Y[static_cast<int64_t>(tok) * p.N + ra] = static_cast<uint16_t>(pack_bf16x2_rn(acc[n][e], 0.f) & 0xFFFFu);
-          if (vb) p.Y[static_cast<int64_t>(tok) * p.N + rb] = static_cast<uint16_t>(pack_bf16x2_rn(acc[n][2 + e], 0.f) & 0xFFFFu);
+          for (int e = 0; e < 2; ++e) {
+            const int tok = 8 * n + 2 * t + e;
+            if (tok < p.M) {
+              if (va) p.Y[static_cast<int64_t>(tok) * p.N + ra] = static_cast<uint16_t>(pack_bf16x2_rn(acc[n][e], 0.f) & 0xFFFFu);
+              if (vb) p.Y[static_cast<int64_t>(tok) * p.N + rb] = static_cast<uint16_t>(pack_bf16x2_rn(acc[n][2 + e], 0.f) & 0xFFFFu);
+            }
+          }
         }
       }
     }
@@ -253,27 +346,26 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
 }
 
 template <int NT>
-cudaError_t launch_decode_variant(const DecodeParams& p, const CUtensorMap& tc, const CUtensorMap& tx,
-                                  cudaStream_t st) {
-  using C = DCfg<NT>;
-  const int smem = C::kSlots * C::kSlot + decode_scale_bytes(p.K >> p.block_shift) + 1024;
+cudaError_t launch_decode_variant(const DecodeParams& p, int grid, const CUtensorMap& tc_lo, const CUtensorMap& tc_hi,
+                                  const CUtensorMap& tx, cudaStream_t st) {
+  const size_t smem = decode_smem_bytes(NT);
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [&] {
     attr_err = cudaFuncSetAttribute(decode_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
   });
   if (attr_err != cudaSuccess) return attr_err;
-  const unsigned grid = static_cast<unsigned>((p.N + 63) / 64);
   count_launch();
-  decode_kernel<NT><<<grid, kThreads, smem, st>>>(p, tc, tx);
+  decode_kernel<NT><<<grid, kThreads, smem, st>>>(p, tc_lo, tc_hi, tx);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 bool decode_supported(const qlr_qweight* w, int64_t M) {
-  return M >= 1 && M <= 16 && w->fmt == QLR_FMT_NFK && w->bits == 4 && w->dq_block == 256 && w->K % 128 == 0 &&
-         w->K <= 32768;
+  if (M < 1 || M > 16 || w->fmt != QLR_FMT_NFK || w->bits != 4 || w->dq_block != 256 || w->K % 128) return false;
+  // the constants fit below the table when the window starts within its first kilobyte
+  return 1024 + decode_const_bytes(w->K / w->block) <= kLutAddr && decode_smem_bytes(M <= 8 ? 1 : 2) <= 227 * 1024;
 }
 
 cudaError_t launch_decode(const qlr_qweight* w, const uint16_t* X, int64_t M, const uint16_t* B, int r,
@@ -285,6 +377,13 @@ cudaError_t launch_decode(const qlr_qweight* w, const uint16_t* X, int64_t M, co
   p.N = w->N;
   p.K = w->K;
   p.M = static_cast<int>(M);
+  p.units = static_cast<int>((w->N + 15) / 16);
+  // one CTA per SM, each owning a contiguous run of units; more CTAs only when a run would exceed kMaxUnits
+  const int sms = device_sm_count();
+  int grid = p.units < sms ? p.units : sms;
+  if (grid < (p.units + kMaxUnits - 1) / kMaxUnits) grid = (p.units + kMaxUnits - 1) / kMaxUnits;
+  p.nu_lo = p.units / grid;
+  const int nu_hi = std::min({p.nu_lo + 1, kMaxUnits, p.units});
   p.B = B;
   p.T_save = T_save;
   p.r = r;
@@ -292,10 +391,12 @@ cudaError_t launch_decode(const qlr_qweight* w, const uint16_t* X, int64_t M, co
   p.lv = levels_for(4);
   p.status = status;
   const int nt = M <= 8 ? 1 : 2;
-  CUtensorMap tc, tx;
-  if (make_tmap(&tc, w->codes, 1, w->N, w->K / 2, 64, 64, 64)) return cudaErrorInvalidValue;
+  CUtensorMap tc_lo, tc_hi, tx;
+  if (make_tmap(&tc_lo, w->codes, 1, w->N, w->K / 2, 16 * p.nu_lo, 64, 64)) return cudaErrorInvalidValue;
+  if (make_tmap(&tc_hi, w->codes, 1, w->N, w->K / 2, 16 * nu_hi, 64, 64)) return cudaErrorInvalidValue;
   if (make_tmap(&tx, X, 2, M, w->K, 8 * nt, 64, 128)) return cudaErrorInvalidValue;
-  return nt == 1 ? launch_decode_variant<1>(p, tc, tx, st) : launch_decode_variant<2>(p, tc, tx, st);
+  return nt == 1 ? launch_decode_variant<1>(p, grid, tc_lo, tc_hi, tx, st)
+                 : launch_decode_variant<2>(p, grid, tc_lo, tc_hi, tx, st);
 }
 
 }  // namespace qlr
