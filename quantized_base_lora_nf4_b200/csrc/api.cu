@@ -3,6 +3,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cstring>
 #include <mutex>
@@ -88,11 +89,23 @@ int check_qweight(const qlr_qweight* w) {
 int check_gemm_weight(const qlr_qweight* w) {
   int rc = check_qweight(w);
   if (rc) return rc;
-  if (w->fmt == QLR_FMT_NFK && w->bits != 4) return QLR_ERR_UNSUPPORTED;
   if (w->K % 64 || w->N % 8) return QLR_ERR_SHAPE;
+  // 3-bit codes are loaded two 64-code steps per box along K (a 24-byte box width is not legal)
+  if (w->fmt == QLR_FMT_NFK && w->bits == 3 && w->K % 128) return QLR_ERR_SHAPE;
   if (w->fmt == QLR_FMT_NFK && w->K % w->block) return QLR_ERR_SHAPE;
   if (w->N > (int64_t(1) << 30) || w->K > (int64_t(1) << 30)) return QLR_ERR_SHAPE;
   return QLR_OK;
+}
+
+// Width of the packed codes: NF-k codes are k bits, INT4 group codes 4.
+int code_bits(const qlr_qweight* w) { return w->fmt == QLR_FMT_NFK ? w->bits : 4; }
+
+// The fused kernel's codes ring: a 32 KB region split into at most 8 slots of one TMA box each.
+void set_code_ring(GemmParams& p, int bits, int steps_per_box, int box_bytes) {
+  p.code_bits = bits;
+  p.code_steps = steps_per_box;
+  p.code_box_bytes = box_bytes;
+  p.code_slots = std::min(8, 32768 / box_bytes);
 }
 
 int check_rank(int r) { return (r == 8 || r == 16 || r == 32 || r == 64) ? QLR_OK : QLR_ERR_SHAPE; }
@@ -362,7 +375,9 @@ int qlr_forward_base(const qlr_qweight* w, const uint16_t* X, int64_t M, const u
   const int bn_tok = tok == 512 ? 256 : tok;                // tokens per activation stage
   GemmMaps maps;
   std::memset(&maps, 0, sizeof(maps));
-  if ((rc = make_tmap(&maps.codes, w->codes, 1, N, K / 2, 128, 32, 0))) return rc;
+  const int kb = code_bits(w);
+  const int csteps = kb == 3 ? 2 : 1;  // 64-code steps per codes box
+  if ((rc = make_tmap(&maps.codes, w->codes, 1, N, K * kb / 8, 128, 8 * kb * csteps, 0))) return rc;
   if ((rc = make_tmap(&maps.b, X, 2, M, K, bn_tok, 64, 128))) return rc;
   if ((rc = make_tmap(&maps.b_tail, T_save, 2, M, r, bn_tok, 64, 128))) return rc;
   maps.a = maps.b;
@@ -378,6 +393,7 @@ int qlr_forward_base(const qlr_qweight* w, const uint16_t* X, int64_t M, const u
   p.m_tiles = static_cast<int>(cdiv(N, 128));
   p.n_tiles = static_cast<int>(cdiv(M, tok));
   p.b_atom = 64;
+  set_code_ring(p, kb, csteps, 128 * 8 * kb * csteps);
   p.out = Y;
   p.ldo = N;
   p.accumulate = 0;
@@ -494,7 +510,8 @@ int qlr_backward_dx(const qlr_qweight* w, const uint16_t* dY, int64_t M, const u
   const int bn_tok = tok == 512 ? 256 : tok;                // tokens per activation stage
   GemmMaps maps;
   std::memset(&maps, 0, sizeof(maps));
-  if ((rc = make_tmap(&maps.codes, w->codes, 1, N, K / 2, 64, 64, 0))) return rc;
+  const int kb = code_bits(w);
+  if ((rc = make_tmap(&maps.codes, w->codes, 1, N, K * kb / 8, 64, 16 * kb, 0))) return rc;
   if ((rc = make_tmap(&maps.b, dY, 2, M, N, bn_tok, 64, 128))) return rc;
   if ((rc = make_tmap(&maps.b_tail, dT, 2, M, r, bn_tok, 64, 128))) return rc;
   maps.a = maps.b;
@@ -510,6 +527,7 @@ int qlr_backward_dx(const qlr_qweight* w, const uint16_t* dY, int64_t M, const u
   p.m_tiles = static_cast<int>(cdiv(K, 128));
   p.n_tiles = static_cast<int>(cdiv(M, tok));
   p.b_atom = 64;
+  set_code_ring(p, kb, 1, 64 * 16 * kb);
   p.out = dX;
   p.ldo = K;
   p.accumulate = accumulate ? 1 : 0;

@@ -1,5 +1,6 @@
-// Device building blocks shared by the tcgen05 GEMM kernels: the 4-bit dequantiser (16-entry bf16
-// table per block or group, byte-permute lookups) and the epilogue stores.
+// Device building blocks shared by the tcgen05 GEMM kernels: the dequantiser (2-, 3- and 4-bit codes
+// unpacked to 4-bit fields, a 16-entry bf16 table per block or group, byte-permute lookups) and the
+// epilogue stores.
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -101,18 +102,65 @@ __device__ __forceinline__ Lut int4_lut_c(uint32_t sc_bits16, uint32_t z_bits16)
   return make_lut(v);
 }
 
-// Dequantise 64 consecutive 4-bit codes (one row of W, its scale data in `c`) into the eight 16-byte
-// chunks of one 128-byte swizzled shared-memory row at `dst_row` (`sw` = row index for the swizzle).
-__device__ __forceinline__ void dequant_row64(const DqParams& dq, const uint8_t* codes_smem, const DqConst& c,
+// 2-bit fields i = 0..7 of a 16-bit word -> 4-bit fields (field i at bits 4i..4i+3).
+__device__ __forceinline__ uint32_t spread2to4(uint32_t x) {
+  x = (x | (x << 8)) & 0x00FF00FFu;
+  x = (x | (x << 4)) & 0x0F0F0F0Fu;
+  return (x | (x << 2)) & 0x33333333u;
+}
+
+// bits t = 0..7 of a byte -> bit 4t.
+__device__ __forceinline__ uint32_t spread1to4(uint32_t x) {
+  x = (x | (x << 12)) & 0x000F000Fu;
+  x = (x | (x << 6)) & 0x03030303u;
+  return (x | (x << 3)) & 0x11111111u;
+}
+
+// The 64 codes of one run, unpacked to eight words of eight 4-bit codes (code 8q + i at bits 4i of
+// word q).  Packed layouts (little-endian): k = 4 two codes per byte, low nibble first (32 bytes,
+// 16-byte aligned); k = 2 four codes per byte, code 4j + t at bits 2t (16 bytes, 16-byte aligned);
+// k = 3 bit planes, per 32 codes three 32-bit words, word p holding bit p of code t at bit t (24 bytes,
+// 8-byte aligned).
+__device__ __forceinline__ void load_codes64(const uint8_t* src, int bits, uint32_t (&w)[8]) {
+  if (bits == 4) {
+    const uint4 c0 = reinterpret_cast<const uint4*>(src)[0], c1 = reinterpret_cast<const uint4*>(src)[1];
+    w[0] = c0.x; w[1] = c0.y; w[2] = c0.z; w[3] = c0.w;
+    w[4] = c1.x; w[5] = c1.y; w[6] = c1.z; w[7] = c1.w;
+  } else if (bits == 2) {
+    const uint4 c = *reinterpret_cast<const uint4*>(src);
+    const uint32_t q[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      w[2 * i] = spread2to4(q[i] & 0xFFFFu);
+      w[2 * i + 1] = spread2to4(q[i] >> 16);
+    }
+  } else {
+    const uint2 a = reinterpret_cast<const uint2*>(src)[0], b = reinterpret_cast<const uint2*>(src)[1],
+                c = reinterpret_cast<const uint2*>(src)[2];
+    const uint32_t pl[2][3] = {{a.x, a.y, b.x}, {b.y, c.x, c.y}};
+#pragma unroll
+    for (int gi = 0; gi < 2; ++gi)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int sh = 8 * j;
+        w[4 * gi + j] = spread1to4((pl[gi][0] >> sh) & 0xFFu) | (spread1to4((pl[gi][1] >> sh) & 0xFFu) << 1) |
+                        (spread1to4((pl[gi][2] >> sh) & 0xFFu) << 2);
+      }
+  }
+}
+
+// Dequantise 64 consecutive codes (one run of a row of W, `bits` wide, its scale data in `c`) into
+// the eight 16-byte chunks of one 128-byte swizzled shared-memory row at `dst_row` (`sw` = row index
+// for the swizzle).
+__device__ __forceinline__ void dequant_row64(const DqParams& dq, const uint8_t* codes_smem, int bits, const DqConst& c,
                                               bool valid, uint8_t* dst_row, int sw) {
-  const uint4* src = reinterpret_cast<const uint4*>(codes_smem);
-  const uint4 c0 = src[0], c1 = src[1];
-  const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
   if (!valid) {
 #pragma unroll
     for (int k = 0; k < 8; ++k) *reinterpret_cast<uint4*>(dst_row + ((k ^ sw) << 4)) = make_uint4(0, 0, 0, 0);
     return;
   }
+  uint32_t w[8];
+  load_codes64(codes_smem, bits, w);
   if (dq.fmt == QLR_FMT_NFK) {
     const Lut t = nf_lut_c(dq, c);
 #pragma unroll

@@ -122,7 +122,7 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
     }
     for (int s = 0; s < NSC; ++s) {
       mbar_init(&bars->c_full[s], 1);
-      mbar_init(&bars->c_empty[s], 128);
+      mbar_init(&bars->c_empty[s], 128 * p.code_steps);  // every step of a box is one dequantiser group
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&bars->acc_full[a], 1);
@@ -180,24 +180,25 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
   } else if (warp == 14) {
     // ------------------------------------------------------------------ codes producer
     if (lane == 0) {
-      uint32_t jc = 0;
+      const int ncs = p.code_slots, kb = p.code_bits;
+      uint32_t jc = 0;  // boxes
       for (int tile = blockIdx.x; tile < n_tiles_total && !*abort_flag; tile += gridDim.x) {
         const int m0 = tile_m0(tile);
-        for (int ks = 0; ks < nmain; ++ks, ++jc) {
-          const int s = jc % NSC;
-          if (!mbar_wait(&bars->c_empty[s], ((jc / NSC) & 1) ^ 1, abort_flag)) break;
+        for (int ks = 0; ks < nmain; ks += p.code_steps, ++jc) {
+          const int s = jc % ncs;
+          if (!mbar_wait(&bars->c_empty[s], ((jc / ncs) & 1) ^ 1, abort_flag)) break;
           uint64_t* fb = &bars->c_full[s];
-          mbar_arrive_expect_tx(fb, C::kC);
-          if (!MN)
-            tma_load_2d(ring_c + s * C::kC, &maps.codes, ks * 32, m0, fb);   // [128 W rows][32 bytes]
-          else
-            tma_load_2d(ring_c + s * C::kC, &maps.codes, m0 / 2, ks * 64, fb);  // [64 W rows][64 bytes]
+          mbar_arrive_expect_tx(fb, p.code_box_bytes);
+          if (!MN)  // [128 W rows][8 kb bytes per step]
+            tma_load_2d(ring_c + s * p.code_box_bytes, &maps.codes, ks * 8 * kb, m0, fb);
+          else      // [64 W rows][16 kb bytes: 128 codes]
+            tma_load_2d(ring_c + s * p.code_box_bytes, &maps.codes, m0 / 8 * kb, ks * 64, fb);
         }
       }
-      const uint32_t first = jc > NSC ? jc - NSC : 0;
+      const uint32_t first = jc > static_cast<uint32_t>(ncs) ? jc - ncs : 0;
       for (uint32_t q = first; q < jc; ++q) {
         volatile int never = 0;
-        mbar_wait(&bars->c_full[q % NSC], (q / NSC) & 1, &never);
+        mbar_wait(&bars->c_full[q % ncs], (q / ncs) & 1, &never);
       }
     }
   } else if (warp == 1) {
@@ -328,17 +329,21 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
       if (!mbar_wait(&bars->a_empty[sa], ((c_j / NSA) & 1) ^ 1, abort_flag)) break;
       uint8_t* st_a = ring_a + sa * C::kA;
       if (c_ks < nmain) {
-        const int sc = c_jc % NSC;
-        if (!mbar_wait(&bars->c_full[sc], (c_jc / NSC) & 1, abort_flag)) break;
-        const uint8_t* st_c = ring_c + sc * C::kC;
+        const int kb = p.code_bits, ncs = p.code_slots;
+        const uint32_t box = p.code_steps == 2 ? c_jc >> 1 : c_jc, sub = p.code_steps == 2 ? (c_jc & 1) : 0;
+        const int sc = box % ncs;
+        if (!mbar_wait(&bars->c_full[sc], (box / ncs) & 1, abort_flag)) break;
+        const uint8_t* st_c = ring_c + sc * p.code_box_bytes;
         int64_t row, col;
         bool valid;
         run_of(c_m0, c_ks * 64, row, col, valid);
-        if (!MN) {
-          eng::dequant_row64(p.dq, st_c + t * 32, cur, valid, st_a + t * 128, t & 7);
-        } else {
+        if (!MN) {  // row t: 8 kb bytes per step, code_steps steps per box row
+          eng::dequant_row64(p.dq, st_c + t * 8 * kb * p.code_steps + sub * 8 * kb, kb, cur, valid, st_a + t * 128,
+                             t & 7);
+        } else {    // reduction row nr: 16 kb bytes (128 codes), half h
           const int nr = t & 63, h = t >> 6;
-          eng::dequant_row64(p.dq, st_c + nr * 64 + h * 32, cur, valid, st_a + h * 8192 + nr * 128, nr & 7);
+          eng::dequant_row64(p.dq, st_c + nr * 16 * kb + h * 8 * kb, kb, cur, valid, st_a + h * 8192 + nr * 128,
+                             nr & 7);
         }
         mbar_arrive(&bars->c_empty[sc]);
       } else {

@@ -105,10 +105,10 @@ def test_host_validation_rejects_before_launch(L):
     # pooled adapter with an NF weight
     assert L.qlr_forward(ctypes.byref(q), P(0x1000), 16, P(0x1000), P(0x1000), 8, 1.0, 1, P(0x1000), P(0x1000),
                          P(0x1000), 1 << 20, None, None) == -4
-    # NF-3 weights are not served by the fused GEMM in this build
-    q3 = _fake_qweight(bits=3)
+    # 3-bit codes stream two 64-code steps per box along K: K must be a multiple of 128
+    q3 = _fake_qweight(bits=3, K=192)
     assert L.qlr_forward(ctypes.byref(q3), P(0x1000), 16, P(0x1000), P(0x1000), 8, 1.0, 0, P(0x1000), P(0x1000),
-                         P(0x1000), 1 << 20, None, None) == -4
+                         P(0x1000), 1 << 20, None, None) == -2
     # missing workspace (the pooled adapter's group expansion needs one)
     q4 = _fake_qweight(fmt=2, group=32)
     assert L.qlr_forward(ctypes.byref(q4), P(0x1000), 16, P(0x1000), P(0x1000), 8, 1.0, 1, P(0x1000), P(0x1000),

@@ -65,6 +65,25 @@ def test_ragged_nf4(cuda_lib, M, r):
     run_and_check(cuda_lib, spec, M, seed=M + r)
 
 
+@pytest.mark.parametrize("bits", [2, 3])
+@pytest.mark.parametrize("M,r,block,dq", [(1, 8, 64, 256), (40, 64, 128, 0), (333, 16, 64, 256), (700, 32, 128, 256)])
+def test_ragged_nf_low_bits(cuda_lib, bits, M, r, block, dq):
+    """NF-2 and NF-3 codes (LQ-LoRA's per-matrix bit widths) through the fused forward and input
+    gradient: 2-bit codes in 16-byte runs, 3-bit bit planes two steps per codes box."""
+    spec = LinearSpec("w", 320, 384, "nfk", bits, block, dq, r=r, s=0.5)
+    run_and_check(cuda_lib, spec, M, seed=100 * bits + M)
+
+
+@pytest.mark.parametrize("bits", [2, 3])
+def test_lqlora_matrix_full_size_sampled_rows(cuda_lib, bits):
+    """The first matrix of the mixed 7B stack drawn with this bit width, at its full shape and 2048 tokens."""
+    wl = workload("lqlora")
+    idx = next(i for i, s in enumerate(wl.linears) if s.bits == bits)
+    spec = wl.linears[idx]
+    rows = np.sort(np.random.default_rng(bits).choice(wl.M, 96, replace=False))
+    run_and_check(cuda_lib, spec, wl.M, seed=idx, rows=rows)
+
+
 @pytest.mark.parametrize("M", [64, 300, 1100])
 def test_ragged_int4_pooled(cuda_lib, M):
     spec = LinearSpec("w", 264, 512, "int4g", group=32, r=16, s=1.0, pooled=True)
