@@ -173,7 +173,7 @@ def run_ours(args, rank, world, dev):
     import numpy as np
     import torch
     import torch.distributed as dist
-    from quantized_base_lora_nf4_b200 import qlr
+    from quantized_base_lora_nf4_b200 import dp, qlr
     from synth import workload, normal
 
     qlr.lib()
@@ -211,6 +211,8 @@ def run_ours(args, rank, world, dev):
         qlr.backward_lora(L.q, L.X, dY, L.T, L.B, s, pooled=pooled, dA=L.dA, dB=L.dB, dT=L.dT, ws=L.ws_b)
         qlr.backward_dx(L.q, dY, L.A, L.dT, pooled=pooled, dX=dX, accumulate=accumulate, ws=L.ws_x)
 
+    bucket = dp.GradBucket([g for L in layers for g in (L.dA, L.dB)]) if world > 1 else None
+
     def step(record=False):
         if wl.kind == "mlp":
             gate, up, down = layers
@@ -230,10 +232,8 @@ def run_ours(args, rank, world, dev):
             qlr.lora_down(L.q, L.X, L.A, L.spec.s, pooled=L.spec.pooled, T_save=L.T, ws=L.ws)
             fwd_base(L, record)
             lin_bwd(L, L.dY, L.dX)
-        if world > 1:
-            for L in layers:
-                dist.all_reduce(L.dA)
-                dist.all_reduce(L.dB)
+        if bucket is not None:
+            bucket.allreduce()  # data parallel: one SUM all-reduce of every adapter gradient
 
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)  # > 126 MB L2
     for _ in range(args.warmup):
