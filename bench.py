@@ -1,7 +1,8 @@
 #!/usr/bin/env python
 """Throughput of the quantised-base + LoRA linear on B200: fwd+bwd tokens/s.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload qalora|tiny|mlp7b] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload qalora|tiny|mlp7b|lqlora|decode70b]
+                    [--impl ours|reference]
 
 One step = forward (adapter down-projection T = s P(X) A^T, fused dequant + tcgen05 base GEMM with the
 adapter term folded in) + backward (dT, dA, dB; fused input gradient) of every linear of the workload,
@@ -46,7 +47,7 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="qalora", choices=["qalora", "tiny", "mlp7b", "decode70b"])
+    ap.add_argument("--workload", default="qalora", choices=["qalora", "tiny", "mlp7b", "lqlora", "decode70b"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -76,6 +77,10 @@ def workload_desc(wl):
                 f"(s={spec.s}), {wl.M} tokens, fwd+bwd")
     if wl.name == "mlp7b":
         return f"mlp7b: LLaMA-7B MLP (gate/up 11008x4096, down 4096x11008) NF4+DQ, r=64, SwiGLU, {wl.M} tokens, fwd+bwd"
+    if wl.name == "lqlora":
+        return (f"lqlora: 32-layer LLaMA-7B stack, 224 linears (q,k,v,o 4096x4096; gate,up 11008x4096; "
+                f"down 4096x11008), per-matrix NF-k (k in 2,3,4) and block (64/128) with double quantisation, "
+                f"r=64, {wl.M} tokens, fwd+bwd")
     return f"tiny: NF4+DQ 256x256, r=8, {wl.M} tokens, fwd+bwd"
 
 
@@ -138,35 +143,67 @@ class ClockSampler:
 
 # ------------------------------------------------------------------------------------------ GPU arm
 class Layer:
-    """Device-resident state of one quantised linear (weights, adapters, activations, gradients)."""
+    """Device-resident state of one quantised linear (weights, adapters, activations, gradients).
 
-    def __init__(self, qlr, spec, M, seed, rank, dev, X=None):
+    With `shared` (the mixed-precision stack), activation buffers are shared between linears of the
+    same shape and the frozen weight is drawn on the device (torch's seeded CUDA generator, same
+    N(0, sigma_W^2) law as the numpy generators), which keeps setup of 224 7B-sized matrices short."""
+
+    def __init__(self, qlr, spec, M, seed, rank, dev, X=None, shared=None):
         import numpy as np
         import torch
         from synth import linear_tensors, normal
 
         self.spec = spec
-        t = linear_tensors(spec, M, seed=seed, matrix_index=0, with_x=X is None, with_dy=False)
         bf = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev).to(torch.bfloat16).contiguous()  # noqa
-        W = torch.from_numpy(t["W"]).to(dev)
+        if shared is None:
+            t = linear_tensors(spec, M, seed=seed, matrix_index=0, with_x=X is None, with_dy=False)
+            W = torch.from_numpy(t["W"]).to(dev)
+            A, B = t["A"], t["B"]
+        else:
+            g = torch.Generator(device=dev)
+            g.manual_seed(seed)
+            W = torch.randn((spec.N, spec.K), generator=g, device=dev, dtype=torch.float32) * spec.sigma_w
+            A = normal(seed, 0, "A", (spec.r, spec.k_adapter), 0.01, bf16=True)
+            B = normal(seed, 0, "B", (spec.N, spec.r), 0.01, bf16=True)
         if spec.fmt == "int4g":
             self.q = qlr.quantize_int4_group(W, spec.group)
         else:
             self.q = qlr.quantize_nf4(W, spec.bits, spec.block, spec.dq_block)
         del W
-        self.A, self.B = bf(t["A"]), bf(t["B"])
-        self.X = bf(t["X"]) if X is None else X
-        self.dY = bf(normal(seed + 1000 * rank, 0, "dY", (M, spec.N), 1.0, bf16=True))
+        self.A, self.B = bf(A), bf(B)
         r = spec.r
-        self.T = torch.empty((M, r), dtype=torch.bfloat16, device=dev)
-        self.Y = torch.empty((M, spec.N), dtype=torch.bfloat16, device=dev)
-        self.dT = torch.empty((M, r), dtype=torch.bfloat16, device=dev)
+
+        def buf(key, shape, dtype=torch.bfloat16, fill=None):
+            if shared is not None and key in shared:
+                return shared[key]
+            x = bf(fill()) if fill is not None else torch.empty(shape, dtype=dtype, device=dev)
+            if shared is not None:
+                shared[key] = x
+            return x
+
+        if X is not None:
+            self.X = X
+        elif shared is None:
+            self.X = bf(t["X"])
+        else:
+            self.X = buf(("X", spec.K), None, fill=lambda: normal(seed, 0, "X", (M, spec.K), 1.0, bf16=True))
+        self.dY = buf(("dY", spec.N), None, fill=lambda: normal(seed + 1000 * rank, 0, "dY", (M, spec.N), 1.0, bf16=True))
+        self.T = buf(("T", r), (M, r))
+        self.Y = buf(("Y", spec.N), (M, spec.N))
+        self.dT = buf(("dT", r), (M, r))
         self.dA = torch.empty((r, spec.k_adapter), dtype=torch.float32, device=dev)
         self.dB = torch.empty((spec.N, r), dtype=torch.float32, device=dev)
-        self.dX = torch.empty((M, spec.K), dtype=torch.bfloat16, device=dev)
-        self.ws = qlr.Workspace(dev)
-        self.ws_b = qlr.Workspace(dev)
-        self.ws_x = qlr.Workspace(dev)
+        self.dX = buf(("dX", spec.K), (M, spec.K))
+
+        def ws(key):
+            if shared is None:
+                return qlr.Workspace(dev)
+            if key not in shared:
+                shared[key] = qlr.Workspace(dev)
+            return shared[key]
+
+        self.ws, self.ws_b, self.ws_x = ws("ws"), ws("ws_b"), ws("ws_x")
 
 
 def run_ours(args, rank, world, dev):
@@ -192,6 +229,10 @@ def run_ours(args, rank, world, dev):
         dHm = torch.empty_like(Hm)
         dG = torch.empty_like(Hm)
         dU = torch.empty_like(Hm)
+    elif wl.kind == "stack":
+        shared = {}
+        layers = [Layer(qlr, spec, M, seed * 100003 + i, rank, dev, shared=shared) for i, spec in enumerate(wl.linears)]
+        torch.cuda.synchronize()
     else:
         layers = [Layer(qlr, wl.linears[0], M, seed, rank, dev)]
     fwd_ev = []
@@ -227,11 +268,11 @@ def run_ours(args, rank, world, dev):
             qlr.swiglu_backward(dHm, gate.Y, up.Y, dG=dG, dU=dU)
             lin_bwd(gate, dG, gate.dX)
             lin_bwd(up, dU, gate.dX, accumulate=True)
-        else:
-            L = layers[0]
-            qlr.lora_down(L.q, L.X, L.A, L.spec.s, pooled=L.spec.pooled, T_save=L.T, ws=L.ws)
-            fwd_base(L, record)
-            lin_bwd(L, L.dY, L.dX)
+        else:  # one linear, or every linear of the stack in turn
+            for L in layers:
+                qlr.lora_down(L.q, L.X, L.A, L.spec.s, pooled=L.spec.pooled, T_save=L.T, ws=L.ws)
+                fwd_base(L, record)
+                lin_bwd(L, L.dY, L.dX)
         if bucket is not None:
             bucket.allreduce()  # data parallel: one SUM all-reduce of every adapter gradient
 
@@ -279,8 +320,11 @@ def run_ours(args, rank, world, dev):
                 (layers[0].dY, torch.empty(layers[0].dY.shape, dtype=torch.bfloat16, pin_memory=True))]
     for d, h in h_in:
         h.copy_(d)
-    h_out = [(L.dA, torch.empty(L.dA.shape, dtype=torch.float32, pin_memory=True)) for L in layers]
-    h_out += [(L.dB, torch.empty(L.dB.shape, dtype=torch.float32, pin_memory=True)) for L in layers]
+    # the step's result read back: every adapter gradient (the stack: the last linear's, as a training
+    # loop would read a metric, not 224 gradients)
+    out_layers = layers[-1:] if wl.kind == "stack" else layers
+    h_out = [(L.dA, torch.empty(L.dA.shape, dtype=torch.float32, pin_memory=True)) for L in out_layers]
+    h_out += [(L.dB, torch.empty(L.dB.shape, dtype=torch.float32, pin_memory=True)) for L in out_layers]
     h2d = sum(h.numel() * h.element_size() for _, h in h_in)
     d2h = sum(h.numel() * h.element_size() for _, h in h_out)
     e2e_steps = max(3, args.steps // 2)
@@ -324,9 +368,19 @@ def oracle_tokens_per_s(wl, seed, budget_s=12.0):
     from oracle import quantize as Q
     from synth import linear_tensors
 
-    m = {"tiny": 16, "qalora": 512, "mlp7b": 32}[wl.name]
+    m = {"tiny": 16, "qalora": 512, "mlp7b": 32, "lqlora": 16}[wl.name]
+    linears = list(wl.linears)
+    scale = 1.0
+    if wl.kind == "stack":  # the first linear of each distinct shape, scaled by FLOPs to the whole stack
+        seen, sample = set(), []
+        for spec in linears:
+            if (spec.N, spec.K) not in seen:
+                seen.add((spec.N, spec.K))
+                sample.append(spec)
+        scale = sum(flops_per_token(s) for s in sample) / sum(flops_per_token(s) for s in linears)
+        linears = sample
     mats = []
-    for i, spec in enumerate(wl.linears):
+    for i, spec in enumerate(linears):
         t = linear_tensors(spec, m, seed=seed + i)
         if spec.fmt == "int4g":
             Wdq = Q.dequant_int4_group(Q.quantize_int4_group(t["W"], spec.group))
@@ -347,18 +401,20 @@ def oracle_tokens_per_s(wl, seed, budget_s=12.0):
             OL.backward(dG, X, gW, gt["A"], gt["B"], gs.s)
             OL.backward(dU, X, uW, ut["A"], ut["B"], us.s)
         else:
-            spec, t, Wdq = mats[0]
-            L = spec.group if spec.pooled else None
-            OL.forward(t["X"], Wdq, t["A"], t["B"], spec.s, L)
-            OL.backward(t["dY"], t["X"], Wdq, t["A"], t["B"], spec.s, L)
+            for spec, t, Wdq in mats:
+                L = spec.group if spec.pooled else None
+                OL.forward(t["X"], Wdq, t["A"], t["B"], spec.s, L)
+                OL.backward(t["dY"], t["X"], Wdq, t["A"], t["B"], spec.s, L)
         reps += 1
         el = time.perf_counter() - t0
         if el >= budget_s or reps >= 2000:
             break
     cores = len(os.sched_getaffinity(0))
-    return {"value": reps * m / el, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": f"{reps} x {m} tokens of the {wl.name} workload, fwd+bwd in fp64 numpy "
-                      f"({el:.1f} s; dequantised weights prepared untimed)"}
+    what = (f"{reps} x {m} tokens through the first linear of each of the {len(mats)} shapes of the stack, "
+            f"scaled by FLOPs (x{scale:.4f}) to all {len(wl.linears)} linears" if wl.kind == "stack"
+            else f"{reps} x {m} tokens of the {wl.name} workload")
+    return {"value": reps * m / el * scale, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{what}, fwd+bwd in fp64 numpy ({el:.1f} s; dequantised weights prepared untimed)"}
 
 
 # ------------------------------------------------------------------------------------------ decode shape
@@ -420,10 +476,15 @@ def main():
 
     wl = workload(args.workload, args.seed)
     fl_tok = sum(flops_per_token(s) for s in wl.linears)
-    cfg = {"workload": workload_desc(wl), "tokens_per_rank": wl.M,
-           "linears": [{"name": s.name, "N": s.N, "K": s.K, "r": s.r, "format": s.fmt,
-                        "bits": s.bits if s.fmt == "nfk" else 4,
-                        "block": s.block if s.fmt == "nfk" else s.group} for s in wl.linears],
+    lin = [{"name": s.name, "N": s.N, "K": s.K, "r": s.r, "format": s.fmt, "bits": s.bits if s.fmt == "nfk" else 4,
+            "block": s.block if s.fmt == "nfk" else s.group} for s in wl.linears]
+    if len(lin) > 8:  # the stack: a summary
+        hist = {}
+        for d in lin:
+            key = f"nf{d['bits']}_b{d['block']}"
+            hist[key] = hist.get(key, 0) + 1
+        lin = {"count": len(lin), "bits_block_histogram": hist}
+    cfg = {"workload": workload_desc(wl), "tokens_per_rank": wl.M, "linears": lin,
            "l2": "256 MiB buffer written, then read, between timed steps (L2 flushed, no dirty lines left)", "seed": args.seed,
            "parallelism": f"dp{world}"}
 
@@ -469,13 +530,18 @@ def main():
     ms = res["ms_per_step"]
     tokens_s = world * M / (ms / 1e3)
     tflops = world * fl_tok * M / (ms / 1e3) / 1e12
-    # dominant kernel: the fused dequant + tcgen05 forward GEMM of the first linear
-    spec0 = wl.linears[0]
+    # dominant kernel: the fused dequant + tcgen05 forward GEMM (of the first linear; the stack: every
+    # launch of the step, total algorithmic FLOPs over total launch time)
     fwd_ms = res["fwd_ms"]
     n_fwd = len(wl.linears)
     per_layer = [statistics.mean(fwd_ms[i::n_fwd]) for i in range(n_fwd)]
-    fwd_launch_ms = per_layer[0]
-    fwd_flops = 2.0 * M * spec0.N * spec0.K + 2.0 * M * spec0.N * spec0.r
+    fl = [2.0 * M * s.N * s.K + 2.0 * M * s.N * s.r for s in wl.linears]
+    if wl.kind == "stack":
+        fwd_launch_ms = sum(per_layer) / n_fwd
+        fwd_flops = sum(fl) / n_fwd
+    else:
+        fwd_launch_ms = per_layer[0]
+        fwd_flops = fl[0]
     achieved = fwd_flops / (fwd_launch_ms / 1e3) / 1e12
     peak = float(peaks["bf16_tflops"])
     traffic = profile_traffic(f"fused_forward_{wl.name}.md")

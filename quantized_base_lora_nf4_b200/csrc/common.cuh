@@ -32,11 +32,7 @@ cudaError_t launch_merge(const qlr_qweight* w, const uint16_t* A, const uint16_t
 cudaError_t launch_swiglu_fwd(const uint16_t* G, const uint16_t* U, uint16_t* H, int64_t n, cudaStream_t st);
 cudaError_t launch_swiglu_bwd(const uint16_t* dH, const uint16_t* G, const uint16_t* U, uint16_t* dG,
                               uint16_t* dU, int64_t n, cudaStream_t st);
-cudaError_t launch_pool(const uint16_t* X, int64_t M, int64_t K, int L, uint16_t* Xp, cudaStream_t st);
 cudaError_t launch_expand_adapter(const uint16_t* A, int r, int64_t K, int L, uint16_t* Aexp, cudaStream_t st);
-cudaError_t launch_reduce_splits(const float* part, int splits, int64_t rows, int64_t cols, int64_t ld_part,
-                                 float scale, int transpose, int out_bf16, void* out, int64_t ld_out,
-                                 cudaStream_t st);
 
 int device_sm_count();
 

@@ -61,22 +61,6 @@ __global__ void swiglu_bwd_kernel(const uint4* __restrict__ dH, const uint4* __r
   }
 }
 
-// Xp[m, g] = bf16( (sum of X[m, gL .. gL+L-1]) / L ): one thread per output, fp32 sum.
-__global__ void pool_kernel(const uint16_t* __restrict__ X, int64_t M, int64_t K, int L, uint16_t* __restrict__ Xp) {
-  const int64_t G = K / L;
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i >= M * G) return;
-  const int64_t m = i / G, g = i % G;
-  const uint4* src = reinterpret_cast<const uint4*>(X + m * K + g * L);
-  float acc = 0.f;
-  for (int c = 0; c < L / 8; ++c) {
-    const uint4 v = src[c];
-    acc += lo_f(v.x) + hi_f(v.x) + lo_f(v.y) + hi_f(v.y) + lo_f(v.z) + hi_f(v.z) + lo_f(v.w) + hi_f(v.w);
-  }
-  const float mean = acc / static_cast<float>(L);
-  Xp[i] = static_cast<uint16_t>(pack_bf16x2_rn(mean, 0.f) & 0xFFFFu);
-}
-
 // Aexp[j, k] = bf16( A[j, k / L] / L ): the adapter seen by the un-pooled input.
 __global__ void expand_kernel(const uint16_t* __restrict__ A, int r, int64_t K, int L, uint16_t* __restrict__ Aexp) {
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -84,31 +68,6 @@ __global__ void expand_kernel(const uint16_t* __restrict__ A, int r, int64_t K, 
   const int64_t j = i / K, k = i % K;
   const float v = bf16_bits_to_f32(A[j * (K / L) + k / L]) / static_cast<float>(L);
   Aexp[i] = static_cast<uint16_t>(pack_bf16x2_rn(v, 0.f) & 0xFFFFu);
-}
-
-// out[row, col] (or out[col, row] when transposed) = scale * sum_s part[s, row, col], summed in
-// split order so the result does not depend on scheduling.
-__global__ void reduce_splits_kernel(const float* __restrict__ part, int splits, int64_t rows, int64_t split_rows,
-                                     int64_t cols, int64_t ld_part, float scale, int transpose, int out_bf16,
-                                     void* out, int64_t ld_out) {
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i >= rows * cols) return;
-  int64_t row, col;
-  if (transpose) {  // consecutive threads walk rows so the transposed store is coalesced
-    col = i / rows;
-    row = i % rows;
-  } else {
-    row = i / cols;
-    col = i % cols;
-  }
-  float acc = 0.f;
-  for (int s = 0; s < splits; ++s) acc += part[(static_cast<int64_t>(s) * split_rows + row) * ld_part + col];
-  acc *= scale;
-  const int64_t o = transpose ? col * ld_out + row : row * ld_out + col;
-  if (out_bf16)
-    static_cast<uint16_t*>(out)[o] = static_cast<uint16_t>(pack_bf16x2_rn(acc, 0.f) & 0xFFFFu);
-  else
-    static_cast<float*>(out)[o] = acc;
 }
 
 // Split-order sum of an adapter GEMM's parts + its output transform, one thread per output element.
@@ -201,29 +160,10 @@ cudaError_t launch_swiglu_bwd(const uint16_t* dH, const uint16_t* G, const uint1
   return cudaGetLastError();
 }
 
-cudaError_t launch_pool(const uint16_t* X, int64_t M, int64_t K, int L, uint16_t* Xp, cudaStream_t st) {
-  const int64_t n = M * (K / L);
-  count_launch();
-  pool_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(X, M, K, L, Xp);
-  return cudaGetLastError();
-}
-
 cudaError_t launch_expand_adapter(const uint16_t* A, int r, int64_t K, int L, uint16_t* Aexp, cudaStream_t st) {
   const int64_t n = static_cast<int64_t>(r) * K;
   count_launch();
   expand_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(A, r, K, L, Aexp);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_reduce_splits(const float* part, int splits, int64_t rows, int64_t cols, int64_t ld_part,
-                                 float scale, int transpose, int out_bf16, void* out, int64_t ld_out,
-                                 cudaStream_t st) {
-  const int64_t n = rows * cols;
-  if (n == 0) return cudaSuccess;
-  const int64_t split_rows = (rows + 127) / 128 * 128;  // each split holds whole 128-row tiles
-  count_launch();
-  reduce_splits_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(
-      part, splits, rows, split_rows, cols, ld_part, scale, transpose, out_bf16, out, ld_out);
   return cudaGetLastError();
 }
 
