@@ -63,6 +63,37 @@ def flush_l2(buf):
     return buf.view(torch.int32).amax()
 
 
+def time_quantizer(qlr, spec, W, flush, reps: int = 10):
+    """HBM roofline of the layer's own quantisation (the memory-bound quantiser path): median CUDA-event
+    time of quantising the fp32 weight W already on the device, and its algorithmic bytes (fp32 read,
+    codes and constants written)."""
+    import torch
+    N, K = spec.N, spec.K
+    if spec.fmt == "int4g":
+        fn = lambda: qlr.quantize_int4_group(W, spec.group)  # noqa: E731
+        out_b = N * K // 2 + 4 * N * K // spec.group
+        kern = f"quantize_int4g_kernel<{spec.group}>"
+    else:
+        fn = lambda: qlr.quantize_nf4(W, spec.bits, spec.block, spec.dq_block)  # noqa: E731
+        nb = N * K // spec.block
+        out_b = N * K * spec.bits // 8 + (nb + 4 * (nb // 256) if spec.dq_block else 4 * nb)
+        kern = "quantize_nfk_kernel"
+    for _ in range(2):
+        fn()
+    ts = []
+    for _ in range(reps):
+        flush_l2(flush)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        ts.append((e0, e1))
+    torch.cuda.synchronize()
+    ms = statistics.median(a.elapsed_time(b) for a, b in ts)
+    nbytes = 4 * N * K + out_b
+    return {"kernel": kern, "shape": [N, K], "ms": ms, "bytes": nbytes, "GBps": nbytes / ms / 1e6}
+
+
 def flops_per_token(spec) -> float:
     """4NK (forward base GEMM + input gradient; the base weight gets no gradient) plus the six rank-r
     adapter products (T, T B^T, dT, dT A, dA, dB), with K/L adapter inputs for the pooled adapter."""
@@ -430,13 +461,15 @@ def run_decode(args, dev):
     spec = wl.linears[0]
     t = linear_tensors(spec, 16, seed=args.seed, with_dy=False)
     W = torch.from_numpy(t["W"]).to(dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    quant = time_quantizer(qlr, spec, W, flush)
+    quant["frac_of_hbm"] = quant["GBps"] / float(peaks["hbm_gbs"])
     q = qlr.quantize_nf4(W, 4, 64, 256)
     del W
     bf = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev).to(torch.bfloat16).contiguous()  # noqa
     A, B = bf(t["A"]), bf(t["B"])
     code_bytes = spec.N * spec.K // 2
     all_bytes = code_bytes + spec.N * spec.K // 64 + 4 * spec.N * spec.K // (64 * 256) + 2 * spec.r * (spec.N + spec.K)
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     out = {}
     for M in wl.token_counts:
         X = bf(t["X"][:M])
@@ -462,6 +495,7 @@ def run_decode(args, dev):
         out[str(M)] = {"ms": t_ms, "code_GBps": code_bytes / t_ms / 1e6, "all_GBps": all_bytes / t_ms / 1e6,
                        "code_frac_of_hbm": code_bytes / t_ms / 1e6 / float(peaks["hbm_gbs"])}
     return {"workload": "decode70b: NF4+DQ 28672x8192, r=64, forward at 1/4/16 tokens", "per_tokens": out,
+            "quantizer": quant,
             "hbm_peak_gbs": float(peaks["hbm_gbs"]), "peak_kind": peak_kind,
             "code_bytes": code_bytes, "all_bytes": all_bytes}
 
@@ -520,6 +554,15 @@ def main():
             dist.destroy_process_group()
         return 0
     res = run_ours(args, rank, world, dev)
+    quant = None
+    if rank == 0:  # the quantiser path of the workload's first linear (memory-bound; HBM roofline)
+        from quantized_base_lora_nf4_b200 import qlr
+        spec0 = wl.linears[0]
+        g = torch.Generator(device=dev)
+        g.manual_seed(args.seed)
+        Wq = torch.randn((spec0.N, spec0.K), generator=g, device=dev, dtype=torch.float32) * spec0.sigma_w
+        quant = time_quantizer(qlr, spec0, Wq, torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev))
+        del Wq
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
@@ -556,6 +599,8 @@ def main():
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                      "peak_kind": f"{peak_kind} bf16 burst", "traffic": traffic,
                      "flops_per_launch": fwd_flops, "launch_ms": fwd_launch_ms},
+        "quantizer": None if quant is None else {**quant, "bound": "hbm", "peak_GBps": float(peaks["hbm_gbs"]),
+                                                 "frac": quant["GBps"] / float(peaks["hbm_gbs"])},
         "gpu_launches": res["launches"],
         "clocks": res["clocks"],
         "e2e": {"value": world * M / (res["e2e_ms_per_step"] / 1e3), "unit": "tokens/s",

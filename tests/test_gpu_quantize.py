@@ -75,7 +75,7 @@ def test_nf_quantize_reports_nonfinite(cuda_lib):
 
 
 @pytest.mark.parametrize("group", [32, 64, 128])
-@pytest.mark.parametrize("shape", [(64, 256), (4096, 4096)])
+@pytest.mark.parametrize("shape", [(64, 256), (40, 384), (4096, 4096)])
 def test_int4_group_quantize_bit_exact(cuda_lib, group, shape):
     qlr = cuda_lib
     W = random_matrix(23, group, "W", shape, 0.02)
