@@ -44,4 +44,24 @@ cudaError_t launch_decode(const qlr_qweight* w, const uint16_t* X, int64_t M, co
 // Counts kernel launches issued by this library (reported by qlr_launch_count).
 void count_launch(int n = 1);
 
+// Launches a hot-path kernel with programmatic stream serialisation, so that its launch and set-up
+// overlap the tail of the previous kernel on the stream; the kernel itself calls pdl_wait before it
+// reads or writes global memory.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  count_launch();
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 }  // namespace qlr

@@ -151,6 +151,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
   const int u_end = static_cast<int>((static_cast<int64_t>(blockIdx.x + 1) * p.units) / gridDim.x);
   const int nsteps = static_cast<int>(p.K / 128);
 
+  pdl_launch_dependents();
+  pdl_wait();
   if (threadIdx.x == 0) {
     for (int s = 0; s < kSlots; ++s) {
       mbar_init(&bars->full[s], 1);
@@ -355,9 +357,7 @@ cudaError_t launch_decode_variant(const DecodeParams& p, int grid, const CUtenso
     attr_err = cudaFuncSetAttribute(decode_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
   });
   if (attr_err != cudaSuccess) return attr_err;
-  count_launch();
-  decode_kernel<NT><<<grid, kThreads, smem, st>>>(p, tc_lo, tc_hi, tx);
-  return cudaGetLastError();
+  return launch_pdl(decode_kernel<NT>, dim3(grid), dim3(kThreads), smem, st, p, tc_lo, tc_hi, tx);
 }
 
 }  // namespace

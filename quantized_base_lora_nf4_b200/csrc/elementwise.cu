@@ -18,6 +18,8 @@ __device__ __forceinline__ float sigmoidf_(float g) { return 1.0f / (1.0f + expf
 
 __global__ void swiglu_fwd_kernel(const uint4* __restrict__ G, const uint4* __restrict__ U, uint4* __restrict__ H,
                                   int64_t n8) {
+  pdl_launch_dependents();
+  pdl_wait();
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const uint4 g = G[i], u = U[i];
@@ -36,6 +38,8 @@ __global__ void swiglu_fwd_kernel(const uint4* __restrict__ G, const uint4* __re
 
 __global__ void swiglu_bwd_kernel(const uint4* __restrict__ dH, const uint4* __restrict__ G, const uint4* __restrict__ U,
                                   uint4* __restrict__ dG, uint4* __restrict__ dU, int64_t n8) {
+  pdl_launch_dependents();
+  pdl_wait();
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const uint4 d = dH[i], g = G[i], u = U[i];
@@ -63,6 +67,8 @@ __global__ void swiglu_bwd_kernel(const uint4* __restrict__ dH, const uint4* __r
 
 // Aexp[j, k] = bf16( A[j, k / L] / L ): the adapter seen by the un-pooled input.
 __global__ void expand_kernel(const uint16_t* __restrict__ A, int r, int64_t K, int L, uint16_t* __restrict__ Aexp) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i >= r * K) return;
   const int64_t j = i / K, k = i % K;
@@ -72,6 +78,8 @@ __global__ void expand_kernel(const uint16_t* __restrict__ A, int r, int64_t K, 
 
 // Split-order sum of an adapter GEMM's parts + its output transform, one thread per output element.
 __global__ void adapter_reduce_kernel(const AdapterParams p, int bn) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t split_stride = static_cast<int64_t>(p.m_tiles) * 128 * bn;
   if (i >= static_cast<int64_t>(p.Mm) * p.r) return;
@@ -98,6 +106,8 @@ __global__ void adapter_reduce_kernel(const AdapterParams p, int bn) {
 // rows by shuffles, and the group totals combine the warp sums (L = 32, 64 or 128 divides 256).
 __global__ void adapter_reduce_pooled_kernel(const AdapterParams p, int bn) {
   __shared__ float warp_sum[8];
+  pdl_launch_dependents();
+  pdl_wait();
   const int64_t split_stride = static_cast<int64_t>(p.m_tiles) * 128 * bn;
   const int64_t blocks_per_col = (p.Mm + 255) / 256;
   const int64_t j = blockIdx.x / blocks_per_col;
@@ -129,42 +139,32 @@ unsigned grid_for(int64_t n_items, int threads) {
 cudaError_t launch_adapter_reduce(const AdapterParams& p, int bn, cudaStream_t st) {
   if (p.out_mode == ADAPTER_COLS_F32 && p.pool_L > 1) {
     const int64_t blocks = (static_cast<int64_t>(p.Mm) + 255) / 256 * p.r;
-    count_launch();
-    adapter_reduce_pooled_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(p, bn);
-    return cudaGetLastError();
+    return launch_pdl(adapter_reduce_pooled_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st, p, bn);
   }
   const int64_t n = static_cast<int64_t>(p.Mm) * p.r;
   if (n == 0) return cudaSuccess;
-  count_launch();
-  adapter_reduce_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(p, bn);
-  return cudaGetLastError();
+  return launch_pdl(adapter_reduce_kernel, dim3(static_cast<unsigned>((n + 255) / 256)), dim3(256), 0, st, p, bn);
 }
 
 cudaError_t launch_swiglu_fwd(const uint16_t* G, const uint16_t* U, uint16_t* H, int64_t n, cudaStream_t st) {
   if (n == 0) return cudaSuccess;
   const int64_t n8 = n / 8;
-  count_launch();
-  swiglu_fwd_kernel<<<grid_for(n8, 256), 256, 0, st>>>(reinterpret_cast<const uint4*>(G),
-                                                       reinterpret_cast<const uint4*>(U), reinterpret_cast<uint4*>(H), n8);
-  return cudaGetLastError();
+  return launch_pdl(swiglu_fwd_kernel, dim3(grid_for(n8, 256)), dim3(256), 0, st, reinterpret_cast<const uint4*>(G),
+                    reinterpret_cast<const uint4*>(U), reinterpret_cast<uint4*>(H), n8);
 }
 
 cudaError_t launch_swiglu_bwd(const uint16_t* dH, const uint16_t* G, const uint16_t* U, uint16_t* dG, uint16_t* dU,
                               int64_t n, cudaStream_t st) {
   if (n == 0) return cudaSuccess;
   const int64_t n8 = n / 8;
-  count_launch();
-  swiglu_bwd_kernel<<<grid_for(n8, 256), 256, 0, st>>>(
-      reinterpret_cast<const uint4*>(dH), reinterpret_cast<const uint4*>(G), reinterpret_cast<const uint4*>(U),
-      reinterpret_cast<uint4*>(dG), reinterpret_cast<uint4*>(dU), n8);
-  return cudaGetLastError();
+  return launch_pdl(swiglu_bwd_kernel, dim3(grid_for(n8, 256)), dim3(256), 0, st, reinterpret_cast<const uint4*>(dH),
+                    reinterpret_cast<const uint4*>(G), reinterpret_cast<const uint4*>(U), reinterpret_cast<uint4*>(dG),
+                    reinterpret_cast<uint4*>(dU), n8);
 }
 
 cudaError_t launch_expand_adapter(const uint16_t* A, int r, int64_t K, int L, uint16_t* Aexp, cudaStream_t st) {
   const int64_t n = static_cast<int64_t>(r) * K;
-  count_launch();
-  expand_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(A, r, K, L, Aexp);
-  return cudaGetLastError();
+  return launch_pdl(expand_kernel, dim3(static_cast<unsigned>((n + 255) / 256)), dim3(256), 0, st, A, r, K, L, Aexp);
 }
 
 }  // namespace qlr

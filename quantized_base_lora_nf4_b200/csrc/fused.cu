@@ -137,6 +137,10 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
     tma_prefetch_desc(&maps.b_tail);
   }
   if (warp == 14 && lane == 0) tma_prefetch_desc(&maps.codes);
+  // everything above touches only shared memory and kernel parameters; from here on the previous
+  // kernel's results are needed (and its TMEM must be free)
+  pdl_launch_dependents();
+  pdl_wait();
   if (warp == 1) {
     tmem_alloc(&bars->tmem_base, C::kTmemCols);
     tmem_relinquish();
@@ -180,13 +184,14 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
   } else if (warp == 14) {
     // ------------------------------------------------------------------ codes producer
     if (lane == 0) {
-      const int ncs = p.code_slots, kb = p.code_bits;
+      const int lg = p.code_slots_log2, ncs = 1 << lg, kb = p.code_bits;
+      const uint32_t mask = static_cast<uint32_t>(ncs - 1);
       uint32_t jc = 0;  // boxes
       for (int tile = blockIdx.x; tile < n_tiles_total && !*abort_flag; tile += gridDim.x) {
         const int m0 = tile_m0(tile);
         for (int ks = 0; ks < nmain; ks += p.code_steps, ++jc) {
-          const int s = jc % ncs;
-          if (!mbar_wait(&bars->c_empty[s], ((jc / ncs) & 1) ^ 1, abort_flag)) break;
+          const int s = static_cast<int>(jc & mask);
+          if (!mbar_wait(&bars->c_empty[s], ((jc >> lg) & 1) ^ 1, abort_flag)) break;
           uint64_t* fb = &bars->c_full[s];
           mbar_arrive_expect_tx(fb, p.code_box_bytes);
           if (!MN)  // [128 W rows][8 kb bytes per step]
@@ -198,7 +203,7 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
       const uint32_t first = jc > static_cast<uint32_t>(ncs) ? jc - ncs : 0;
       for (uint32_t q = first; q < jc; ++q) {
         volatile int never = 0;
-        mbar_wait(&bars->c_full[q % ncs], (q / ncs) & 1, &never);
+        mbar_wait(&bars->c_full[q & mask], (q >> lg) & 1, &never);
       }
     }
   } else if (warp == 1) {
@@ -329,10 +334,10 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
       if (!mbar_wait(&bars->a_empty[sa], ((c_j / NSA) & 1) ^ 1, abort_flag)) break;
       uint8_t* st_a = ring_a + sa * C::kA;
       if (c_ks < nmain) {
-        const int kb = p.code_bits, ncs = p.code_slots;
+        const int kb = p.code_bits, lg = p.code_slots_log2;
         const uint32_t box = p.code_steps == 2 ? c_jc >> 1 : c_jc, sub = p.code_steps == 2 ? (c_jc & 1) : 0;
-        const int sc = box % ncs;
-        if (!mbar_wait(&bars->c_full[sc], (box / ncs) & 1, abort_flag)) break;
+        const int sc = static_cast<int>(box & ((1u << lg) - 1u));
+        if (!mbar_wait(&bars->c_full[sc], (box >> lg) & 1, abort_flag)) break;
         const uint8_t* st_c = ring_c + sc * p.code_box_bytes;
         int64_t row, col;
         bool valid;
@@ -391,9 +396,7 @@ cudaError_t launch_fused_variant(const GemmParams& p, const GemmMaps& maps, cuda
   if (attr_err != cudaSuccess) return attr_err;
   const int tiles = p.m_tiles * p.n_tiles;
   const int grid = tiles < device_sm_count() ? tiles : device_sm_count();
-  count_launch();
-  kern<<<grid, kThreadsFused, C::kSmem + 1024, st>>>(p, maps);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(grid), dim3(kThreadsFused), C::kSmem + 1024, st, p, maps);
 }
 
 }  // namespace

@@ -142,6 +142,10 @@ __global__ void __launch_bounds__(kThreadsAdapter, 1)
     tma_prefetch_desc(&maps.a);
     tma_prefetch_desc(&maps.b);
   }
+  // everything above touches only shared memory and kernel parameters; from here on the previous
+  // kernel's results are needed (and its TMEM must be free)
+  pdl_launch_dependents();
+  pdl_wait();
   if (warp == 1) {
     tmem_alloc(&bars->tmem_base, C::kTmemCols);
     tmem_relinquish();
@@ -286,9 +290,7 @@ cudaError_t launch_adapter_variant(const AdapterParams& p, const GemmMaps& maps,
   if (attr_err != cudaSuccess) return attr_err;
   const int items = p.m_tiles * p.splits;
   const int grid = items < device_sm_count() ? items : device_sm_count();
-  count_launch();
-  kern<<<grid, kThreadsAdapter, C::kSmem + 1024, st>>>(p, maps);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(grid), dim3(kThreadsAdapter), C::kSmem + 1024, st, p, maps);
 }
 
 }  // namespace

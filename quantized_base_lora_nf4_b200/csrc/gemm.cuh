@@ -46,8 +46,9 @@ struct GemmParams {
   int accumulate;        // OUT_BF16_T: add the previous contents of out
   DqParams dq;
   // codes ring of the fused kernel: one TMA box per slot covering code_steps main steps (2 for 3-bit
-  // codes along K, whose 24-byte runs are not a legal box width), code_slots slots of code_box_bytes
-  int code_bits, code_steps, code_slots, code_box_bytes;
+  // codes along K, whose 24-byte runs are not a legal box width), 2^code_slots_log2 slots of
+  // code_box_bytes
+  int code_bits, code_steps, code_slots_log2, code_box_bytes;
   // fused kernels: the tail's weight-side operand, copied into the A tile by the dequantiser warps
   // (forward: B [N, r], row-major; input gradient: A or its group expansion [r, K], row-major)
   const uint16_t* tail_a;

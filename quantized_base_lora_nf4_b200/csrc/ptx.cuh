@@ -58,6 +58,13 @@ QLR_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag)
   }
 }
 
+// Programmatic dependent launch.  A kernel lets the next kernel of its stream be scheduled as soon as
+// every one of its CTAs has started (the next kernel's CTAs then set up and park in pdl_wait), and
+// waits for the previous kernel to complete, with its writes visible, before touching global memory.
+// Both are no-ops for a kernel launched without the programmatic-serialization attribute.
+QLR_DEV void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+QLR_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 QLR_DEV void named_bar_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
