@@ -176,7 +176,8 @@ QLR_API int qlr_forward(const qlr_qweight* w, const uint16_t* X, int64_t M, cons
                 int32_t* status, void* stream);
 
 /* The two stages of qlr_forward, callable separately (same arguments and buffers):
- *   qlr_lora_down     T_save = bf16(s * P(X) A^T)      (split-K tensor-core GEMM + fixed-order sum)
+ *   qlr_lora_down     T_save = bf16(s * P(X) A^T)      (split-K tensor-core GEMM + fixed-order sum; for
+ *                     1..16 tokens without pooling, one fixed-order reduction kernel and no workspace)
  *   qlr_forward_base  Y = bf16(X dequant(W)^T + T_save B^T)   (the fused dequant + tcgen05 kernel)
  * qlr_lora_down uses the workspace of qlr_forward_workspace_bytes; qlr_forward_base needs none. */
 QLR_API int qlr_lora_down(const qlr_qweight* w, const uint16_t* X, int64_t M, const uint16_t* A, int r, float s,

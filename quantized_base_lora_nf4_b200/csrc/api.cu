@@ -323,6 +323,7 @@ int qlr_qalora_merge(const qlr_qweight* w, const uint16_t* A, const uint16_t* B,
 
 size_t qlr_forward_workspace_bytes(const qlr_qweight* w, int64_t M, int r, int pooled) {
   if (check_qweight(w) || M <= 0 || check_rank(r)) return 0;
+  if (!pooled && lora_down_small_supported(M)) return 0;  // the few-token kernel needs no scratch
   // the group expansion of A (pooled adapter), then the split partial sums
   return (pooled ? align256(size_t(r) * w->K * 2) : 0) + adapter_ws_bytes(M, w->K, r);
 }
@@ -345,6 +346,7 @@ int qlr_lora_down(const qlr_qweight* w, const uint16_t* X, int64_t M, const uint
   cudaStream_t st = as_stream(stream);
   int32_t* stat = status_or_sink(status);
   const int64_t K = w->K;
+  if (!pooled && lora_down_small_supported(M)) return cuda_rc(launch_lora_down_small(X, M, K, A, r, s, T_save, st));
   // T_save = bf16(s * P(X) A^T) = bf16(s * X Aexp^T), Aexp[j, k] = A[j, k / L] / L for the pooled adapter
   const uint16_t* Ab = A;
   uint8_t* ws = static_cast<uint8_t*>(workspace);

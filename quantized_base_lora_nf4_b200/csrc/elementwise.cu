@@ -128,6 +128,61 @@ __global__ void adapter_reduce_pooled_kernel(const AdapterParams p, int bn) {
   }
 }
 
+// Adapter down-projection for a few tokens: T[m, j] = bf16(s * sum_k X[m, k] A[j, k]), m < M <= 16.
+// One CTA per (adapter row j, pair of tokens); each thread takes 8 inputs per pass, sums them in fp32,
+// and the partial sums are combined in a fixed order (within each warp, then over the warps), so the
+// result does not depend on scheduling.  Used instead of the split-K tensor-core GEMM, whose 128-token
+// tiles, partial sums and reduction launch cost more than the whole product at these sizes.
+constexpr int kSmallTokens = 16;
+constexpr int kSmallPerCta = 2;
+
+__global__ void __launch_bounds__(256) lora_down_small_kernel(const uint16_t* __restrict__ X, int M, int64_t K,
+                                                              const uint16_t* __restrict__ A, int r, float s,
+                                                              uint16_t* __restrict__ T) {
+  __shared__ float part[8][kSmallPerCta];
+  pdl_launch_dependents();
+  pdl_wait();
+  const int j = blockIdx.x % r, m0 = (blockIdx.x / r) * kSmallPerCta;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float acc[kSmallPerCta];
+#pragma unroll
+  for (int m = 0; m < kSmallPerCta; ++m) acc[m] = 0.f;
+  const uint4* a = reinterpret_cast<const uint4*>(A + static_cast<int64_t>(j) * K);
+  const int64_t n8 = K / 8;
+  for (int64_t c = threadIdx.x; c < n8; c += 256) {
+    const uint4 av = __ldg(a + c);
+    const float af[8] = {lo_f(av.x), hi_f(av.x), lo_f(av.y), hi_f(av.y), lo_f(av.z), hi_f(av.z), lo_f(av.w), hi_f(av.w)};
+#pragma unroll
+    for (int m = 0; m < kSmallPerCta; ++m) {
+      if (m0 + m < M) {
+        const uint4 xv = __ldg(reinterpret_cast<const uint4*>(X + static_cast<int64_t>(m0 + m) * K) + c);
+        float d = af[0] * lo_f(xv.x);
+        d = fmaf(af[1], hi_f(xv.x), d);
+        d = fmaf(af[2], lo_f(xv.y), d);
+        d = fmaf(af[3], hi_f(xv.y), d);
+        d = fmaf(af[4], lo_f(xv.z), d);
+        d = fmaf(af[5], hi_f(xv.z), d);
+        d = fmaf(af[6], lo_f(xv.w), d);
+        d = fmaf(af[7], hi_f(xv.w), d);
+        acc[m] += d;
+      }
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < kSmallPerCta; ++m) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc[m] += __shfl_xor_sync(0xffffffffu, acc[m], o);
+    if (lane == 0) part[warp][m] = acc[m];
+  }
+  __syncthreads();
+  if (threadIdx.x < kSmallPerCta && m0 + threadIdx.x < M) {
+    float t = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) t += part[w][threadIdx.x];
+    T[static_cast<int64_t>(m0 + threadIdx.x) * r + j] = static_cast<uint16_t>(pack_bf16x2_rn(s * t, 0.f) & 0xFFFFu);
+  }
+}
+
 unsigned grid_for(int64_t n_items, int threads) {
   const int64_t want = (n_items + threads - 1) / threads;
   const int64_t cap = static_cast<int64_t>(device_sm_count()) * 8;
@@ -160,6 +215,14 @@ cudaError_t launch_swiglu_bwd(const uint16_t* dH, const uint16_t* G, const uint1
   return launch_pdl(swiglu_bwd_kernel, dim3(grid_for(n8, 256)), dim3(256), 0, st, reinterpret_cast<const uint4*>(dH),
                     reinterpret_cast<const uint4*>(G), reinterpret_cast<const uint4*>(U), reinterpret_cast<uint4*>(dG),
                     reinterpret_cast<uint4*>(dU), n8);
+}
+
+bool lora_down_small_supported(int64_t M) { return M >= 1 && M <= kSmallTokens; }
+
+cudaError_t launch_lora_down_small(const uint16_t* X, int64_t M, int64_t K, const uint16_t* A, int r, float s,
+                                   uint16_t* T, cudaStream_t st) {
+  const unsigned grid = static_cast<unsigned>(r * ((M + kSmallPerCta - 1) / kSmallPerCta));
+  return launch_pdl(lora_down_small_kernel, dim3(grid), dim3(256), 0, st, X, static_cast<int>(M), K, A, r, s, T);
 }
 
 cudaError_t launch_expand_adapter(const uint16_t* A, int r, int64_t K, int L, uint16_t* Aexp, cudaStream_t st) {
