@@ -324,6 +324,7 @@ int qlr_qalora_merge(const qlr_qweight* w, const uint16_t* A, const uint16_t* B,
 size_t qlr_forward_workspace_bytes(const qlr_qweight* w, int64_t M, int r, int pooled) {
   if (check_qweight(w) || M <= 0 || check_rank(r)) return 0;
   if (!pooled && lora_down_small_supported(M)) return 0;  // the few-token kernel needs no scratch
+  if (pooled && pooled_adapter_supported(w->K, w->group, r)) return 0;  // nor does the pooled-input kernel
   // the group expansion of A (pooled adapter), then the split partial sums
   return (pooled ? align256(size_t(r) * w->K * 2) : 0) + adapter_ws_bytes(M, w->K, r);
 }
@@ -347,6 +348,8 @@ int qlr_lora_down(const qlr_qweight* w, const uint16_t* X, int64_t M, const uint
   int32_t* stat = status_or_sink(status);
   const int64_t K = w->K;
   if (!pooled && lora_down_small_supported(M)) return cuda_rc(launch_lora_down_small(X, M, K, A, r, s, T_save, st));
+  if (pooled && pooled_adapter_supported(K, w->group, r))
+    return cuda_rc(launch_pooled_lora_down(X, M, K, w->group, A, r, s, T_save, st));
   // T_save = bf16(s * P(X) A^T) = bf16(s * X Aexp^T), Aexp[j, k] = A[j, k / L] / L for the pooled adapter
   const uint16_t* Ab = A;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -426,12 +429,12 @@ int qlr_forward(const qlr_qweight* w, const uint16_t* X, int64_t M, const uint16
 // ---- backward: adapter gradients -------------------------------------------------------------------
 
 size_t qlr_backward_lora_workspace_bytes(const qlr_qweight* w, int64_t M, int r, int pooled) {
-  (void)pooled;
   if (check_qweight(w) || M <= 0 || check_rank(r)) return 0;
-  // split partial sums of the three GEMMs, which run one after another
+  // split partial sums of the three GEMMs, which run one after another (the pooled adapter's dA
+  // comes from its own kernel and needs none)
   const size_t a = adapter_ws_bytes(M, w->N, r);
   const size_t b = adapter_ws_bytes(w->N, M, r);
-  const size_t c = adapter_ws_bytes(w->K, M, r);
+  const size_t c = (pooled && pooled_adapter_supported(w->K, w->group, r)) ? 0 : adapter_ws_bytes(w->K, M, r);
   return a > b ? (a > c ? a : c) : (b > c ? b : c);
 }
 
@@ -474,6 +477,9 @@ int qlr_backward_lora(const qlr_qweight* w, const uint16_t* X, const uint16_t* d
     AdapterGemm g{A_TMA_MN, B_TMA_MN, bn, N, M, dY, M, N, T_save, M, r};
     if ((rc = run_adapter(g, r, ADAPTER_ROWS_F32, 1.0f, 1, dB, r, ws, stat, st))) return rc;
   }
+  // pooled adapter: dA = dT^T P(X) from the group means of X
+  if (pooled && pooled_adapter_supported(K, w->group, r))
+    return cuda_rc(launch_pooled_dA(X, M, K, w->group, dT_out, r, dA, st));
   // dA^T = X^T dT over all K inputs; the pooled adapter sums each group of L inputs and divides by L
   {
     AdapterGemm g{A_TMA_MN, B_TMA_MN, bn, K, M, X, M, K, dT_out, M, r};

@@ -33,6 +33,13 @@ cudaError_t launch_swiglu_fwd(const uint16_t* G, const uint16_t* U, uint16_t* H,
 cudaError_t launch_swiglu_bwd(const uint16_t* dH, const uint16_t* G, const uint16_t* U, uint16_t* dG,
                               uint16_t* dU, int64_t n, cudaStream_t st);
 cudaError_t launch_expand_adapter(const uint16_t* A, int r, int64_t K, int L, uint16_t* Aexp, cudaStream_t st);
+// The pooled adapter (pooled.cu): T_save = bf16(s P(X) A^T) and dA = dT^T P(X) straight from X.
+bool pooled_adapter_supported(int64_t K, int L, int r);
+cudaError_t launch_pooled_lora_down(const uint16_t* X, int64_t M, int64_t K, int L, const uint16_t* A, int r, float s,
+                                    uint16_t* T, cudaStream_t st);
+cudaError_t launch_pooled_dA(const uint16_t* X, int64_t M, int64_t K, int L, const uint16_t* dT, int r, float* dA,
+                             cudaStream_t st);
+
 // T = bf16(s X A^T) for 1..16 tokens without pooling: one fixed-order reduction kernel, no workspace.
 bool lora_down_small_supported(int64_t M);
 cudaError_t launch_lora_down_small(const uint16_t* X, int64_t M, int64_t K, const uint16_t* A, int r, float s,

@@ -109,9 +109,8 @@ def test_host_validation_rejects_before_launch(L):
     q3 = _fake_qweight(bits=3, K=192)
     assert L.qlr_forward(ctypes.byref(q3), P(0x1000), 16, P(0x1000), P(0x1000), 8, 1.0, 0, P(0x1000), P(0x1000),
                          P(0x1000), 1 << 20, None, None) == -2
-    # missing workspace (the pooled adapter's group expansion needs one)
-    q4 = _fake_qweight(fmt=2, group=32)
-    assert L.qlr_forward(ctypes.byref(q4), P(0x1000), 16, P(0x1000), P(0x1000), 8, 1.0, 1, P(0x1000), P(0x1000),
+    # missing workspace (64 tokens: the adapter GEMM's split partial sums need one)
+    assert L.qlr_forward(ctypes.byref(q), P(0x1000), 64, P(0x1000), P(0x1000), 8, 1.0, 0, P(0x1000), P(0x1000),
                          None, 0, None, None) == -8
     # merge needs an INT4 group weight
     assert L.qlr_qalora_merge(ctypes.byref(q), P(0x1000), P(0x1000), 8, 1.0, None, None) == -1
