@@ -177,7 +177,8 @@ QLR_API int qlr_forward(const qlr_qweight* w, const uint16_t* X, int64_t M, cons
 
 /* The two stages of qlr_forward, callable separately (same arguments and buffers):
  *   qlr_lora_down     T_save = bf16(s * P(X) A^T)      (split-K tensor-core GEMM + fixed-order sum; for
- *                     1..16 tokens without pooling, one fixed-order reduction kernel and no workspace)
+ *                     1..16 tokens without pooling, and for the pooled adapter, one fixed-order
+ *                     reduction kernel straight from X and no workspace)
  *   qlr_forward_base  Y = bf16(X dequant(W)^T + T_save B^T)   (the fused dequant + tcgen05 kernel)
  * qlr_lora_down uses the workspace of qlr_forward_workspace_bytes; qlr_forward_base needs none. */
 QLR_API int qlr_lora_down(const qlr_qweight* w, const uint16_t* X, int64_t M, const uint16_t* A, int r, float s,
@@ -196,7 +197,8 @@ QLR_API uint64_t qlr_launch_count(void);
  *   dB = dY^T T_save               [N, r]   fp32
  *   dA = dT^T P(X)                 [r, Ka]  fp32  (dT taken in bf16)
  * Each fp32 reduction over tokens is split across CTAs and summed in a fixed order, so the
- * results are deterministic.
+ * results are deterministic.  With the pooled adapter (QA-LoRA), dA is formed directly from the group
+ * means of X (one CTA per group, tokens summed in a fixed order) and needs no workspace.
  */
 QLR_API size_t qlr_backward_lora_workspace_bytes(const qlr_qweight* w, int64_t M, int r, int pooled);
 QLR_API int qlr_backward_lora(const qlr_qweight* w, const uint16_t* X, const uint16_t* dY, const uint16_t* T_save,

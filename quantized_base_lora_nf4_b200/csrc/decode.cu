@@ -226,6 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       float acc[NT][4];
 #pragma unroll
       for (int n = 0; n < NT; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+      float my_scale = 0.f;  // this lane's share of the block scales of the current step pair
       for (int s = 0; s < nsteps; ++s) {
         const uint32_t j = jslot + s;
         const int sl = j % kSlots;
@@ -274,16 +275,23 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
               mma_bf16_16816(part[n], af, (m & 1) ? x4.z : x4.x, (m & 1) ? x4.w : x4.y);
             }
           }
-          const uint32_t b = static_cast<uint32_t>((s * 128 + 64 * hh) >> bshift);
-          float sa = 0.f, sb = 0.f;
-          if (va) {
-            const __half_raw hr = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(lds_u8(c8_a + b)), __NV_E4M3);
-            sa = __fmul_rn(__half2float(__half(hr)), lds_f32(s2_addr + ((s2_a + b) >> 8) * 4));
+          // block scales: the four lanes of a row pair share them, so on even steps lane t computes the
+          // scale of row (t odd ? b : a) at step s + t / 2, and every step fetches its two by shuffles
+          if ((s & 1) == 0) {
+            const int s_own = s + (t >> 1);
+            const bool v_own = (t & 1) ? vb : va;
+            my_scale = 0.f;
+            if (v_own && s_own < nsteps) {
+              const uint32_t b = static_cast<uint32_t>((s_own * 128 + 64 * hh) >> bshift);
+              const uint32_t c8_own = (t & 1) ? c8_b : c8_a, s2_own = (t & 1) ? s2_b : s2_a;
+              const __half_raw hr =
+                  __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(lds_u8(c8_own + b)), __NV_E4M3);
+              my_scale = __fmul_rn(__half2float(__half(hr)), lds_f32(s2_addr + ((s2_own + b) >> 8) * 4));
+            }
           }
-          if (vb) {
-            const __half_raw hr = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(lds_u8(c8_b + b)), __NV_E4M3);
-            sb = __fmul_rn(__half2float(__half(hr)), lds_f32(s2_addr + ((s2_b + b) >> 8) * 4));
-          }
+          const int src = (lane & ~3) + 2 * (s & 1);
+          const float sa = __shfl_sync(0xffffffffu, my_scale, src);
+          const float sb = __shfl_sync(0xffffffffu, my_scale, src + 1);
 #pragma unroll
           for (int n = 0; n < NT; ++n) {
             acc[n][0] = fmaf(sa, part[n][0], acc[n][0]);

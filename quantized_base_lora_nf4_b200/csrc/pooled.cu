@@ -46,6 +46,7 @@ __global__ void __launch_bounds__(256) pooled_lora_down_kernel(const uint16_t* _
   const int64_t n8 = K / 8;
   for (int64_t m = static_cast<int64_t>(blockIdx.x) * 8 + warp; m < M; m += static_cast<int64_t>(gridDim.x) * 8) {
     const uint4* xr = reinterpret_cast<const uint4*>(X + m * K);
+#pragma unroll 4
     for (int64_t c0 = 0; c0 < n8; c0 += 32) {
       const int64_t i = c0 + lane;
       float v = i < n8 ? sum8(__ldg(xr + i)) : 0.f;
@@ -76,6 +77,8 @@ __global__ void __launch_bounds__(256) pooled_dA_kernel(const uint16_t* __restri
   float acc[R];
 #pragma unroll
   for (int j = 0; j < R; ++j) acc[j] = 0.f;
+  constexpr int kUnroll = L >= 128 ? 2 : 4;  // tokens in flight per thread (X loads of L / 8 chunks each)
+#pragma unroll kUnroll
   for (int64_t m = threadIdx.x; m < M; m += 256) {
     const uint4* xr = reinterpret_cast<const uint4*>(X + m * K + static_cast<int64_t>(g) * L);
     float xs = 0.f;
