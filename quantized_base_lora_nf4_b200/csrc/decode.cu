@@ -170,7 +170,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
   __syncthreads();  // barriers and table ready
 
   {
-    const uint32_t jslot = 0;
     const int nu = u_end - u_begin;  // nu_lo or nu_lo + 1, at most kMaxUnits (host grid sizing)
     const int64_t prow0 = static_cast<int64_t>(u_begin) * 16;
     const int prows = static_cast<int>(static_cast<int64_t>(nu) * 16 < p.N - prow0 ? nu * 16 : p.N - prow0);
@@ -183,15 +182,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         const CUtensorMap* tm_codes = nu == p.nu_lo ? &tm_codes_lo : &tm_codes_hi;
         tma_prefetch_desc(tm_codes);
         tma_prefetch_desc(&tm_x);
+        int sl = 0;
+        uint32_t ph = 0;  // ring slot and the parity of its current fill
         for (int s = 0; s < nsteps; ++s) {
-          const uint32_t j = jslot + s;
-          const int sl = j % kSlots;
-          if (!mbar_wait(&bars->empty[sl], ((j / kSlots) & 1) ^ 1, abort_flag)) break;
+          if (!mbar_wait(&bars->empty[sl], ph ^ 1, abort_flag)) break;
           uint8_t* slot = gen(kRingAddr + sl * C::kSlot);
           mbar_arrive_expect_tx(&bars->full[sl], nu * 1024 + 2 * C::kXHalf);
           tma_load_2d(slot, tm_codes, s * 64, static_cast<int32_t>(prow0), &bars->full[sl]);
           tma_load_2d(slot + kMaxUnits * 1024, &tm_x, s * 128, 0, &bars->full[sl]);
           tma_load_2d(slot + kMaxUnits * 1024 + C::kXHalf, &tm_x, s * 128 + 64, 0, &bars->full[sl]);
+          if (++sl == kSlots) {
+            sl = 0;
+            ph ^= 1;
+          }
         }
       }
     } else {
@@ -227,10 +230,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
 #pragma unroll
       for (int n = 0; n < NT; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
       float my_scale = 0.f;  // this lane's share of the block scales of the current step pair
+      int sl = 0;
+      uint32_t ph = 0;  // ring slot and the parity of its current fill
+#pragma unroll 2
       for (int s = 0; s < nsteps; ++s) {
-        const uint32_t j = jslot + s;
-        const int sl = j % kSlots;
-        const bool ok = mbar_wait(&bars->full[sl], (j / kSlots) & 1, abort_flag);
+        const bool ok = mbar_wait(&bars->full[sl], ph, abort_flag);
         if (!__all_sync(0xffffffffu, ok)) break;
         // copy this step's ring data (this half's codes and input) to registers, then free the slot
         const uint32_t slot = kRingAddr + sl * C::kSlot;  // codes [unit][16 rows][64 B] (64-byte swizzle), then X
@@ -299,6 +303,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             acc[n][2] = fmaf(sb, part[n][2], acc[n][2]);
             acc[n][3] = fmaf(sb, part[n][3], acc[n][3]);
           }
+        }
+        if (++sl == kSlots) {
+          sl = 0;
+          ph ^= 1;
         }
       }
       // the second-half warp hands its sums to the first-half warp of the same unit
