@@ -57,11 +57,14 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// One step = 256 reduction inputs: per unit 16 rows x 128 code bytes (128-byte swizzle), and the input
+// tile as four quarters of [8 NT tokens][64 bf16].
 template <int NT>
 struct DCfg {
-  static constexpr int kXHalf = 8 * NT * 128;                   // [8 NT tokens][64 bf16]
-  static constexpr int kSlot = kMaxUnits * 1024 + 2 * kXHalf;   // codes of every unit + input tile
-  static constexpr int kSlots = NT == 1 ? 6 : 5;
+  static constexpr int kUnitCodes = 16 * 128;
+  static constexpr int kXQ = 8 * NT * 128;
+  static constexpr int kSlot = kMaxUnits * kUnitCodes + 4 * kXQ;
+  static constexpr int kSlots = NT == 1 ? 3 : 2;
 };
 
 // Shared-memory map, as shared-window addresses.  The dequantisation table sits at 64 KB so that one
@@ -149,7 +152,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
   // this CTA's contiguous range of 16-row units
   const int u_begin = static_cast<int>((static_cast<int64_t>(blockIdx.x) * p.units) / gridDim.x);
   const int u_end = static_cast<int>((static_cast<int64_t>(blockIdx.x + 1) * p.units) / gridDim.x);
-  const int nsteps = static_cast<int>(p.K / 128);
+  const int nsteps = static_cast<int>(p.K / 256);
 
   pdl_launch_dependents();
   pdl_wait();
@@ -177,7 +180,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
 
     if (warp == kComputeWarps) {
       // ---------------------------------------------------------------- TMA producer
-      // one box of all this CTA's rows (16 nu x 64 B of codes) and two input halves per step
+      // one box of all this CTA's rows (16 nu x 128 B of codes) and four input quarters per step
       if (lane == 0) {
         const CUtensorMap* tm_codes = nu == p.nu_lo ? &tm_codes_lo : &tm_codes_hi;
         tma_prefetch_desc(tm_codes);
@@ -187,10 +190,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         for (int s = 0; s < nsteps; ++s) {
           if (!mbar_wait(&bars->empty[sl], ph ^ 1, abort_flag)) break;
           uint8_t* slot = gen(kRingAddr + sl * C::kSlot);
-          mbar_arrive_expect_tx(&bars->full[sl], nu * 1024 + 2 * C::kXHalf);
-          tma_load_2d(slot, tm_codes, s * 64, static_cast<int32_t>(prow0), &bars->full[sl]);
-          tma_load_2d(slot + kMaxUnits * 1024, &tm_x, s * 128, 0, &bars->full[sl]);
-          tma_load_2d(slot + kMaxUnits * 1024 + C::kXHalf, &tm_x, s * 128 + 64, 0, &bars->full[sl]);
+          mbar_arrive_expect_tx(&bars->full[sl], nu * C::kUnitCodes + 4 * C::kXQ);
+          tma_load_2d(slot, tm_codes, s * 128, static_cast<int32_t>(prow0), &bars->full[sl]);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            tma_load_2d(slot + kMaxUnits * C::kUnitCodes + q * C::kXQ, &tm_x, s * 256 + 64 * q, 0, &bars->full[sl]);
           if (++sl == kSlots) {
             sl = 0;
             ph ^= 1;
@@ -208,101 +212,122 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       }
       named_bar_sync(1, kComputeWarps * 32);
       const int g = lane >> 2, t = lane & 3;
-      const int unit = warp >> 1, hh = warp & 1;  // this warp's unit and half (64 codes) of every step
+      const int unit = warp >> 1, hh = warp & 1;  // this warp's unit and half (quarters 2 hh, 2 hh + 1) of every step
       const bool active = unit < nu;
-      // MMA row g reads weight row pi(g) of the unit (bits 1 and 2 of g swapped), which spreads the eight
-      // byte code loads of each half-warp over all 32 banks under the 64-byte swizzle
-      const int pg = (g & 1) | ((g & 2) << 1) | ((g & 4) >> 1);
+      // MMA row g reads weight row pi(g): rows 0, 2, 4, 6 for g = 0..3 and 1, 3, 5, 7 for g = 4..7, which spreads
+      // each half-warp's code loads over all 32 banks under the 128-byte swizzle
+      const int pg = ((g & 3) << 1) | (g >> 2);
       const int lr_a = unit * 16 + pg, lr_b = lr_a + 8;  // rows of this CTA, 0 .. 16 nu - 1
       const int64_t ra = prow0 + lr_a, rb = prow0 + lr_b;
       const bool va = active && ra < p.N, vb = active && rb < p.N;
       const uint32_t lut_lane = kLutAddr | (4u * lane);
-      // per-lane parts of the shared addresses that do not change from step to step
-      // codes: 16-byte chunk 2 hh + t/2 of the row, 64-byte swizzle; input: chunks 2t, 2t+1 of a 128-byte row
-      const uint32_t code_a = unit * 1024 + pg * 64 + 8 * (t & 1), code_b = code_a + 8 * 64;
-      const uint32_t chunk_a = (((2 * hh + (t >> 1)) ^ ((pg >> 1) & 3)) << 4);
-      const uint32_t chunk_b = (((2 * hh + (t >> 1)) ^ (((pg + 8) >> 1) & 3)) << 4);
+      // per-lane parts of the shared addresses that do not change from step to step: quarter q of a row is
+      // 16-byte chunks 2q, 2q + 1 (lane t reads 8 bytes of chunk 2q + t/2), XOR-swizzled by the row index mod 8
+      // (rows pg and pg + 8 have the same index mod 8, so one swizzled chunk offset serves both)
+      const uint32_t code_a = unit * C::kUnitCodes + pg * 128 + 8 * (t & 1), code_b = code_a + 8 * 128;
+      const uint32_t chunk0 = static_cast<uint32_t>(((4 * hh + (t >> 1)) ^ (pg & 7)) << 4);
+      const uint32_t chunk1 = chunk0 ^ (2u << 4);  // quarter 2 hh + 1: chunk index + 2 (bit 1, untouched by t / 2)
       const uint32_t c8_a = c8_addr + lr_a * c8_stride, c8_b = c8_addr + lr_b * c8_stride;
       const uint32_t s2_off = static_cast<uint32_t>((prow0 * bpr) & 255);
       const uint32_t s2_a = lr_a * static_cast<uint32_t>(bpr) + s2_off, s2_b = lr_b * static_cast<uint32_t>(bpr) + s2_off;
       const int bshift = p.block_shift;
+      // lane t computes the scale of row (t odd ? b : a) in quarter 2 hh + t / 2; the other lanes of the row
+      // pair fetch it by shuffle
+      const bool v_own = (t & 1) ? vb : va;
+      const uint32_t c8_own = (t & 1) ? c8_b : c8_a, s2_own = (t & 1) ? s2_b : s2_a;
+      const int q_own = 2 * hh + (t >> 1);
       float acc[NT][4];
 #pragma unroll
       for (int n = 0; n < NT; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
-      float my_scale = 0.f;  // this lane's share of the block scales of the current step pair
+
+      // the input fragments of quarter q for this lane: X[tok][64 q + 16 t .. +15], two swizzled 16-byte chunks
+      auto load_x = [&](uint32_t xs, int q, uint4 (&xv)[NT][2]) {
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+          const int tok = 8 * n + g;
+          const uint32_t xr = xs + q * C::kXQ + tok * 128;
+          if (tok < p.M) {  // rows past the last token are zero; skipping them saves shared-memory wavefronts
+            xv[n][0] = lds_v4(xr + (((2 * t) ^ (tok & 7)) << 4));
+            xv[n][1] = lds_v4(xr + (((2 * t + 1) ^ (tok & 7)) << 4));
+          } else {
+            xv[n][0] = xv[n][1] = make_uint4(0u, 0u, 0u, 0u);
+          }
+        }
+      };
+      // one quarter: 4 MMAs per token tile on unscaled levels, then the block scale applied once
+      auto quarter = [&](const uint2 wa, const uint2 wb, const uint4 (&xv)[NT][2], float my_scale, int qi) {
+        float part[NT][4];
+#pragma unroll
+        for (int n = 0; n < NT; ++n) part[n][0] = part[n][1] = part[n][2] = part[n][3] = 0.f;
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          // this lane's codes: k = 256 s + 64 q + 16 t + i; MMA m takes i = 4m .. 4m+3 (bytes 2m, 2m+1)
+          const uint32_t qa = m < 2 ? wa.x : wa.y, qb = m < 2 ? wb.x : wb.y;
+          // byte permute: address bytes 0, 2, 3 from (4 lane | 64 KB), byte 1 = the code byte
+          constexpr uint32_t kSelLo[2] = {0x7604u, 0x7624u}, kSelHi[2] = {0x7614u, 0x7634u};
+          uint32_t af[4];
+          af[0] = lds_table(__byte_perm(qa, lut_lane, kSelLo[m & 1]));
+          af[2] = lds_table(__byte_perm(qa, lut_lane, kSelHi[m & 1]));
+          af[1] = lds_table(__byte_perm(qb, lut_lane, kSelLo[m & 1]));
+          af[3] = lds_table(__byte_perm(qb, lut_lane, kSelHi[m & 1]));
+#pragma unroll
+          for (int n = 0; n < NT; ++n) {
+            const uint4 x4 = xv[n][m >> 1];
+            mma_bf16_16816(part[n], af, (m & 1) ? x4.z : x4.x, (m & 1) ? x4.w : x4.y);
+          }
+        }
+        const float sa = __shfl_sync(0xffffffffu, my_scale, (lane & ~3) + 2 * qi);
+        const float sb = __shfl_sync(0xffffffffu, my_scale, (lane & ~3) + 2 * qi + 1);
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+          acc[n][0] = fmaf(sa, part[n][0], acc[n][0]);
+          acc[n][1] = fmaf(sa, part[n][1], acc[n][1]);
+          acc[n][2] = fmaf(sb, part[n][2], acc[n][2]);
+          acc[n][3] = fmaf(sb, part[n][3], acc[n][3]);
+        }
+      };
+
       int sl = 0;
       uint32_t ph = 0;  // ring slot and the parity of its current fill
-#pragma unroll 2
       for (int s = 0; s < nsteps; ++s) {
         const bool ok = mbar_wait(&bars->full[sl], ph, abort_flag);
         if (!__all_sync(0xffffffffu, ok)) break;
-        // copy this step's ring data (this half's codes and input) to registers, then free the slot
-        const uint32_t slot = kRingAddr + sl * C::kSlot;  // codes [unit][16 rows][64 B] (64-byte swizzle), then X
-        uint2 wa, wb;
-        uint4 xv[NT][2];
+        const uint32_t slot = kRingAddr + sl * C::kSlot;  // codes [unit][16 rows][128 B], then the input quarters
+        const uint32_t xs = slot + kMaxUnits * C::kUnitCodes;
         if (active) {
-          wa = lds_v2(slot + code_a + chunk_a);
-          wb = lds_v2(slot + code_b + chunk_b);
-          // input X[tok][64 hh + 16 t .. +15]: two 16-byte chunks of a 128-byte swizzled row
+          uint2 wa[2], wb[2];
+          wa[0] = lds_v2(slot + code_a + chunk0);
+          wb[0] = lds_v2(slot + code_b + chunk0);
+          wa[1] = lds_v2(slot + code_a + chunk1);
+          wb[1] = lds_v2(slot + code_b + chunk1);
+          float my_scale = 0.f;
+          if (v_own) {
+            const uint32_t b = static_cast<uint32_t>((s * 256 + 64 * q_own) >> bshift);
+            const __half_raw hr =
+                __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(lds_u8(c8_own + b)), __NV_E4M3);
+            my_scale = __fmul_rn(__half2float(__half(hr)), lds_f32(s2_addr + ((s2_own + b) >> 8) * 4));
+          }
+          if (NT == 1) {  // copy both quarters' input to registers and free the slot before the arithmetic
+            uint4 xv[2][NT][2];
+            load_x(xs, 2 * hh, xv[0]);
+            load_x(xs, 2 * hh + 1, xv[1]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->empty[sl]);
+            quarter(wa[0], wb[0], xv[0], my_scale, 0);
+            quarter(wa[1], wb[1], xv[1], my_scale, 1);
+          } else {  // 16 tokens: registers allow one quarter's input at a time; free the slot afterwards
 #pragma unroll
-          for (int n = 0; n < NT; ++n) {
-            const int tok = 8 * n + g;
-            const uint32_t xr = slot + kMaxUnits * 1024 + hh * C::kXHalf + tok * 128;
-            if (tok < p.M) {  // rows past the last token are zero; skipping them saves shared-memory wavefronts
-              xv[n][0] = lds_v4(xr + (((2 * t) ^ (tok & 7)) << 4));
-              xv[n][1] = lds_v4(xr + (((2 * t + 1) ^ (tok & 7)) << 4));
-            } else {
-              xv[n][0] = xv[n][1] = make_uint4(0u, 0u, 0u, 0u);
+            for (int qi = 0; qi < 2; ++qi) {
+              uint4 xv[NT][2];
+              load_x(xs, 2 * hh + qi, xv);
+              quarter(wa[qi], wb[qi], xv, my_scale, qi);
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->empty[sl]);
           }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->empty[sl]);
-        if (active) {
-          float part[NT][4];
-#pragma unroll
-          for (int n = 0; n < NT; ++n) part[n][0] = part[n][1] = part[n][2] = part[n][3] = 0.f;
-#pragma unroll
-          for (int m = 0; m < 4; ++m) {
-            // this lane's codes: k = 128 s + 64 hh + 16 t + i; MMA m takes i = 4m .. 4m+3 (bytes 2m, 2m+1)
-            const uint32_t qa = m < 2 ? wa.x : wa.y, qb = m < 2 ? wb.x : wb.y;
-            // byte permute: address bytes 0, 2, 3 from (4 lane | 64 KB), byte 1 = the code byte
-            constexpr uint32_t kSelLo[2] = {0x7604u, 0x7624u}, kSelHi[2] = {0x7614u, 0x7634u};
-            uint32_t af[4];
-            af[0] = lds_table(__byte_perm(qa, lut_lane, kSelLo[m & 1]));
-            af[2] = lds_table(__byte_perm(qa, lut_lane, kSelHi[m & 1]));
-            af[1] = lds_table(__byte_perm(qb, lut_lane, kSelLo[m & 1]));
-            af[3] = lds_table(__byte_perm(qb, lut_lane, kSelHi[m & 1]));
-#pragma unroll
-            for (int n = 0; n < NT; ++n) {
-              const uint4 x4 = xv[n][m >> 1];
-              mma_bf16_16816(part[n], af, (m & 1) ? x4.z : x4.x, (m & 1) ? x4.w : x4.y);
-            }
-          }
-          // block scales: the four lanes of a row pair share them, so on even steps lane t computes the
-          // scale of row (t odd ? b : a) at step s + t / 2, and every step fetches its two by shuffles
-          if ((s & 1) == 0) {
-            const int s_own = s + (t >> 1);
-            const bool v_own = (t & 1) ? vb : va;
-            my_scale = 0.f;
-            if (v_own && s_own < nsteps) {
-              const uint32_t b = static_cast<uint32_t>((s_own * 128 + 64 * hh) >> bshift);
-              const uint32_t c8_own = (t & 1) ? c8_b : c8_a, s2_own = (t & 1) ? s2_b : s2_a;
-              const __half_raw hr =
-                  __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(lds_u8(c8_own + b)), __NV_E4M3);
-              my_scale = __fmul_rn(__half2float(__half(hr)), lds_f32(s2_addr + ((s2_own + b) >> 8) * 4));
-            }
-          }
-          const int src = (lane & ~3) + 2 * (s & 1);
-          const float sa = __shfl_sync(0xffffffffu, my_scale, src);
-          const float sb = __shfl_sync(0xffffffffu, my_scale, src + 1);
-#pragma unroll
-          for (int n = 0; n < NT; ++n) {
-            acc[n][0] = fmaf(sa, part[n][0], acc[n][0]);
-            acc[n][1] = fmaf(sa, part[n][1], acc[n][1]);
-            acc[n][2] = fmaf(sb, part[n][2], acc[n][2]);
-            acc[n][3] = fmaf(sb, part[n][3], acc[n][3]);
-          }
+        } else {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars->empty[sl]);
         }
         if (++sl == kSlots) {
           sl = 0;
@@ -379,7 +404,7 @@ cudaError_t launch_decode_variant(const DecodeParams& p, int grid, const CUtenso
 }  // namespace
 
 bool decode_supported(const qlr_qweight* w, int64_t M) {
-  if (M < 1 || M > 16 || w->fmt != QLR_FMT_NFK || w->bits != 4 || w->dq_block != 256 || w->K % 128) return false;
+  if (M < 1 || M > 16 || w->fmt != QLR_FMT_NFK || w->bits != 4 || w->dq_block != 256 || w->K % 256) return false;
   // the constants fit below the table when the window starts within its first kilobyte
   return 1024 + decode_const_bytes(w->K / w->block) <= kLutAddr && decode_smem_bytes(M <= 8 ? 1 : 2) <= 227 * 1024;
 }
@@ -408,8 +433,8 @@ cudaError_t launch_decode(const qlr_qweight* w, const uint16_t* X, int64_t M, co
   p.status = status;
   const int nt = M <= 8 ? 1 : 2;
   CUtensorMap tc_lo, tc_hi, tx;
-  if (make_tmap(&tc_lo, w->codes, 1, w->N, w->K / 2, 16 * p.nu_lo, 64, 64)) return cudaErrorInvalidValue;
-  if (make_tmap(&tc_hi, w->codes, 1, w->N, w->K / 2, 16 * nu_hi, 64, 64)) return cudaErrorInvalidValue;
+  if (make_tmap(&tc_lo, w->codes, 1, w->N, w->K / 2, 16 * p.nu_lo, 128, 128)) return cudaErrorInvalidValue;
+  if (make_tmap(&tc_hi, w->codes, 1, w->N, w->K / 2, 16 * nu_hi, 128, 128)) return cudaErrorInvalidValue;
   if (make_tmap(&tx, X, 2, M, w->K, 8 * nt, 64, 128)) return cudaErrorInvalidValue;
   return nt == 1 ? launch_decode_variant<1>(p, grid, tc_lo, tc_hi, tx, st)
                  : launch_decode_variant<2>(p, grid, tc_lo, tc_hi, tx, st);

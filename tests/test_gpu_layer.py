@@ -159,6 +159,7 @@ def test_decode_projection_full_size_sampled_rows(cuda_lib, M):
 @pytest.mark.parametrize("M", [1, 5, 16])
 @pytest.mark.parametrize("block,r", [(64, 8), (128, 64)])
 def test_decode_ragged(cuda_lib, M, block, r):
-    """Decode kernel on a weight whose rows do not fill the last 64-row CTA."""
-    spec = LinearSpec("w", 320, 384, "nfk", 4, block, 256, r=r, s=0.5)
+    """Decode kernel (256-input steps) on a weight whose 20 units of 16 rows give one unit per CTA and whose
+    rows do not fill the last unit: 312 rows, K = 768 (three steps, an odd count)."""
+    spec = LinearSpec("w", 312, 768, "nfk", 4, block, 256, r=r, s=0.5)
     run_and_check(cuda_lib, spec, M, seed=11 + M)
