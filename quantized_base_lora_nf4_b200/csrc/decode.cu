@@ -3,10 +3,11 @@
 // At a few tokens the layer is a matrix-vector product bound by the HBM read of the packed 4-bit
 // codes (QLoRA explainer, "The complete QLoRA forward pass": each frozen NF4 block is dequantised to
 // bf16 on the fly and multiplied by the input).  One persistent CTA per SM owns a contiguous range of
-// 16-row units (about 12 for a 28672-row weight on 148 SMs), one compute warp per unit; a producer
-// warp streams every 128-wide reduction step -- each unit's codes (16 rows x 64 bytes, 64-byte
-// swizzle) and the input tile (tokens x 128, 128-byte swizzle) -- by TMA into a ring of shared-memory
-// slots that all compute warps consume in step.
+// 16-row units (12 or 13 for a 28672-row weight on 148 SMs), two compute warps per unit (each takes
+// half of every step); a producer warp streams every 256-wide reduction step -- one box of all the
+// CTA's codes (16 rows x 128 bytes per unit, 128-byte swizzle) and the input tile as four quarters of
+// tokens x 64 (128-byte swizzle) -- by TMA into a ring of shared-memory slots that all compute warps
+// consume in step.
 //
 // A code byte (two 4-bit codes) becomes the bf16 pair (level[lo], level[hi]) with one shared-memory
 // load from a 256-entry table replicated per lane (conflict-free), which is exactly one mma.sync
