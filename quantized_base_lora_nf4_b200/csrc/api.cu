@@ -430,11 +430,12 @@ int qlr_forward(const qlr_qweight* w, const uint16_t* X, int64_t M, const uint16
 
 size_t qlr_backward_lora_workspace_bytes(const qlr_qweight* w, int64_t M, int r, int pooled) {
   if (check_qweight(w) || M <= 0 || check_rank(r)) return 0;
-  // split partial sums of the three GEMMs, which run one after another (the pooled adapter's dA
-  // comes from its own kernel and needs none)
+  // split partial sums of the three GEMMs, which run one after another (the pooled adapter's dA: the
+  // partial sums of its token blocks)
   const size_t a = adapter_ws_bytes(M, w->N, r);
   const size_t b = adapter_ws_bytes(w->N, M, r);
-  const size_t c = (pooled && pooled_adapter_supported(w->K, w->group, r)) ? 0 : adapter_ws_bytes(w->K, M, r);
+  const size_t c = (pooled && pooled_adapter_supported(w->K, w->group, r)) ? pooled_dA_workspace_bytes(M, w->K, w->group, r)
+                                                                          : adapter_ws_bytes(w->K, M, r);
   return a > b ? (a > c ? a : c) : (b > c ? b : c);
 }
 
@@ -479,7 +480,7 @@ int qlr_backward_lora(const qlr_qweight* w, const uint16_t* X, const uint16_t* d
   }
   // pooled adapter: dA = dT^T P(X) from the group means of X
   if (pooled && pooled_adapter_supported(K, w->group, r))
-    return cuda_rc(launch_pooled_dA(X, M, K, w->group, dT_out, r, dA, st));
+    return cuda_rc(launch_pooled_dA(X, M, K, w->group, dT_out, r, dA, reinterpret_cast<float*>(ws), st));
   // dA^T = X^T dT over all K inputs; the pooled adapter sums each group of L inputs and divides by L
   {
     AdapterGemm g{A_TMA_MN, B_TMA_MN, bn, K, M, X, M, K, dT_out, M, r};

@@ -37,8 +37,9 @@ cudaError_t launch_expand_adapter(const uint16_t* A, int r, int64_t K, int L, ui
 bool pooled_adapter_supported(int64_t K, int L, int r);
 cudaError_t launch_pooled_lora_down(const uint16_t* X, int64_t M, int64_t K, int L, const uint16_t* A, int r, float s,
                                     uint16_t* T, cudaStream_t st);
+size_t pooled_dA_workspace_bytes(int64_t M, int64_t K, int L, int r);
 cudaError_t launch_pooled_dA(const uint16_t* X, int64_t M, int64_t K, int L, const uint16_t* dT, int r, float* dA,
-                             cudaStream_t st);
+                             float* part, cudaStream_t st);
 
 // T = bf16(s X A^T) for 1..16 tokens without pooling: one fixed-order reduction kernel, no workspace.
 bool lora_down_small_supported(int64_t M);

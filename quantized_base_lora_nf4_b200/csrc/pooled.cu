@@ -22,134 +22,159 @@ __device__ __forceinline__ float sum8(const uint4 q) {
   return ((lo_bf(q.x) + hi_bf(q.x)) + (lo_bf(q.y) + hi_bf(q.y))) + ((lo_bf(q.z) + hi_bf(q.z)) + (lo_bf(q.w) + hi_bf(q.w)));
 }
 
-// T_save: one warp per token.  Lanes walk the token's row in 16-byte chunks, the L / 8 lanes of a group
-// combine their sums with shuffles, the group means go to shared memory, and lane j then forms
-// T[m, j] = bf16(s sum_g mean_g A[j, g]) against the adapter staged (fp32, [G][r]) in shared memory.
+// T_save: one CTA per pair of tokens, K / 16 threads per token (each owns 4 consecutive 16-byte
+// chunks = 32 inputs, all loaded before any arithmetic).  The L / 32 threads of a group combine their
+// sums with shuffles and the group means go to shared memory; then 8 threads per output T[m, j]
+// split the K / L-long dot product with A and combine it with shuffles, in a fixed order.
+constexpr int kDownTok = 2;
+
 template <int L>
 __global__ void __launch_bounds__(256) pooled_lora_down_kernel(const uint16_t* __restrict__ X, int64_t M, int64_t K,
                                                                const uint16_t* __restrict__ A, int r, float s,
                                                                uint16_t* __restrict__ T) {
-  constexpr int LPG = L / 8;  // lanes per group
+  constexpr int TPG = L / 32;  // threads per group (1, 2 or 4)
   extern __shared__ float smem_f[];
   const int G = static_cast<int>(K / L);
-  float* sA = smem_f;                    // [G][r]
-  float* sXp = smem_f + G * r;           // [8 warps][G]
+  const int tpt = static_cast<int>(K / 32);  // threads per token
+  float* sXp = smem_f;                       // [kDownTok][G]
   pdl_launch_dependents();
   pdl_wait();
-  for (int i = threadIdx.x; i < G * r; i += blockDim.x) {
-    const int g = i / r, j = i - g * r;
-    sA[i] = __uint_as_float(static_cast<uint32_t>(A[static_cast<int64_t>(j) * G + g]) << 16);
+  const int64_t m0 = static_cast<int64_t>(blockIdx.x) * kDownTok;
+  // pooling: thread i of token tk sums inputs [32 i, 32 i + 32) of row m0 + tk
+  // the loop bound is uniform over the CTA so that every lane reaches the shuffles; a group's TPG
+  // threads are adjacent lanes and never straddle the end (tpt is a multiple of TPG)
+  for (int base = 0; base < kDownTok * tpt; base += blockDim.x) {
+    const int i = base + threadIdx.x;
+    const bool in = i < kDownTok * tpt;
+    const int tk = in ? i / tpt : 0, c = in ? i - tk * tpt : 0;
+    float v = 0.f;
+    if (in && m0 + tk < M) {
+      const uint4* xr = reinterpret_cast<const uint4*>(X + (m0 + tk) * K) + 4 * c;
+      const uint4 q0 = __ldg(xr), q1 = __ldg(xr + 1), q2 = __ldg(xr + 2), q3 = __ldg(xr + 3);
+      v = (sum8(q0) + sum8(q1)) + (sum8(q2) + sum8(q3));
+    }
+#pragma unroll
+    for (int o = TPG / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (in && (c & (TPG - 1)) == 0) sXp[tk * G + c / TPG] = v * (1.0f / L);  // L is a power of two: exact
   }
   __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float* xp = sXp + warp * G;
-  const int64_t n8 = K / 8;
-  for (int64_t m = static_cast<int64_t>(blockIdx.x) * 8 + warp; m < M; m += static_cast<int64_t>(gridDim.x) * 8) {
-    const uint4* xr = reinterpret_cast<const uint4*>(X + m * K);
-#pragma unroll 4
-    for (int64_t c0 = 0; c0 < n8; c0 += 32) {
-      const int64_t i = c0 + lane;
-      float v = i < n8 ? sum8(__ldg(xr + i)) : 0.f;
-#pragma unroll
-      for (int o = LPG / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      if (i < n8 && (lane & (LPG - 1)) == 0) xp[i / LPG] = v * (1.0f / L);  // L is a power of two: exact
-    }
-    __syncwarp();
-    for (int j = lane; j < r; j += 32) {
-      float acc = 0.f;
-      for (int g = 0; g < G; ++g) acc = fmaf(xp[g], sA[g * r + j], acc);
-      T[m * r + j] = static_cast<uint16_t>(pack_bf16x2_rn(s * acc, 0.f) & 0xFFFFu);
-    }
-    __syncwarp();
+  // T[m0 + tk, j]: 8 threads per output, group g = sub, sub + 8, ...
+  const int sub = threadIdx.x & 7;
+  for (int o = threadIdx.x >> 3; o < kDownTok * r; o += blockDim.x >> 3) {
+    const int tk = o / r, j = o - tk * r;
+    const float* xp = sXp + tk * G;
+    const uint16_t* arow = A + static_cast<int64_t>(j) * G;
+    float acc = 0.f;
+    for (int g = sub; g < G; g += 8) acc = fmaf(xp[g], __uint_as_float(static_cast<uint32_t>(__ldg(arow + g)) << 16), acc);
+    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+    acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+    if (sub == 0 && m0 + tk < M)
+      T[(m0 + tk) * r + j] = static_cast<uint16_t>(pack_bf16x2_rn(s * acc, 0.f) & 0xFFFFu);
   }
 }
 
-// dA: one CTA per group g.  Thread t takes tokens t, t + 256, ...: the group mean of X[m] times the
-// token's dT row, accumulated in fp32 registers, then summed over the CTA in a fixed order.
-template <int L, int R>
-__global__ void __launch_bounds__(256) pooled_dA_kernel(const uint16_t* __restrict__ X, int64_t M, int64_t K,
-                                                        const uint16_t* __restrict__ dT, float* __restrict__ dA) {
-  __shared__ float red[8][R];
+// dA, first pass: one CTA per block of 16 tokens pools their rows (coalesced, as above) into shared
+// memory with their dT rows, and writes the block's partial dA[j, g] = sum_m dT[m, j] mean_g(X[m]).
+constexpr int kDaTok = 16;
+
+template <int L>
+__global__ void __launch_bounds__(256) pooled_dA_partial_kernel(const uint16_t* __restrict__ X, int64_t M, int64_t K,
+                                                                const uint16_t* __restrict__ dT, int r,
+                                                                float* __restrict__ part) {
+  constexpr int TPG = L / 32;
+  extern __shared__ float smem_f[];
+  const int G = static_cast<int>(K / L);
+  const int tpt = static_cast<int>(K / 32);
+  float* sXp = smem_f;                  // [kDaTok][G]
+  float* sdT = smem_f + kDaTok * G;     // [kDaTok][r]
   pdl_launch_dependents();
   pdl_wait();
-  const int G = static_cast<int>(K / L), g = blockIdx.x;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float acc[R];
-#pragma unroll
-  for (int j = 0; j < R; ++j) acc[j] = 0.f;
-  constexpr int kUnroll = L >= 128 ? 2 : 4;  // tokens in flight per thread (X loads of L / 8 chunks each)
-#pragma unroll kUnroll
-  for (int64_t m = threadIdx.x; m < M; m += 256) {
-    const uint4* xr = reinterpret_cast<const uint4*>(X + m * K + static_cast<int64_t>(g) * L);
-    float xs = 0.f;
-#pragma unroll
-    for (int c = 0; c < L / 8; ++c) xs += sum8(__ldg(xr + c));
-    xs *= 1.0f / L;
-    const uint4* tr = reinterpret_cast<const uint4*>(dT + m * R);
-#pragma unroll
-    for (int c = 0; c < R / 8; ++c) {
-      const uint4 q = __ldg(tr + c);
-      acc[8 * c + 0] = fmaf(lo_bf(q.x), xs, acc[8 * c + 0]);
-      acc[8 * c + 1] = fmaf(hi_bf(q.x), xs, acc[8 * c + 1]);
-      acc[8 * c + 2] = fmaf(lo_bf(q.y), xs, acc[8 * c + 2]);
-      acc[8 * c + 3] = fmaf(hi_bf(q.y), xs, acc[8 * c + 3]);
-      acc[8 * c + 4] = fmaf(lo_bf(q.z), xs, acc[8 * c + 4]);
-      acc[8 * c + 5] = fmaf(hi_bf(q.z), xs, acc[8 * c + 5]);
-      acc[8 * c + 6] = fmaf(lo_bf(q.w), xs, acc[8 * c + 6]);
-      acc[8 * c + 7] = fmaf(hi_bf(q.w), xs, acc[8 * c + 7]);
+  const int64_t m0 = static_cast<int64_t>(blockIdx.x) * kDaTok;
+  for (int base = 0; base < kDaTok * tpt; base += blockDim.x) {  // uniform bound: see above
+    const int i = base + threadIdx.x;
+    const bool in = i < kDaTok * tpt;
+    const int tk = in ? i / tpt : 0, c = in ? i - tk * tpt : 0;
+    float v = 0.f;
+    if (in && m0 + tk < M) {
+      const uint4* xr = reinterpret_cast<const uint4*>(X + (m0 + tk) * K) + 4 * c;
+      const uint4 q0 = __ldg(xr), q1 = __ldg(xr + 1), q2 = __ldg(xr + 2), q3 = __ldg(xr + 3);
+      v = (sum8(q0) + sum8(q1)) + (sum8(q2) + sum8(q3));
     }
+#pragma unroll
+    for (int o = TPG / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (in && (c & (TPG - 1)) == 0) sXp[tk * G + c / TPG] = v * (1.0f / L);
   }
-#pragma unroll
-  for (int j = 0; j < R; ++j) {
-    float v = acc[j];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if (lane == 0) red[warp][j] = v;
+  for (int i = threadIdx.x; i < kDaTok * r; i += blockDim.x) {
+    const int tk = i / r;
+    sdT[i] = (m0 + tk < M) ? __uint_as_float(static_cast<uint32_t>(dT[m0 * r + i]) << 16) : 0.f;
   }
   __syncthreads();
-  if (threadIdx.x < R) {
-    float t = 0.f;
+  float* out = part + static_cast<int64_t>(blockIdx.x) * r * G;
+  for (int o = threadIdx.x; o < r * G; o += blockDim.x) {
+    const int j = o / G, g = o - j * G;
+    float acc = 0.f;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) t += red[w][threadIdx.x];
-    dA[static_cast<int64_t>(threadIdx.x) * G + g] = t;
+    for (int tk = 0; tk < kDaTok; ++tk) acc = fmaf(sdT[tk * r + j], sXp[tk * G + g], acc);
+    out[o] = acc;
   }
 }
 
-size_t lora_down_smem(int64_t K, int L, int r) { return static_cast<size_t>(K / L) * (r + 8) * 4; }
+// dA, second pass: dA[j, g] = sum over the token blocks of the partials, in block order.
+__global__ void __launch_bounds__(256) pooled_dA_reduce_kernel(const float* __restrict__ part, int nblk, int n,
+                                                               float* __restrict__ dA) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int o = blockIdx.x * blockDim.x + threadIdx.x;
+  if (o >= n) return;
+  float acc = 0.f;
+  for (int b = 0; b < nblk; ++b) acc += part[static_cast<int64_t>(b) * n + o];
+  dA[o] = acc;
+}
+
+size_t lora_down_smem(int64_t K, int L) { return static_cast<size_t>(K / L) * kDownTok * 4; }
+size_t dA_smem(int64_t K, int L, int r) { return (static_cast<size_t>(K / L) + r) * kDaTok * 4; }
+
+template <typename Kern>
+cudaError_t allow_smem(Kern kern, size_t smem) {
+  if (smem <= 48 * 1024) return cudaSuccess;
+  return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+}
 
 template <int L>
 cudaError_t launch_down_L(const uint16_t* X, int64_t M, int64_t K, const uint16_t* A, int r, float s, uint16_t* T,
                           cudaStream_t st) {
-  const size_t smem = lora_down_smem(K, L, r);
-  if (smem > 48 * 1024) {
-    const cudaError_t e =
-        cudaFuncSetAttribute(pooled_lora_down_kernel<L>, cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024);
-    if (e != cudaSuccess) return e;
-  }
-  int64_t grid = (M + 7) / 8;
-  const int64_t cap = static_cast<int64_t>(device_sm_count()) * 4;
-  if (grid > cap) grid = cap;
-  return launch_pdl(pooled_lora_down_kernel<L>, dim3(static_cast<unsigned>(grid)), dim3(256), smem, st, X, M, K, A, r,
-                    s, T);
+  const size_t smem = lora_down_smem(K, L);
+  cudaError_t e = allow_smem(pooled_lora_down_kernel<L>, smem);
+  if (e != cudaSuccess) return e;
+  const unsigned grid = static_cast<unsigned>((M + kDownTok - 1) / kDownTok);
+  return launch_pdl(pooled_lora_down_kernel<L>, dim3(grid), dim3(256), smem, st, X, M, K, A, r, s, T);
 }
 
 template <int L>
-cudaError_t launch_dA_L(const uint16_t* X, int64_t M, int64_t K, const uint16_t* dT, int r, float* dA, cudaStream_t st) {
-  const dim3 grid(static_cast<unsigned>(K / L)), block(256);
-  switch (r) {
-    case 8: return launch_pdl(pooled_dA_kernel<L, 8>, grid, block, 0, st, X, M, K, dT, dA);
-    case 16: return launch_pdl(pooled_dA_kernel<L, 16>, grid, block, 0, st, X, M, K, dT, dA);
-    case 32: return launch_pdl(pooled_dA_kernel<L, 32>, grid, block, 0, st, X, M, K, dT, dA);
-    case 64: return launch_pdl(pooled_dA_kernel<L, 64>, grid, block, 0, st, X, M, K, dT, dA);
-    default: return cudaErrorInvalidValue;
-  }
+cudaError_t launch_dA_L(const uint16_t* X, int64_t M, int64_t K, const uint16_t* dT, int r, float* dA, float* part,
+                        cudaStream_t st) {
+  const size_t smem = dA_smem(K, L, r);
+  cudaError_t e = allow_smem(pooled_dA_partial_kernel<L>, smem);
+  if (e != cudaSuccess) return e;
+  const int nblk = static_cast<int>((M + kDaTok - 1) / kDaTok);
+  e = launch_pdl(pooled_dA_partial_kernel<L>, dim3(static_cast<unsigned>(nblk)), dim3(256), smem, st, X, M, K, dT, r,
+                 part);
+  if (e != cudaSuccess) return e;
+  const int n = static_cast<int>(r * (K / L));
+  return launch_pdl(pooled_dA_reduce_kernel, dim3(static_cast<unsigned>((n + 255) / 256)), dim3(256), 0, st,
+                    static_cast<const float*>(part), nblk, n, dA);
 }
 
 }  // namespace
 
 bool pooled_adapter_supported(int64_t K, int L, int r) {
   return (L == 32 || L == 64 || L == 128) && K % L == 0 && (r == 8 || r == 16 || r == 32 || r == 64) &&
-         lora_down_smem(K, L, r) <= 160 * 1024;
+         dA_smem(K, L, r) <= 160 * 1024;
+}
+
+size_t pooled_dA_workspace_bytes(int64_t M, int64_t K, int L, int r) {
+  return static_cast<size_t>((M + kDaTok - 1) / kDaTok) * r * (K / L) * 4;
 }
 
 cudaError_t launch_pooled_lora_down(const uint16_t* X, int64_t M, int64_t K, int L, const uint16_t* A, int r, float s,
@@ -163,11 +188,11 @@ cudaError_t launch_pooled_lora_down(const uint16_t* X, int64_t M, int64_t K, int
 }
 
 cudaError_t launch_pooled_dA(const uint16_t* X, int64_t M, int64_t K, int L, const uint16_t* dT, int r, float* dA,
-                             cudaStream_t st) {
+                             float* part, cudaStream_t st) {
   switch (L) {
-    case 32: return launch_dA_L<32>(X, M, K, dT, r, dA, st);
-    case 64: return launch_dA_L<64>(X, M, K, dT, r, dA, st);
-    case 128: return launch_dA_L<128>(X, M, K, dT, r, dA, st);
+    case 32: return launch_dA_L<32>(X, M, K, dT, r, dA, part, st);
+    case 64: return launch_dA_L<64>(X, M, K, dT, r, dA, part, st);
+    case 128: return launch_dA_L<128>(X, M, K, dT, r, dA, part, st);
     default: return cudaErrorInvalidValue;
   }
 }
