@@ -91,6 +91,7 @@ __global__ void __launch_bounds__(256) pooled_dA_partial_kernel(const uint16_t* 
   pdl_launch_dependents();
   pdl_wait();
   const int64_t m0 = static_cast<int64_t>(blockIdx.x) * kDaTok;
+#pragma unroll 4
   for (int base = 0; base < kDaTok * tpt; base += blockDim.x) {  // uniform bound: see above
     const int i = base + threadIdx.x;
     const bool in = i < kDaTok * tpt;
@@ -120,16 +121,29 @@ __global__ void __launch_bounds__(256) pooled_dA_partial_kernel(const uint16_t* 
   }
 }
 
-// dA, second pass: dA[j, g] = sum over the token blocks of the partials, in block order.
+// dA, second pass: dA[j, g] = sum over the token blocks of the partials.  A CTA takes 32 consecutive
+// outputs; warp w sums the blocks w, w + 8, ... (coalesced rows of 32 partials, several loads in
+// flight) and the eight warp sums are added in warp order, so the result is deterministic.
 __global__ void __launch_bounds__(256) pooled_dA_reduce_kernel(const float* __restrict__ part, int nblk, int n,
                                                                float* __restrict__ dA) {
+  __shared__ float red[8][32];
   pdl_launch_dependents();
   pdl_wait();
-  const int o = blockIdx.x * blockDim.x + threadIdx.x;
-  if (o >= n) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int o = blockIdx.x * 32 + lane;
   float acc = 0.f;
-  for (int b = 0; b < nblk; ++b) acc += part[static_cast<int64_t>(b) * n + o];
-  dA[o] = acc;
+  if (o < n) {
+#pragma unroll 4
+    for (int b = warp; b < nblk; b += 8) acc += part[static_cast<int64_t>(b) * n + o];
+  }
+  red[warp][lane] = acc;
+  __syncthreads();
+  if (warp == 0 && o < n) {
+    float t = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) t += red[w][lane];
+    dA[o] = t;
+  }
 }
 
 size_t lora_down_smem(int64_t K, int L) { return static_cast<size_t>(K / L) * kDownTok * 4; }
@@ -162,7 +176,7 @@ cudaError_t launch_dA_L(const uint16_t* X, int64_t M, int64_t K, const uint16_t*
                  part);
   if (e != cudaSuccess) return e;
   const int n = static_cast<int>(r * (K / L));
-  return launch_pdl(pooled_dA_reduce_kernel, dim3(static_cast<unsigned>((n + 255) / 256)), dim3(256), 0, st,
+  return launch_pdl(pooled_dA_reduce_kernel, dim3(static_cast<unsigned>((n + 31) / 32)), dim3(256), 0, st,
                     static_cast<const float*>(part), nblk, n, dA);
 }
 
