@@ -148,6 +148,32 @@ QLR_API int qlr_quantize_int4_group(const float* W, int64_t N, int64_t K, int gr
 QLR_API int qlr_dequant(const qlr_qweight* w, uint16_t* W_out, int32_t* status, void* stream);
 
 /*
+ * LQ-LoRA initialisation (LQ-LoRA abstract: an iterative algorithm decomposes each pretrained matrix
+ * into a high-precision low-rank component and a memory-efficient quantized component; the quantized
+ * part stays frozen and the low-rank part is the adapter).  Read as the alternation
+ *   Q_0 = 0;  for t = 1..iters:  L_t = rank-r truncated SVD of (W - dequant(Q_{t-1})),
+ *                                Q_t = NF-k quantisation (bits, block, dq_block) of (W - L_t)
+ * with, from the last SVD L = U_r S_r V_r^T,  A = bf16(sqrt(S_r) V_r^T)  [r, K]  and
+ * B = bf16(U_r sqrt(S_r) / s)  [N, r], so that dequant(Q) + s B A approximates W.  iters = 0 is plain
+ * quantisation with A = B = 0.
+ *   W       fp32 [N, K] row-major (device, 16-byte aligned), read only.
+ *   out     NF-k weight descriptor with buffers sized by qlr_qweight_part_bytes (fmt, bits, block,
+ *           dq_block, N, K must match the arguments); codes and constants are written.
+ *   r       1 .. 64 and <= min(N, K);  s > 0;  iters 0 .. 64.
+ *   workspace  qlr_lqlora_init_workspace_bytes(N, K, r) bytes, 256-byte aligned (residual, the SVD
+ *           factors and cuSOLVER's work area; about 4 N K floats).
+ * The SVD is cuSOLVER's single-precision gesvd, loaded at run time; without it the call returns
+ * QLR_ERR_UNSUPPORTED (iters = 0 needs no solver).  This is an offline, once-per-weight call: it
+ * synchronises the stream (the factorisation's status is read back after every SVD) and creates its
+ * solver handle per call.  Singular vectors are unique up to sign, so A and B may differ in sign from
+ * another implementation's; their product does not.
+ */
+QLR_API size_t qlr_lqlora_init_workspace_bytes(int64_t N, int64_t K, int r);
+QLR_API int qlr_lqlora_init(const float* W, int64_t N, int64_t K, int bits, int block, int dq_block, int r, float s,
+                            int iters, qlr_qweight* out, uint16_t* A, uint16_t* B, void* workspace,
+                            size_t workspace_bytes, int32_t* status, void* stream);
+
+/*
  * QA-LoRA merge (QA-LoRA abstract: after fine-tuning the adapter is integrated into the
  * quantised model without loss of accuracy).  With the pooled adapter, s (B A)[o, g] / L is
  * added to every weight of group g of row o, which is a shift of the zero point:

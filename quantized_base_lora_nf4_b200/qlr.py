@@ -29,7 +29,8 @@ EXPORTED = (
     "qlr_quantize_int4_group", "qlr_dequant", "qlr_qalora_merge", "qlr_forward_workspace_bytes", "qlr_forward",
     "qlr_backward_lora_workspace_bytes", "qlr_backward_lora", "qlr_backward_dx_workspace_bytes",
     "qlr_backward_dx", "qlr_swiglu_forward", "qlr_swiglu_backward", "qlr_device_sm_count", "qlr_lora_down",
-    "qlr_forward_base", "qlr_launch_count", "qlr_backward_lora_noalloc",
+    "qlr_forward_base", "qlr_launch_count", "qlr_backward_lora_noalloc", "qlr_lqlora_init_workspace_bytes",
+    "qlr_lqlora_init",
 )
 
 
@@ -81,6 +82,8 @@ def lib() -> ctypes.CDLL:
         "qlr_forward_base": (I, [QP, P, I64, P, I, P, P, P, P]),
         "qlr_launch_count": (ctypes.c_uint64, []),
         "qlr_backward_lora_noalloc": (I, [QP, P, P, P, P, I64, I, F, I, P, P, P, P, P]),
+        "qlr_lqlora_init_workspace_bytes": (SZ, [I64, I64, I]),
+        "qlr_lqlora_init": (I, [P, I64, I64, I, I, I, I, F, I, QP, P, P, P, SZ, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -213,6 +216,20 @@ def dequant(q: QWeight, out: Optional[torch.Tensor] = None, stream=None) -> torc
 def qalora_merge(q: QWeight, A: torch.Tensor, B: torch.Tensor, s: float, stream=None) -> None:
     _check(lib().qlr_qalora_merge(q.ref(), _ptr(A), _ptr(B), A.shape[0], float(s), None, _stream(stream)),
            "qlr_qalora_merge")
+
+
+def lqlora_init(W: torch.Tensor, bits: int, block: int, dq_block: int, r: int, s: float, iters: int,
+                status: Optional[torch.Tensor] = None, stream=None) -> Tuple[QWeight, torch.Tensor, torch.Tensor]:
+    """LQ-LoRA initialisation of an fp32 weight: the quantised part and the adapter (A [r, K], B [N, r])."""
+    N, K = W.shape
+    q = alloc_qweight(FMT_NFK, N, K, W.device, bits, block, dq_block)
+    A = torch.empty((r, K), dtype=torch.bfloat16, device=W.device)
+    B = torch.empty((N, r), dtype=torch.bfloat16, device=W.device)
+    nbytes = int(lib().qlr_lqlora_init_workspace_bytes(N, K, r)) if iters > 0 else 0
+    ws = _empty(max(nbytes, 256), W.device)
+    _check(lib().qlr_lqlora_init(_ptr(W), N, K, bits, block, dq_block, r, float(s), iters, q.ref(), _ptr(A), _ptr(B),
+                                 _ptr(ws), nbytes, _ptr(status), _stream(stream)), "qlr_lqlora_init")
+    return q, A, B
 
 
 class Workspace:
