@@ -47,7 +47,8 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="qalora", choices=["qalora", "tiny", "mlp7b", "lqlora", "decode70b"])
+    ap.add_argument("--workload", default="qalora",
+                    choices=["qalora", "tiny", "mlp7b", "lqlora", "decode70b", "lqlora_init"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -478,6 +479,41 @@ def oracle_tokens_per_s(wl, seed, budget_s=12.0):
             "sample": f"{what}, fwd+bwd in fp64 numpy ({el:.1f} s; dequantised weights prepared untimed)"}
 
 
+# ------------------------------------------------------------------------------------------ LQ-LoRA init
+def run_lqlora_init(args, dev, iters: int = 2):
+    """LQ-LoRA initialisation (alternating rank-64 SVD of the residual and NF-k quantisation) of the first
+    matrix of each distinct shape of the 7B stack, with its drawn bit width and block; CUDA-event time of
+    the whole call (the SVD is cuSOLVER's), projected to the stack's 224 matrices."""
+    import torch
+    from quantized_base_lora_nf4_b200 import qlr
+    from synth import workload
+
+    wl = workload("lqlora", args.seed)
+    seen, out = {}, {}
+    for spec in wl.linears:
+        if (spec.N, spec.K) in seen:
+            continue
+        g = torch.Generator(device=dev)
+        g.manual_seed(args.seed)
+        W = torch.randn((spec.N, spec.K), generator=g, device=dev, dtype=torch.float32) * spec.sigma_w
+        qlr.lqlora_init(W, spec.bits, spec.block, spec.dq_block, spec.r, spec.s, iters)  # warm-up (solver load)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        qlr.lqlora_init(W, spec.bits, spec.block, spec.dq_block, spec.r, spec.s, iters)
+        e1.record()
+        torch.cuda.synchronize()
+        seen[(spec.N, spec.K)] = e0.elapsed_time(e1)
+        out[f"{spec.N}x{spec.K}"] = {"ms": seen[(spec.N, spec.K)], "bits": spec.bits, "block": spec.block,
+                                     "r": spec.r, "iters": iters}
+        del W
+    stack_s = sum(seen[(s_.N, s_.K)] for s_ in wl.linears) / 1e3
+    return {"metric": "LQ-LoRA initialisation time per matrix (ms), whole call", "per_shape": out,
+            "stack_projection_s": stack_s, "stack_matrices": len(wl.linears),
+            "note": "truncated SVD: single-precision cuSOLVER gesvd on the full matrix; residual, rank-r "
+                    "subtraction, factor split and quantisation in this library's kernels"}
+
+
 # ------------------------------------------------------------------------------------------ decode shape
 def run_decode(args, dev):
     """Forward of the 28672 x 8192 NF4+DQ projection at 1, 4 and 16 tokens: HBM-bound on the codes."""
@@ -538,7 +574,7 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     from synth import workload
 
-    wl = workload(args.workload, args.seed)
+    wl = workload("lqlora" if args.workload == "lqlora_init" else args.workload, args.seed)
     fl_tok = sum(flops_per_token(s) for s in wl.linears)
     lin = [{"name": s.name, "N": s.N, "K": s.K, "r": s.r, "format": s.fmt, "bits": s.bits if s.fmt == "nfk" else 4,
             "block": s.block if s.fmt == "nfk" else s.group} for s in wl.linears]
@@ -575,6 +611,13 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     dev = torch.device("cuda", local if world > 1 else 0)
     torch.cuda.set_device(dev)
+    if args.workload == "lqlora_init":
+        if rank == 0:
+            print(json.dumps(run_lqlora_init(args, dev)))
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return 0
     if args.workload == "decode70b":
         if rank == 0:
             print(json.dumps({"metric": "decode forward time and HBM GB/s on the 4-bit code bytes",
