@@ -174,6 +174,35 @@ QLR_API int qlr_lqlora_init(const float* W, int64_t N, int64_t K, int bits, int 
                             size_t workspace_bytes, int32_t* status, void* stream);
 
 /*
+ * Squared reconstruction error of NF-k quantisation, ||W - dequant(Q(W))||_F^2 with the dequantised
+ * bf16 weight the layer uses: the per-option input of qlr_lqlora_allocate.
+ *   W        fp32 [N, K] (device, 16-byte aligned);  bits 2..4, block 64 or 128, dq_block 0 or 256.
+ *   err_out  one double in DEVICE memory (8-byte aligned), written on the stream.
+ *   workspace  qlr_nf_quant_error_workspace_bytes(...) bytes, 256-byte aligned (the quantised weight
+ *            and the fp64 partial sums).  Deterministic: fixed mapping and reduction order.
+ */
+QLR_API size_t qlr_nf_quant_error_workspace_bytes(int64_t N, int64_t K, int bits, int block, int dq_block);
+QLR_API int qlr_nf_quant_error(const float* W, int64_t N, int64_t K, int bits, int block, int dq_block,
+                               double* err_out, void* workspace, size_t workspace_bytes, int32_t* status,
+                               void* stream);
+
+/*
+ * LQ-LoRA's budgeted allocation (LQ-LoRA abstract: an integer linear programming formulation that
+ * configures the quantisation parameters, e.g. bit width and block size, of each matrix for an overall
+ * memory budget).  Read as a multiple-choice knapsack: matrix i takes one option o out of n_opt with
+ * error err[i * n_opt + o] and storage cost_bits[i * n_opt + o]; the summed error is minimised with the
+ * summed storage within budget_bits.  Exact dynamic programming over the budget in whole units of
+ * unit_bits (costs rounded up, so the plan never exceeds the budget); the plan is read back last matrix
+ * first, each taking the lowest option index among its minima.  HOST memory, no GPU:
+ *   err        double [n_mat * n_opt];  cost_bits  int64 [n_mat * n_opt];  n_opt <= 255.
+ *   choice     int [n_mat], the option of each matrix;  total_err (optional) the plan's summed error.
+ * QLR_ERR_SHAPE when the budget is below the cheapest plan, or when (budget_bits / unit_bits + 1) *
+ * n_mat exceeds 2^30 (use a larger unit).
+ */
+QLR_API int qlr_lqlora_allocate(const double* err, const int64_t* cost_bits, int n_mat, int n_opt, int64_t budget_bits,
+                                int64_t unit_bits, int* choice, double* total_err);
+
+/*
  * QA-LoRA merge (QA-LoRA abstract: after fine-tuning the adapter is integrated into the
  * quantised model without loss of accuracy).  With the pooled adapter, s (B A)[o, g] / L is
  * added to every weight of group g of row o, which is a shift of the zero point:

@@ -16,6 +16,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "nfk.cuh"
 #include "ptx.cuh"
 
 namespace qlr {
@@ -50,36 +51,11 @@ const Solver& solver() {
 }
 
 // ---- kernels -----------------------------------------------------------------------------------
-__device__ __forceinline__ float bf16_round(float x) {
-  return __uint_as_float((pack_bf16x2_rn(x, 0.f) & 0xFFFFu) << 16);
-}
-
-__device__ __forceinline__ uint32_t code_at(const uint8_t* codes, int bits, int64_t i) {
-  if (bits == 4) return (codes[i >> 1] >> ((i & 1) * 4)) & 0xFu;
-  if (bits == 2) return (codes[i >> 2] >> ((i & 3) * 2)) & 0x3u;
-  const uint32_t* w = reinterpret_cast<const uint32_t*>(codes) + 3 * (i >> 5);
-  const int t = static_cast<int>(i & 31);
-  return ((w[0] >> t) & 1u) | (((w[1] >> t) & 1u) << 1) | (((w[2] >> t) & 1u) << 2);
-}
-
-// R = W - dequant(Q): the weight the quantised layer actually uses, bf16(level * scale) (fp32 product)
-__global__ void residual_kernel(const float* __restrict__ W, int64_t n, const uint8_t* __restrict__ codes, int bits,
-                                int block_shift, int dq, const float* __restrict__ c1,
-                                const uint8_t* __restrict__ c1_fp8, const float* __restrict__ s2, Levels lv,
-                                float* __restrict__ R) {
+// R = W - dequant(Q): the weight the quantised layer actually uses
+__global__ void residual_kernel(const float* __restrict__ W, int64_t n, const nfk::View v, float* __restrict__ R) {
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t b = i >> block_shift;
-    float scale;
-    if (dq) {
-      const __half_raw hr = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(c1_fp8[b]), __NV_E4M3);
-      scale = __fmul_rn(__half2float(__half(hr)), s2[b >> 8]);
-    } else {
-      scale = c1[b];
-    }
-    const float deq = bf16_round(__fmul_rn(lv.v[code_at(codes, bits, i)], scale));
-    R[i] = __fsub_rn(W[i], deq);
-  }
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    R[i] = __fsub_rn(W[i], nfk::dequant_at(v, i));
 }
 
 // column-major copy (N x K, leading dimension N) of the row-major N x K matrix R
@@ -270,8 +246,6 @@ extern "C" int qlr_lqlora_init(const float* W, int64_t N, int64_t K, int bits, i
   float* work = reinterpret_cast<float*>(ws + L.work);
   const bool wide = K >= N;
   const int m = static_cast<int>(wide ? K : N), n = static_cast<int>(wide ? N : K);
-  const int shift = block == 128 ? 7 : 6;
-  const Levels lv = levels_for(bits);
 
   cusolverDnHandle_t h = nullptr;
   if (sv.create(&h) != CUSOLVER_STATUS_SUCCESS) return QLR_ERR_CUDA;
@@ -285,8 +259,7 @@ extern "C" int qlr_lqlora_init(const float* W, int64_t N, int64_t K, int bits, i
       }
     } else {
       count_launch();
-      residual_kernel<<<grid_of(N * K), 256, 0, st>>>(W, N * K, out->codes, bits, shift, dq_block ? 1 : 0, out->c1,
-                                                      out->c1_fp8, out->s2, lv, R);
+      residual_kernel<<<grid_of(N * K), 256, 0, st>>>(W, N * K, nfk::view_of(out), R);
     }
     // column-major operand with at least as many rows as columns
     float* Acm = R;  // row-major N x K read as column-major K x N (ld K)

@@ -30,7 +30,7 @@ EXPORTED = (
     "qlr_backward_lora_workspace_bytes", "qlr_backward_lora", "qlr_backward_dx_workspace_bytes",
     "qlr_backward_dx", "qlr_swiglu_forward", "qlr_swiglu_backward", "qlr_device_sm_count", "qlr_lora_down",
     "qlr_forward_base", "qlr_launch_count", "qlr_backward_lora_noalloc", "qlr_lqlora_init_workspace_bytes",
-    "qlr_lqlora_init",
+    "qlr_lqlora_init", "qlr_nf_quant_error_workspace_bytes", "qlr_nf_quant_error", "qlr_lqlora_allocate",
 )
 
 
@@ -84,6 +84,9 @@ def lib() -> ctypes.CDLL:
         "qlr_backward_lora_noalloc": (I, [QP, P, P, P, P, I64, I, F, I, P, P, P, P, P]),
         "qlr_lqlora_init_workspace_bytes": (SZ, [I64, I64, I]),
         "qlr_lqlora_init": (I, [P, I64, I64, I, I, I, I, F, I, QP, P, P, P, SZ, P, P]),
+        "qlr_nf_quant_error_workspace_bytes": (SZ, [I64, I64, I, I, I]),
+        "qlr_nf_quant_error": (I, [P, I64, I64, I, I, I, P, P, SZ, P, P]),
+        "qlr_lqlora_allocate": (I, [P, P, I, I, I64, I64, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -230,6 +233,33 @@ def lqlora_init(W: torch.Tensor, bits: int, block: int, dq_block: int, r: int, s
     _check(lib().qlr_lqlora_init(_ptr(W), N, K, bits, block, dq_block, r, float(s), iters, q.ref(), _ptr(A), _ptr(B),
                                  _ptr(ws), nbytes, _ptr(status), _stream(stream)), "qlr_lqlora_init")
     return q, A, B
+
+
+def nf_quant_error(W: torch.Tensor, bits: int, block: int, dq_block: int, out: Optional[torch.Tensor] = None,
+                   ws: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Squared reconstruction error of NF-k quantising W, as a one-element float64 device tensor."""
+    N, K = W.shape
+    nbytes = int(lib().qlr_nf_quant_error_workspace_bytes(N, K, bits, block, dq_block))
+    if ws is None or ws.numel() < nbytes:
+        ws = _empty(max(nbytes, 256), W.device)
+    if out is None:
+        out = torch.empty(1, dtype=torch.float64, device=W.device)
+    _check(lib().qlr_nf_quant_error(_ptr(W), N, K, bits, block, dq_block, _ptr(out), _ptr(ws), nbytes, None,
+                                    _stream(stream)), "qlr_nf_quant_error")
+    return out
+
+
+def lqlora_allocate(err, cost_bits, budget_bits: int, unit_bits: int):
+    """Budgeted option per matrix (host arrays [n_mat, n_opt]): returns (choices, total error)."""
+    import numpy as np
+    e = np.ascontiguousarray(err, dtype=np.float64)
+    c = np.ascontiguousarray(cost_bits, dtype=np.int64)
+    n_mat, n_opt = e.shape
+    choice = np.zeros(n_mat, dtype=np.int32)
+    total = ctypes.c_double(0.0)
+    _check(lib().qlr_lqlora_allocate(e.ctypes.data, c.ctypes.data, n_mat, n_opt, int(budget_bits), int(unit_bits),
+                                     choice.ctypes.data, ctypes.byref(total)), "qlr_lqlora_allocate")
+    return [int(x) for x in choice], float(total.value)
 
 
 class Workspace:
