@@ -508,10 +508,64 @@ def run_lqlora_init(args, dev, iters: int = 2):
                                      "r": spec.r, "iters": iters}
         del W
     stack_s = sum(seen[(s_.N, s_.K)] for s_ in wl.linears) / 1e3
+    alloc = run_lqlora_allocation(args, dev, wl)
     return {"metric": "LQ-LoRA initialisation time per matrix (ms), whole call", "per_shape": out,
-            "stack_projection_s": stack_s, "stack_matrices": len(wl.linears),
+            "stack_projection_s": stack_s, "stack_matrices": len(wl.linears), "allocation": alloc,
             "note": "truncated SVD: single-precision cuSOLVER gesvd on the full matrix; residual, rank-r "
                     "subtraction, factor split and quantisation in this library's kernels"}
+
+
+def run_lqlora_allocation(args, dev, wl):
+    """Budgeted (bits, block) plan for the 224 matrices of the 7B stack: the quantisation error of all six
+    options of every matrix on the GPU, then the library's exact allocation at the storage budget of the
+    stack's seeded per-matrix draw; reports both plans' total errors."""
+    import numpy as np
+    import torch
+    from quantized_base_lora_nf4_b200 import qlr
+
+    L = qlr.lib()
+    options = [(k, b) for k in (2, 3, 4) for b in (64, 128)]
+    m = len(wl.linears)
+    err = np.zeros((m, len(options)))
+    cost = np.zeros((m, len(options)), dtype=np.int64)
+    drawn = []
+    out = torch.empty((m, len(options)), dtype=torch.float64, device=dev)
+    ws = None
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    gpu_ms = 0.0
+    for i, spec in enumerate(wl.linears):
+        g = torch.Generator(device=dev)
+        g.manual_seed(args.seed * 100003 + i)
+        W = torch.randn((spec.N, spec.K), generator=g, device=dev, dtype=torch.float32) * spec.sigma_w
+        nbytes = max(int(L.qlr_nf_quant_error_workspace_bytes(spec.N, spec.K, k, b, 256)) for k, b in options)
+        if ws is None or ws.numel() < nbytes:
+            ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+        e0.record()
+        for o, (k, b) in enumerate(options):
+            qlr.nf_quant_error(W, k, b, 256, out=out[i, o:o + 1], ws=ws)
+        e1.record()
+        torch.cuda.synchronize()
+        gpu_ms += e0.elapsed_time(e1)
+        for o, (k, b) in enumerate(options):
+            cost[i, o] = 8 * sum(qlr.part_bytes(qlr.FMT_NFK, spec.N, spec.K, k, b, 256, 32, part)
+                                 for part in (qlr.PART_CODES, qlr.PART_C1_FP8, qlr.PART_S2))
+        drawn.append(options.index((spec.bits, spec.block)))
+        del W
+    err[:] = out.cpu().numpy()
+    budget = int(sum(cost[i, o] for i, o in enumerate(drawn)))
+    t0 = time.perf_counter()
+    choice, total = qlr.lqlora_allocate(err, cost, budget, 1 << 20)
+    host_ms = 1e3 * (time.perf_counter() - t0)
+    params = sum(s_.N * s_.K for s_ in wl.linears)
+    hist = {}
+    for o in choice:
+        key = f"nf{options[o][0]}_b{options[o][1]}"
+        hist[key] = hist.get(key, 0) + 1
+    return {"options": [f"nf{k}_b{b}" for k, b in options], "error_pass_ms": gpu_ms, "allocate_ms": host_ms,
+            "budget_bits_per_param": budget / params,
+            "plan_bits_per_param": sum(cost[i, o] for i, o in enumerate(choice)) / params,
+            "plan_total_sq_error": total, "seeded_draw_total_sq_error": float(sum(err[i, o] for i, o in enumerate(drawn))),
+            "plan_histogram": hist, "unit_bits": 1 << 20}
 
 
 # ------------------------------------------------------------------------------------------ decode shape
