@@ -1,6 +1,7 @@
 // Shared declarations of the library's kernels and host helpers.
 #pragma once
 #include <cstdint>
+#include <mutex>
 #include <cuda_runtime.h>
 
 #include "../../include/qlr.h"
@@ -55,6 +56,23 @@ cudaError_t launch_decode(const qlr_qweight* w, const uint16_t* X, int64_t M, co
 
 // Counts kernel launches issued by this library (reported by qlr_launch_count).
 void count_launch(int n = 1);
+
+// Raises a kernel's dynamic shared-memory limit once per device (the attribute is set for the
+// device that is current when it is set, so a process that drives several GPUs needs it on each).
+template <typename Kern>
+cudaError_t ensure_max_dynamic_smem(Kern kern, int bytes) {
+  static std::mutex mu;
+  static int done_bytes[64] = {0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  std::lock_guard<std::mutex> lock(mu);
+  if (done_bytes[dev] >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done_bytes[dev] = bytes;
+  return e;
+}
 
 // Launches a hot-path kernel with programmatic stream serialisation, so that its launch and set-up
 // overlap the tail of the previous kernel on the stream; the kernel itself calls pdl_wait before it

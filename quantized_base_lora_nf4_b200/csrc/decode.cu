@@ -393,11 +393,7 @@ template <int NT>
 cudaError_t launch_decode_variant(const DecodeParams& p, int grid, const CUtensorMap& tc_lo, const CUtensorMap& tc_hi,
                                   const CUtensorMap& tx, cudaStream_t st) {
   const size_t smem = decode_smem_bytes(NT);
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [&] {
-    attr_err = cudaFuncSetAttribute(decode_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-  });
+  const cudaError_t attr_err = ensure_max_dynamic_smem(decode_kernel<NT>, 227 * 1024);
   if (attr_err != cudaSuccess) return attr_err;
   return launch_pdl(decode_kernel<NT>, dim3(grid), dim3(kThreads), smem, st, p, tc_lo, tc_hi, tx);
 }

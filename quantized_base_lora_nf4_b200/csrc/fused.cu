@@ -388,11 +388,7 @@ template <int A_SRC, int BN, bool PAIR>
 cudaError_t launch_fused_variant(const GemmParams& p, const GemmMaps& maps, cudaStream_t st) {
   using C = FCfg<BN>;
   auto kern = fused_kernel<A_SRC, BN, PAIR>;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [&] {
-    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem + 1024);
-  });
+  const cudaError_t attr_err = ensure_max_dynamic_smem(kern, C::kSmem + 1024);
   if (attr_err != cudaSuccess) return attr_err;
   const int tiles = p.m_tiles * p.n_tiles;
   const int grid = tiles < device_sm_count() ? tiles : device_sm_count();

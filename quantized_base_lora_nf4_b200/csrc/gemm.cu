@@ -282,11 +282,7 @@ template <int A_SRC, int B_SRC, int BN>
 cudaError_t launch_adapter_variant(const AdapterParams& p, const GemmMaps& maps, cudaStream_t st) {
   using C = ACfg<BN>;
   auto kern = adapter_kernel<A_SRC, B_SRC, BN>;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [&] {
-    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem + 1024);
-  });
+  const cudaError_t attr_err = ensure_max_dynamic_smem(kern, C::kSmem + 1024);
   if (attr_err != cudaSuccess) return attr_err;
   const int items = p.m_tiles * p.splits;
   const int grid = items < device_sm_count() ? items : device_sm_count();

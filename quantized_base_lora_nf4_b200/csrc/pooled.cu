@@ -152,7 +152,7 @@ size_t dA_smem(int64_t K, int L, int r) { return (static_cast<size_t>(K / L) + r
 template <typename Kern>
 cudaError_t allow_smem(Kern kern, size_t smem) {
   if (smem <= 48 * 1024) return cudaSuccess;
-  return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  return ensure_max_dynamic_smem(kern, static_cast<int>(smem));
 }
 
 template <int L>
