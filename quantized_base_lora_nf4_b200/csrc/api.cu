@@ -6,7 +6,9 @@
 #include <algorithm>
 #include <atomic>
 #include <cstring>
+#include <map>
 #include <mutex>
+#include <utility>
 
 #include "common.cuh"
 #include "gemm.cuh"
@@ -39,6 +41,20 @@ Levels levels_for(int bits) {
   for (int i = 0; i < 16; ++i) l.v[i] = 0.f;
   if (bits >= 2 && bits <= 4) nf_levels_f32(bits, l.v);
   return l;
+}
+
+cudaError_t ensure_max_dynamic_smem_fn(const void* kern, int bytes) {
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, int> done;  // (kernel, device) -> limit set
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = done.find({kern, dev});
+  if (it != done.end() && it->second >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done[{kern, dev}] = bytes;
+  return e;
 }
 
 int device_sm_count() {

@@ -1,7 +1,6 @@
 // Shared declarations of the library's kernels and host helpers.
 #pragma once
 #include <cstdint>
-#include <mutex>
 #include <cuda_runtime.h>
 
 #include "../../include/qlr.h"
@@ -57,21 +56,13 @@ cudaError_t launch_decode(const qlr_qweight* w, const uint16_t* X, int64_t M, co
 // Counts kernel launches issued by this library (reported by qlr_launch_count).
 void count_launch(int n = 1);
 
-// Raises a kernel's dynamic shared-memory limit once per device (the attribute is set for the
-// device that is current when it is set, so a process that drives several GPUs needs it on each).
+// Raises a kernel's dynamic shared-memory limit to `bytes` on the current device, once per (kernel,
+// device): the attribute belongs to the device that is current when it is set, so a process that
+// drives several GPUs needs it on each.
+cudaError_t ensure_max_dynamic_smem_fn(const void* kern, int bytes);
 template <typename Kern>
 cudaError_t ensure_max_dynamic_smem(Kern kern, int bytes) {
-  static std::mutex mu;
-  static int done_bytes[64] = {0};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64) return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  std::lock_guard<std::mutex> lock(mu);
-  if (done_bytes[dev] >= bytes) return cudaSuccess;
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e == cudaSuccess) done_bytes[dev] = bytes;
-  return e;
+  return ensure_max_dynamic_smem_fn(reinterpret_cast<const void*>(kern), bytes);
 }
 
 // Launches a hot-path kernel with programmatic stream serialisation, so that its launch and set-up

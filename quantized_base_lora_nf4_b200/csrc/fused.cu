@@ -211,6 +211,12 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
     if (lane == 0) {
       uint32_t j = 0, jb = 0;  // A-ring steps, B-ring stages
       int it = 0;
+      // descriptors of ring slot 0; a slot or a 16-wide reduction slice is a fixed address offset, which
+      // adds to the descriptor's address field (addr >> 4) without carrying out of it
+      const uint64_t a_desc0 = MN ? smem_desc(smem_u32(ring_a), 8192, 1024, kSw128)
+                                  : smem_desc(smem_u32(ring_a), 16, 1024, kSw128);
+      const uint64_t b_desc0 = smem_desc(smem_u32(ring_b), 16, 1024, kSw128);
+      constexpr uint32_t kAk = MN ? (2048 >> 4) : (32 >> 4), kBk = 32 >> 4;
       bool ok = true;
       for (int tile = blockIdx.x; tile < n_tiles_total && ok; tile += gridDim.x, ++it) {
         const int acc = PAIR ? 0 : (it & 1);
@@ -220,7 +226,7 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
         for (int ks = 0; ks < nsteps && ok; ++ks, ++j) {
           const int sa = j % NSA;
           if (!mbar_wait(&bars->a_full[sa], (j / NSA) & 1, abort_flag)) { ok = false; break; }
-          const uint32_t a_addr = smem_u32(ring_a + sa * C::kA);
+          const uint64_t ad0 = a_desc0 + static_cast<uint32_t>((sa * C::kA) >> 4);
           int nsub = 4;
           if (ks >= nmain) {
             const int rem = p.r_tail - (ks - nmain) * 64;
@@ -230,13 +236,15 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
             const int sb = jb % NSB;
             if (!mbar_wait(&bars->b_full[sb], (jb / NSB) & 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t b_addr = smem_u32(ring_b + sb * C::kB);
+            const uint64_t bd0 = b_desc0 + static_cast<uint32_t>((sb * C::kB) >> 4);
             const uint32_t d_tmem = tmem_base + (PAIR ? h : acc) * BN;
-            for (int kk = 0; kk < nsub; ++kk) {
-              const uint64_t ad = MN ? smem_desc(a_addr + kk * 2048, 8192, 1024, kSw128)
-                                     : smem_desc(a_addr + kk * 32, 16, 1024, kSw128);
-              const uint64_t bd = smem_desc(b_addr + kk * 32, 16, 1024, kSw128);
-              umma_bf16_ss(d_tmem, ad, bd, kIdesc, (ks > 0 || kk > 0) ? 1u : 0u);
+            if (nsub == 4) {
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                umma_bf16_ss(d_tmem, ad0 + kk * kAk, bd0 + kk * kBk, kIdesc, (ks > 0 || kk > 0) ? 1u : 0u);
+            } else {
+              for (int kk = 0; kk < nsub; ++kk)
+                umma_bf16_ss(d_tmem, ad0 + kk * kAk, bd0 + kk * kBk, kIdesc, (ks > 0 || kk > 0) ? 1u : 0u);
             }
             umma_commit(&bars->b_empty[sb]);
           }
