@@ -14,8 +14,9 @@
 //   A ring     (3-4 x 16 KB) written by the dequantiser warps in the canonical 128-byte-swizzled
 //                            UMMA layout (they also copy the tail's weight-side rows);
 //   B ring     (4-8 stages)  activation tiles by TMA.
-// Warp roles: 0 activation producer, 1 TMEM allocator + MMA issuer, 2..5 epilogue, 6..13 two groups
-// of dequantisers taking alternate reduction steps, 14 codes producer.  Two TMEM accumulators
+// Warp roles: 1 TMEM allocator + MMA issuer, 9 activation producer, 13 codes producer, 2..5 epilogue,
+// 0, 6, 7, 8, 10, 11, 12, 14 two groups of dequantisers taking alternate reduction steps (warps 1, 5, 9
+// and 13 share a scheduler, which keeps the dequantisers' work off the issuer's).  Two TMEM accumulators
 // (2 x BN fp32 columns) overlap each tile's epilogue with the next tile's main loop.  Every wait is
 // bounded; a wait that runs out aborts the CTA and reports QLR_ERR_TIMEOUT.
 #include <mutex>
@@ -27,6 +28,25 @@ namespace qlr {
 namespace {
 
 constexpr int kThreadsFused = 480;
+// Warp roles.  A warp runs on scheduler (warp % 4); the single-thread MMA issuer (warp 1) shares its
+// scheduler only with light roles (the two TMA producers and one epilogue warp), so the dequantisers'
+// integer work does not delay the issue of the next MMAs.  Epilogue warps 2..5 read TMEM lane quadrants
+// 2, 3, 0, 1 (a warp may only read the quadrant warp % 4).
+constexpr int kActWarp = 9, kCodesWarp = 13, kIssuerWarp = 1;
+// dequantiser slot of each warp (slot / 4 = group, slot % 4 = 32-row block), -1 for other roles
+__device__ __forceinline__ int dq_slot(int warp) {
+  switch (warp) {
+    case 0: return 0;
+    case 6: return 1;
+    case 7: return 2;
+    case 8: return 3;
+    case 10: return 4;
+    case 11: return 5;
+    case 12: return 6;
+    case 14: return 7;
+    default: return -1;
+  }
+}
 
 template <int BN>
 struct FCfg {
@@ -132,16 +152,16 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
     bars->abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 0 && lane == 0) {
+  if (warp == kActWarp && lane == 0) {
     tma_prefetch_desc(&maps.b);
     tma_prefetch_desc(&maps.b_tail);
   }
-  if (warp == 14 && lane == 0) tma_prefetch_desc(&maps.codes);
+  if (warp == kCodesWarp && lane == 0) tma_prefetch_desc(&maps.codes);
   // everything above touches only shared memory and kernel parameters; from here on the previous
   // kernel's results are needed (and its TMEM must be free)
   pdl_launch_dependents();
   pdl_wait();
-  if (warp == 1) {
+  if (warp == kIssuerWarp) {
     tmem_alloc(&bars->tmem_base, C::kTmemCols);
     tmem_relinquish();
   }
@@ -155,7 +175,7 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
   auto tile_m0 = [&](int tile) { return (tile / p.n_tiles) * 128; };
   auto tile_n0 = [&](int tile) { return (tile % p.n_tiles) * TOK; };
 
-  if (warp == 0) {
+  if (warp == kActWarp) {
     // ------------------------------------------------------------------ activation producer
     if (lane == 0) {
       uint32_t j = 0;
@@ -181,7 +201,7 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
         mbar_wait(&bars->b_full[q % NSB], (q / NSB) & 1, &never);
       }
     }
-  } else if (warp == 14) {
+  } else if (warp == kCodesWarp) {
     // ------------------------------------------------------------------ codes producer
     if (lane == 0) {
       const int lg = p.code_slots_log2, ncs = 1 << lg, kb = p.code_bits;
@@ -206,7 +226,7 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
         mbar_wait(&bars->c_full[q & mask], (q >> lg) & 1, &never);
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == kIssuerWarp) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       uint32_t j = 0, jb = 0;  // A-ring steps, B-ring stages
@@ -258,7 +278,7 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
       volatile int never = 0;
       mbar_wait(&bars->drain, 0, &never);
     }
-  } else if (warp < 6) {
+  } else if (warp >= 2 && warp <= 5) {
     // ------------------------------------------------------------------ epilogue
     const int q = warp & 3;
     uint16_t* stg = reinterpret_cast<uint16_t*>(staging) + q * 32 * 32;
@@ -283,9 +303,9 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
     }
   } else {
     // ------------------------------------------------------------------ dequantisers (warps 6..13)
-    const int dt = threadIdx.x - 6 * 32;
-    const int grp = dt >> 7;
-    const int t = dt & 127;
+    const int slot = dq_slot(warp);
+    const int grp = slot >> 2;
+    const int t = (slot & 3) * 32 + lane;
     auto run_of = [&](int m0, int k0, int64_t& row, int64_t& col, bool& valid) {
       if (!MN) {  // row t of the W tile: W[m0 + t, k0 .. k0 + 63] -> K-major row t
         row = m0 + t;
@@ -384,7 +404,7 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kIssuerWarp) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem_base, C::kTmemCols);
