@@ -148,8 +148,8 @@ QLR_API int qlr_quantize_int4_group(const float* W, int64_t N, int64_t K, int gr
 QLR_API int qlr_dequant(const qlr_qweight* w, uint16_t* W_out, int32_t* status, void* stream);
 
 /*
- * LQ-LoRA initialisation (LQ-LoRA abstract: an iterative algorithm decomposes each pretrained matrix
- * into a high-precision low-rank component and a memory-efficient quantized component; the quantized
+ * LQ-LoRA initialisation (LQ-LoRA abstract: an iterative method splits each pretrained matrix into a
+ * low-rank part kept in high precision plus a quantised part that is cheap to store; the quantised
  * part stays frozen and the low-rank part is the adapter).  Read as the alternation
  *   Q_0 = 0;  for t = 1..iters:  L_t = rank-r truncated SVD of (W - dequant(Q_{t-1})),
  *                                Q_t = NF-k quantisation (bits, block, dq_block) of (W - L_t)
@@ -187,9 +187,8 @@ QLR_API int qlr_nf_quant_error(const float* W, int64_t N, int64_t K, int bits, i
                                void* stream);
 
 /*
- * LQ-LoRA's budgeted allocation (LQ-LoRA abstract: an integer linear programming formulation that
- * configures the quantisation parameters, e.g. bit width and block size, of each matrix for an overall
- * memory budget).  Read as a multiple-choice knapsack: matrix i takes one option o out of n_opt with
+ * LQ-LoRA's budgeted allocation (LQ-LoRA abstract: an integer linear programme picks each matrix's
+ * bit width and block size so that the whole model meets a memory budget).  Read as a multiple-choice knapsack: matrix i takes one option o out of n_opt with
  * error err[i * n_opt + o] and storage cost_bits[i * n_opt + o]; the summed error is minimised with the
  * summed storage within budget_bits.  Exact dynamic programming over the budget in whole units of
  * unit_bits (costs rounded up, so the plan never exceeds the budget); the plan is read back last matrix
@@ -203,8 +202,8 @@ QLR_API int qlr_lqlora_allocate(const double* err, const int64_t* cost_bits, int
                                 int64_t unit_bits, int* choice, double* total_err);
 
 /*
- * QA-LoRA merge (QA-LoRA abstract: after fine-tuning the adapter is integrated into the
- * quantised model without loss of accuracy).  With the pooled adapter, s (B A)[o, g] / L is
+ * QA-LoRA merge (QA-LoRA abstract: once fine-tuned, the adapter folds into the quantised weight
+ * and the model loses no accuracy).  With the pooled adapter, s (B A)[o, g] / L is
  * added to every weight of group g of row o, which is a shift of the zero point:
  *   zero'[o, g] = fp16( zero - s * (B A)[o, g] / (group * scale[o, g]) ),  in fp64;
  * groups with scale == 0 keep their zero.  w->zero is rewritten in place.

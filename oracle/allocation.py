@@ -1,9 +1,8 @@
 """LQ-LoRA's per-matrix choice of quantisation parameters under a memory budget (oracle; test
 infrastructure).
 
-LQ-LoRA (abstract): "an integer linear programming formulation of the quantization component which
-enables dynamic configuration of quantization parameters (e.g., bit-width, block size) for each
-matrix given an overall target memory budget".  Read as a multiple-choice knapsack: matrix i takes
+LQ-LoRA (abstract): an integer linear programme picks each matrix's quantisation parameters (bit
+width, block size) so that the whole model meets a memory budget.  Read as a multiple-choice knapsack: matrix i takes
 exactly one option o (a bit width and block size) with reconstruction error err[i][o] (squared
 Frobenius norm of W_i - dequant(Q_o(W_i))) and storage cost[i][o] (bits of its codes and constants);
 minimise the summed error with the summed cost within the budget.

@@ -1,8 +1,8 @@
 """LQ-LoRA initialisation (oracle; test infrastructure).
 
-LQ-LoRA (abstract): "an iterative algorithm to decompose each pretrained matrix into a high-precision
-low-rank component and a memory-efficient quantized component"; during finetuning the quantized
-component stays fixed and only the low-rank component (the adapter) is trained.  The abstract gives
+LQ-LoRA (abstract): an iterative method splits each pretrained matrix into a low-rank part kept in
+high precision plus a quantised part that is cheap to store; during finetuning the quantised part
+stays fixed and only the low-rank component (the adapter) is trained.  The abstract gives
 no further steps; the reading used here is the plain alternation between the two components:
 
     Q_0 = 0

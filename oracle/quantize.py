@@ -29,7 +29,7 @@ Readings where the pages leave a step open (each is listed in the design notes):
     bf16_rn(level[code] * c1).
 
 QA-LoRA (abstract: group-wise INT4 quantisation, an adapter with fewer degrees of
-freedom, and a merge "without loss of accuracy") is read as:
+freedom, and a merge into the quantised weight that costs no accuracy) is read as:
   * per (row o, group g of L consecutive inputs): lo = min(0, min w), hi = max(0, max w),
     scale = fp16_rn(fp32(fp32(hi - lo) / 15)), z = clamp(rne(fp32(-lo / scale)), 0, 15)
     stored as fp16 (an integer, so a zero is +0), code = clamp(rne(fp32(fp32(w / scale) + z)), 0, 15); a group whose

@@ -1,7 +1,6 @@
-// LQ-LoRA's budgeted choice of quantisation parameters per matrix (LQ-LoRA abstract: "an integer
-// linear programming formulation of the quantization component which enables dynamic configuration of
-// quantization parameters (e.g., bit-width, block size) for each matrix given an overall target memory
-// budget").  A multiple-choice knapsack: each matrix takes one option, the summed reconstruction error
+// LQ-LoRA's budgeted choice of quantisation parameters per matrix (LQ-LoRA abstract: an integer linear
+// programme picks each matrix's bit width and block size so that the whole model meets a memory
+// budget).  A multiple-choice knapsack: each matrix takes one option, the summed reconstruction error
 // is minimised and the summed storage stays within the budget.  Host code; exact dynamic programming
 // over the budget in whole units (costs rounded up, so a plan never exceeds the budget).
 #include <cstdint>

@@ -1,6 +1,6 @@
-// LQ-LoRA initialisation (LQ-LoRA abstract: each pretrained matrix is decomposed "into a high-precision
-// low-rank component and a memory-efficient quantized component" by an iterative algorithm; the
-// quantized part stays frozen and the low-rank part is the trainable adapter).  Read as the
+// LQ-LoRA initialisation (LQ-LoRA abstract: an iterative method splits each pretrained matrix into a
+// low-rank part kept in high precision plus a quantised part that is cheap to store; the
+// quantised part stays frozen and the low-rank part is the trainable adapter).  Read as the
 // alternation
 //     Q_0 = 0;  for t = 1..T:  L_t = rank-r truncated SVD of (W - dequant(Q_{t-1})),
 //                              Q_t = NF-k quantisation of (W - L_t)

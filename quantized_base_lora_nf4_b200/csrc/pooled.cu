@@ -1,5 +1,5 @@
-// The pooled adapter of QA-LoRA (abstract: the adapter's input is reduced group-wise, "decreasing the
-// degrees of freedom of adaptation", so that the product B A can later be merged into the group
+// The pooled adapter of QA-LoRA (abstract: the adapter's input is reduced group-wise, which gives the
+// adaptation fewer degrees of freedom, so that the product B A can later be merged into the group
 // zero points).  With P(X)[m, g] = mean of X[m, gL .. gL + L - 1] (the group of L inputs that shares a
 // scale and zero point), the two adapter products that involve P(X) are small dense problems over
 // the pooled input instead of full-K GEMMs:

@@ -220,7 +220,7 @@ def test_int4_group_brute_force_tiny():
 
 
 def test_qalora_merge_is_lossless_in_fp64():
-    """Merged and unmerged outputs agree (fp64, unrounded z'): the abstract's "without loss of accuracy"."""
+    """Merged and unmerged outputs agree (fp64, unrounded z'): QA-LoRA's abstract says the merge loses no accuracy."""
     N, K, L, r, M, s = 64, 256, 32, 4, 8, 1.5
     W = random_matrix(11, 0, "W", (N, K), 0.02)
     A = random_matrix(11, 1, "A", (r, K // L), 0.01, bf16=True)
