@@ -14,11 +14,10 @@
 //   A ring     (3-4 x 16 KB) written by the dequantiser warps in the canonical 128-byte-swizzled
 //                            UMMA layout (they also copy the tail's weight-side rows);
 //   B ring     (4-8 stages)  activation tiles by TMA.
-// Warp roles: 1 TMEM allocator + MMA issuer, 9 activation producer, 13 codes producer, 2..5 epilogue,
-// 0, 6, 7, 8, 10, 11, 12, 14 two groups of dequantisers taking alternate reduction steps (warps 1, 5, 9
-// and 13 share a scheduler, which keeps the dequantisers' work off the issuer's).  Two TMEM accumulators
-// (2 x BN fp32 columns) overlap each tile's epilogue with the next tile's main loop.  Every wait is
-// bounded; a wait that runs out aborts the CTA and reports QLR_ERR_TIMEOUT.
+// Warp roles (Roles below): 1 TMEM allocator + MMA issuer, 2..5 epilogue, one activation and one codes
+// producer, and eight warps in two groups of dequantisers taking alternate reduction steps.  Two TMEM
+// accumulators (2 x BN fp32 columns) overlap each tile's epilogue with the next tile's main loop.
+// Every wait is bounded; a wait that runs out aborts the CTA and reports QLR_ERR_TIMEOUT.
 #include <mutex>
 
 #include "engine.cuh"
@@ -28,25 +27,33 @@ namespace qlr {
 namespace {
 
 constexpr int kThreadsFused = 480;
-// Warp roles.  A warp runs on scheduler (warp % 4); the single-thread MMA issuer (warp 1) shares its
-// scheduler only with light roles (the two TMA producers and one epilogue warp), so the dequantisers'
-// integer work does not delay the issue of the next MMAs.  Epilogue warps 2..5 read TMEM lane quadrants
-// 2, 3, 0, 1 (a warp may only read the quadrant warp % 4).
-constexpr int kActWarp = 9, kCodesWarp = 13, kIssuerWarp = 1;
-// dequantiser slot of each warp (slot / 4 = group, slot % 4 = 32-row block), -1 for other roles
-__device__ __forceinline__ int dq_slot(int warp) {
-  switch (warp) {
-    case 0: return 0;
-    case 6: return 1;
-    case 7: return 2;
-    case 8: return 3;
-    case 10: return 4;
-    case 11: return 5;
-    case 12: return 6;
-    case 14: return 7;
-    default: return -1;
+// Warp roles.  A warp runs on scheduler (warp % 4).  Warp 1 allocates TMEM and issues the MMAs from
+// one thread; epilogue warps 2..5 read TMEM lane quadrants 2, 3, 0, 1 (a warp may only read the
+// quadrant warp % 4).  With 2 x BN-token tiles (MMA-heavy: each dequantised stage feeds two MMA
+// groups) the issuer's scheduler holds only light roles, the two TMA producers and one epilogue warp,
+// so the dequantisers' integer work does not delay the next MMAs.  With BN-token tiles the
+// dequantisation per MMA doubles and the eight dequantiser warps are spread two per scheduler instead.
+constexpr int kIssuerWarp = 1;
+template <bool PAIR>
+struct Roles {
+  static constexpr int kActWarp = PAIR ? 9 : 0;
+  static constexpr int kCodesWarp = PAIR ? 13 : 14;
+  // dequantiser slot of a warp (slot / 4 = group, slot % 4 = 32-row block), -1 for other roles
+  __device__ __forceinline__ static int dq_slot(int warp) {
+    if (!PAIR) return warp >= 6 && warp <= 13 ? warp - 6 : -1;
+    switch (warp) {
+      case 0: return 0;
+      case 6: return 1;
+      case 7: return 2;
+      case 8: return 3;
+      case 10: return 4;
+      case 11: return 5;
+      case 12: return 6;
+      case 14: return 7;
+      default: return -1;
+    }
   }
-}
+};
 
 template <int BN>
 struct FCfg {
@@ -152,6 +159,7 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
     bars->abort_flag = 0;
     fence_barrier_init();
   }
+  constexpr int kActWarp = Roles<PAIR>::kActWarp, kCodesWarp = Roles<PAIR>::kCodesWarp;
   if (warp == kActWarp && lane == 0) {
     tma_prefetch_desc(&maps.b);
     tma_prefetch_desc(&maps.b_tail);
@@ -303,7 +311,7 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
     }
   } else {
     // ------------------------------------------------------------------ dequantisers (warps 6..13)
-    const int slot = dq_slot(warp);
+    const int slot = Roles<PAIR>::dq_slot(warp);
     const int grp = slot >> 2;
     const int t = (slot & 3) * 32 + lane;
     auto run_of = [&](int m0, int k0, int64_t& row, int64_t& col, bool& valid) {
