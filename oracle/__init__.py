@@ -21,11 +21,16 @@ Modules
             INT4 group-wise quantiser (QA-LoRA) and the adapter merge
   layer     forward / backward of the quantised-base + LoRA linear, group pooling, SwiGLU
   storage   bits-per-parameter and byte accounting of the formats
+  lqlora    LQ-LoRA initialisation: alternating truncated SVD and NF-k quantisation
+  allocation LQ-LoRA's budgeted (bits, block) choice per matrix (multiple-choice knapsack)
 
 Parity-pinned: every function is checked in ``tests/test_oracle_*.py`` against
 closed forms, invariants, brute force on tiny inputs, library routines or the
-pages' printed figures.  Parity unpinned: the LQ-LoRA per-matrix choice of
-(bits, block) beyond its storage arithmetic (the pages give no worked example).
+pages' printed figures (the allocation against exhaustive search and the two
+closed-form ends of the budget; the initialisation against constructed SVDs, an
+exactly low-rank matrix and its zero-iteration case).  The pages print no worked
+example for the two LQ-LoRA parts, so what they pin is the reading of the
+abstract that these modules state, not numbers from the pages.
 """
 
-from . import numerics, codebook, quantize, layer, storage  # noqa: F401
+from . import numerics, codebook, quantize, layer, storage, lqlora, allocation  # noqa: F401
