@@ -1,7 +1,8 @@
 #!/usr/bin/env python
 """Throughput of the quantised-base + LoRA linear on B200: fwd+bwd tokens/s.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload qalora|tiny|mlp7b|lqlora|decode70b]
+    python bench.py [--gpus N] [--steps K] [--warmup W]
+                    [--workload qalora|tiny|mlp7b|lqlora|decode70b|lqlora_init]
                     [--impl ours|reference]
 
 One step = forward (adapter down-projection T = s P(X) A^T, fused dequant + tcgen05 base GEMM with the
