@@ -1,5 +1,6 @@
 """Pins of the LQ-LoRA initialisation oracle, each against something other than the oracle itself:
-an SVD built by hand, an exactly low-rank matrix, plain quantisation at T = 0, and the method's own
+an SVD built by hand, an exactly low-rank matrix, plain quantisation at T = 0, the optimality
+conditions of the second iteration's low-rank part, and the method's own
 purpose (a strong low-rank component is reconstructed better than by quantisation alone)."""
 import numpy as np
 
@@ -58,3 +59,23 @@ def test_strong_low_rank_component_beats_plain_quantisation():
     out = LQ.lqlora_init(W, 2, 64, 256, r, 0.25, 3)
     assert out["error"] < 0.5 * err_plain
     assert len(out["errors"]) == 3
+
+
+def test_second_iteration_fits_the_residual_of_the_first():
+    # L_2 must be the best rank-r approximation of W - dequant(Q_1), not of W: its residual E is
+    # orthogonal to its own column and row spaces (the first-order condition of a truncated SVD), and
+    # it fits that residual strictly better than L_1 does (Q_1 is far from zero at 2 bits)
+    rng = np.random.default_rng(4)
+    N, K, r = 64, 128, 4
+    W = (rng.standard_normal((N, r)) @ rng.standard_normal((r, K)) * 0.03
+         + 0.02 * rng.standard_normal((N, K))).astype(np.float32)
+    one = LQ.lqlora_init(W, 2, 64, 0, r, 1.0, 1)
+    two = LQ.lqlora_init(W, 2, 64, 0, r, 1.0, 2)
+    R1 = W.astype(np.float64) - Q.dequant_nfk(one["q"]).astype(np.float64)
+    L2 = two["lowrank"]
+    E = R1 - L2
+    col, _ = np.linalg.qr(L2 @ rng.standard_normal((K, r)))   # basis of L2's column space
+    row, _ = np.linalg.qr(L2.T @ rng.standard_normal((N, r)))  # basis of its row space
+    assert np.linalg.norm(col.T @ E) <= 1e-9 * np.linalg.norm(E)
+    assert np.linalg.norm(E @ row) <= 1e-9 * np.linalg.norm(E)
+    assert np.linalg.norm(E) < np.linalg.norm(R1 - one["lowrank"])

@@ -172,7 +172,17 @@ def test_nf_dequant_error_bound(bits, block, dq):
     halfgap = np.max(np.diff(lev)) / 2
     c1 = np.repeat(q["c1"], block)[: W.size].reshape(W.shape).astype(np.float64)
     sc = np.repeat(Q.nf_block_scales(q), block)[: W.size].reshape(W.shape).astype(np.float64)
-    bound = c1 * halfgap * (1 + 1e-6) + np.abs(c1 - sc) + np.abs(Wd) * 2.0 ** -8
+    # the block scale is c1 itself, or with double quantisation c1 to E4M3 precision: a relative
+    # error of at most 2^-4 in the normal range, half the subnormal spacing (2^-10 s2) below it
+    if dq:
+        s2 = np.repeat(np.repeat(q["s2"], dq)[: q["c1"].size], block)[: W.size].reshape(W.shape).astype(np.float64)
+        scale_err = c1 * 2.0 ** -4 * (1 + 1e-6) + s2 * 2.0 ** -10
+        assert np.all(np.abs(sc - c1) <= scale_err)
+    else:
+        scale_err = np.zeros_like(c1)
+        np.testing.assert_array_equal(sc, c1)
+    # |level| <= 1, so the scale's error moves a value by at most scale_err
+    bound = c1 * halfgap * (1 + 1e-6) + scale_err + np.abs(Wd) * 2.0 ** -8
     assert np.all(np.abs(W - Wd) <= bound)
     # dequant is level * scale rounded to bf16, level taken from the code
     ref = bf16_rn((nf_codebook_f32(bits)[q["codes"][: W.size]] * sc.reshape(-1).astype(np.float32)).astype(np.float32))
