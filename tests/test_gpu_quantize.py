@@ -91,6 +91,23 @@ def test_int4_group_quantize_bit_exact(cuda_lib, group, shape):
     np.testing.assert_array_equal(bf16_bits(host(Wd)), bf16_bits(Q.dequant_int4_group(ref)))
 
 
+def test_int4_group_quantize_ties_bit_exact(cuda_lib):
+    # values at exact k + 1/2 steps of a 0.0625 scale: both sides round code and zero point half to even
+    qlr = cuda_lib
+    s = 0.0625
+    W = random_matrix(24, 0, "W", (8, 128), 0.02)
+    W[0, :32] = 0.0
+    W[0, :5] = [15 * s, 0.5 * s, 1.5 * s, 2.5 * s, 3.5 * s]
+    W[1, :32] = 0.0
+    W[1, :4] = [-2.5 * s, 12.5 * s, 0.5 * s, 1.5 * s]
+    ref = Q.quantize_int4_group(W, 32)
+    q = qlr.quantize_int4_group(f32_dev(W), 32)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(host_bytes(q.codes), ref["packed"])
+    np.testing.assert_array_equal(q.scale.cpu().numpy().view(np.uint16), ref["scale"].view(np.uint16))
+    np.testing.assert_array_equal(q.zero.cpu().numpy().view(np.uint16), ref["zero"].view(np.uint16))
+
+
 def test_qalora_merge_bit_exact_and_lossless(cuda_lib):
     qlr = cuda_lib
     wl = workload("qalora")

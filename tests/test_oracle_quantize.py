@@ -249,3 +249,33 @@ def test_qalora_merge_is_lossless_in_fp64():
     zp16 = Q.qalora_merge(q, A, B, s)
     merged16 = f64(X) @ Q.dequant_int4_group(q, zero=zp16).astype(np.float64).T
     assert rel_fro(merged16, unmerged) < 1e-2
+
+
+def test_int4_exact_halves_round_to_even():
+    # scale 0.0625 exactly (span 0.9375 = 15 x 0.0625); values at k + 1/2 steps are fp32-exact ties
+    s = 0.0625
+    W = np.zeros((2, 32), np.float32)
+    W[0, :5] = [15 * s, 0.5 * s, 1.5 * s, 2.5 * s, 3.5 * s]           # lo = 0 -> z = 0
+    W[1, :4] = [-2.5 * s, 12.5 * s, 0.5 * s, 1.5 * s]                 # -lo / scale = 2.5 -> z = 2
+    q = Q.quantize_int4_group(W, 32)
+    assert np.all(q["scale"].astype(np.float32) == np.float32(s))
+    assert float(q["zero"][0, 0]) == 0.0 and float(q["zero"][1, 0]) == 2.0
+    codes = q["codes"].reshape(2, 32)
+    assert list(codes[0, :5]) == [15, 0, 2, 2, 4]                      # 0.5 -> 0, 1.5 -> 2, 2.5 -> 2, 3.5 -> 4
+    assert list(codes[1, :4]) == [0, 14, 2, 4]                         # -0.5 -> 0, 14.5 -> 14, 2.5 -> 2, 3.5 -> 4
+
+
+def test_qalora_merge_rounds_once_from_fp64():
+    # z' = 2 - a / 32 = 1 + 2^-11 + 2^-30: one rounding to fp16 goes up to 1 + 2^-10; rounding through
+    # fp32 first would land on the tie 1 + 2^-11 and then round to even, 1
+    a = 32.0 - 2.0 ** -6 - 2.0 ** -25
+    q = {"group": 32, "scale": np.array([[1.0]], np.float16), "zero": np.array([[2.0]], np.float16)}
+    zp = Q.qalora_merge(q, np.array([[a]]), np.array([[1.0]]), 1.0)
+    assert float(zp[0, 0]) == 1.0 + 2.0 ** -10
+
+
+def test_nf_partial_last_block_is_zero_padded():
+    W = random_matrix(12, 0, "W", (1, 192), 0.02)     # block 128: the second block has 64 weights
+    q = Q.quantize_nfk(W, 4, 128, 0)
+    assert q["c1"][1] == np.float32(np.abs(W[0, 128:]).max())
+    assert np.all(q["codes"][192:] == zero_index(4))   # the padding takes the zero level
