@@ -188,9 +188,9 @@ QLR_API int qlr_nf_quant_error(const float* W, int64_t N, int64_t K, int bits, i
 
 /*
  * LQ-LoRA's budgeted allocation (LQ-LoRA abstract: an integer linear programme picks each matrix's
- * bit width and block size so that the whole model meets a memory budget).  Read as a multiple-choice knapsack: matrix i takes one option o out of n_opt with
- * error err[i * n_opt + o] and storage cost_bits[i * n_opt + o]; the summed error is minimised with the
- * summed storage within budget_bits.  Exact dynamic programming over the budget in whole units of
+ * bit width and block size so that the whole model meets a memory budget).  Read as a multiple-choice
+ * knapsack: matrix i takes one option o out of n_opt with error err[i * n_opt + o] and storage
+ * cost_bits[i * n_opt + o]; the summed error is minimised with the summed storage within budget_bits.  Exact dynamic programming over the budget in whole units of
  * unit_bits (costs rounded up, so the plan never exceeds the budget); the plan is read back last matrix
  * first, each taking the lowest option index among its minima.  HOST memory, no GPU:
  *   err        double [n_mat * n_opt];  cost_bits  int64 [n_mat * n_opt];  n_opt <= 255.
@@ -220,7 +220,8 @@ QLR_API int qlr_qalora_merge(const qlr_qweight* w, const uint16_t* A, const uint
  * The dequantised weight never reaches global memory: the fused kernel streams the packed
  * codes into shared memory, dequantises them there and feeds tcgen05 tensor-core tiles;
  * the adapter term is added as r extra reduction columns of the same accumulator.
- * Token counts M <= 16 with 4-bit NF codes take a memory-streaming decode kernel instead.
+ * Token counts M <= 16 with 4-bit NF codes, double quantisation over 256 blocks and K a multiple of
+ * 256 take a memory-streaming decode kernel instead.
  *   X bf16 [M, K];  A bf16 [r, Ka];  B bf16 [N, r];  Y bf16 [M, N];  T_save bf16 [M, r].
  *   r in {8, 16, 32, 64};  K a multiple of 64 (and of w->block);  N a multiple of 8.
  */
@@ -251,8 +252,9 @@ QLR_API uint64_t qlr_launch_count(void);
  *   dB = dY^T T_save               [N, r]   fp32
  *   dA = dT^T P(X)                 [r, Ka]  fp32  (dT taken in bf16)
  * Each fp32 reduction over tokens is split across CTAs and summed in a fixed order, so the
- * results are deterministic.  With the pooled adapter (QA-LoRA), dA is formed directly from the group
- * means of X (one CTA per group, tokens summed in a fixed order) and needs no workspace.
+ * results are deterministic.  With the pooled adapter (QA-LoRA), dA is formed from the group means of
+ * X: one kernel writes, per slice of 16 tokens, the products of those means with the tokens' dT rows
+ * to the workspace, and a second sums the slices in a fixed order.
  */
 QLR_API size_t qlr_backward_lora_workspace_bytes(const qlr_qweight* w, int64_t M, int r, int pooled);
 QLR_API int qlr_backward_lora(const qlr_qweight* w, const uint16_t* X, const uint16_t* dY, const uint16_t* T_save,
