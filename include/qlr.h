@@ -190,9 +190,10 @@ QLR_API int qlr_nf_quant_error(const float* W, int64_t N, int64_t K, int bits, i
  * LQ-LoRA's budgeted allocation (LQ-LoRA abstract: an integer linear programme picks each matrix's
  * bit width and block size so that the whole model meets a memory budget).  Read as a multiple-choice
  * knapsack: matrix i takes one option o out of n_opt with error err[i * n_opt + o] and storage
- * cost_bits[i * n_opt + o]; the summed error is minimised with the summed storage within budget_bits.  Exact dynamic programming over the budget in whole units of
- * unit_bits (costs rounded up, so the plan never exceeds the budget); the plan is read back last matrix
- * first, each taking the lowest option index among its minima.  HOST memory, no GPU:
+ * cost_bits[i * n_opt + o]; the summed error is minimised with the summed storage within budget_bits.
+ * Exact dynamic programming over the budget in whole units of unit_bits (costs rounded up, so the plan
+ * never exceeds the budget); the plan is read back last matrix first, each taking the lowest option
+ * index among its minima.  HOST memory, no GPU:
  *   err        double [n_mat * n_opt];  cost_bits  int64 [n_mat * n_opt];  n_opt <= 255.
  *   choice     int [n_mat], the option of each matrix;  total_err (optional) the plan's summed error.
  * QLR_ERR_SHAPE when the budget is below the cheapest plan, or when (budget_bits / unit_bits + 1) *
