@@ -285,7 +285,16 @@ def run_ours(args, rank, world, dev):
         qlr.backward_lora(L.q, L.X, dY, L.T, L.B, s, pooled=pooled, dA=L.dA, dB=L.dB, dT=L.dT, ws=L.ws_b)
         qlr.backward_dx(L.q, dY, L.A, L.dT, pooled=pooled, dX=dX, accumulate=accumulate, ws=L.ws_x)
 
-    bucket = dp.GradBucket([g for L in layers for g in (L.dA, L.dB)]) if world > 1 else None
+    # data parallel: the adapter gradients are summed over ranks.  A stack's linears are exchanged in
+    # buckets whose all-reduce starts as soon as the last linear in them has finished its backward, so
+    # the exchange overlaps the backward of the linears after it; a single linear or an MLP block is
+    # one bucket, started when its backward ends
+    buckets = None
+    if world > 1:
+        if wl.kind == "stack":
+            buckets = dp.OverlappedBuckets([[L.dA, L.dB] for L in layers])
+        else:
+            buckets = dp.OverlappedBuckets([[g for L in layers for g in (L.dA, L.dB)]])
 
     def step(record=False):
         if wl.kind == "mlp":
@@ -302,12 +311,16 @@ def run_ours(args, rank, world, dev):
             lin_bwd(gate, dG, gate.dX)
             lin_bwd(up, dU, gate.dX, accumulate=True)
         else:  # one linear, or every linear of the stack in turn
-            for L in layers:
+            for i, L in enumerate(layers):
                 qlr.lora_down(L.q, L.X, L.A, L.spec.s, pooled=L.spec.pooled, T_save=L.T, ws=L.ws)
                 fwd_base(L, record)
                 lin_bwd(L, L.dY, L.dX)
-        if bucket is not None:
-            bucket.allreduce()  # data parallel: one SUM all-reduce of every adapter gradient
+                if buckets is not None and wl.kind == "stack":
+                    buckets.layer_done(i)
+        if buckets is not None:
+            if wl.kind != "stack":
+                buckets.layer_done(0)
+            buckets.finish()
 
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)  # > 126 MB L2
     for _ in range(args.warmup):

@@ -12,7 +12,7 @@ import torch.multiprocessing as mp
 
 from oracle import layer as OL
 from oracle import quantize as Q
-from quantized_base_lora_nf4_b200.dp import GradBucket, allreduce_adapter_grads, shard_rows
+from quantized_base_lora_nf4_b200.dp import GradBucket, OverlappedBuckets, allreduce_adapter_grads, shard_rows
 from synth import LinearSpec, linear_tensors
 
 
@@ -83,6 +83,57 @@ def test_two_rank_gradient_allreduce_matches_full_batch(pooled):
     q = ctx.Queue()
     port = _free_port()
     procs = [ctx.Process(target=_rank_main, args=(r, world, port, pooled, M, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    results = [q.get(timeout=120) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        if p.is_alive():
+            p.kill()
+    assert all(ok for _, ok, _ in results), results
+
+
+def test_overlapped_buckets_follow_layer_order_and_cap():
+    grads = [[torch.zeros(100), torch.zeros(28)], [torch.zeros(64)], [torch.zeros(200)], [torch.zeros(8)]]
+    ob = OverlappedBuckets(grads, cap_bytes=4 * 150)  # 150 floats
+    # layer 0 (128 floats) stays under the cap, layer 1 brings it to 192: first bucket after layer 1;
+    # layer 2 alone exceeds it; layer 3 is the last layer and closes the final bucket
+    assert ob.start_after == {1: 0, 2: 1, 3: 2}
+    assert [len(b.grads) for b in ob.buckets] == [3, 1, 1]
+    ob.layer_done(0)
+    ob.layer_done(1)  # no process group: nothing to exchange, nothing pending to wait on
+    ob.finish()
+
+
+def _overlap_rank_main(rank: int, world: int, port: int, q) -> None:
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    try:
+        dist.init_process_group("gloo", rank=rank, world_size=world)
+        g = torch.Generator().manual_seed(17)
+        shapes = [[(16, 64), (96, 16)], [(16, 32)], [(8, 128), (40, 8)], [(4, 4)], [(16, 256), (64, 16)]]
+        base = [[torch.randn(s, generator=g, dtype=torch.float64) for s in layer] for layer in shapes]
+        mine = [[(rank + 1) * t for t in layer] for layer in base]
+        ob = OverlappedBuckets(mine, cap_bytes=8 * 2000)
+        for i in range(len(mine)):  # the backward: a layer's gradients are final when it is done
+            ob.layer_done(i)
+        ob.finish()
+        total = sum(r + 1 for r in range(world))
+        ok = all(torch.equal(t, total * b) for lm, lb in zip(mine, base) for t, b in zip(lm, lb))
+        q.put((rank, ok and len(ob.buckets) > 1, None))
+    except Exception as e:  # reported to the parent, which fails the test
+        q.put((rank, False, repr(e)))
+    finally:
+        if dist.is_initialized():
+            dist.destroy_process_group()
+
+
+def test_two_rank_overlapped_buckets_sum_every_gradient():
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_overlap_rank_main, args=(r, world, port, q)) for r in range(world)]
     for p in procs:
         p.start()
     results = [q.get(timeout=120) for _ in range(world)]
