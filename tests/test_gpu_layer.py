@@ -163,3 +163,28 @@ def test_decode_ragged(cuda_lib, M, block, r):
     rows do not fill the last unit: 312 rows, K = 768 (three steps, an odd count)."""
     spec = LinearSpec("w", 312, 768, "nfk", 4, block, 256, r=r, s=0.5)
     run_and_check(cuda_lib, spec, M, seed=11 + M)
+
+
+def test_several_tiles_per_cta_without_token_pairs(cuda_lib):
+    # 10240 rows (and 10240 reduction columns for dX) give 80 row tiles; 100 tokens take two 64-token
+    # tiles and 300 tokens two 256-token tiles, so 160 tiles run on at most 148 persistent CTAs and some
+    # CTAs alternate their two TMEM accumulators across tiles, in the forward and in the input gradient
+    qlr = cuda_lib
+    spec = LinearSpec("w", 10240, 10240, "nfk", 4, 64, 256, r=16, s=0.5)
+    t0 = linear_tensors(spec, 300, seed=31)
+    q, Wdq = quantize_both(qlr, spec, t0["W"])
+    for M in (100, 300):
+        X, dY = t0["X"][:M], t0["dY"][:M]
+        st = qlr.new_status(DEV)
+        A, B = bf16_dev(t0["A"]), bf16_dev(t0["B"])
+        Y, T = qlr.forward(q, bf16_dev(X), A, B, spec.s, status=st)
+        dA, dB, dT = qlr.backward_lora(q, bf16_dev(X), bf16_dev(dY), T, B, spec.s, status=st)
+        dX = qlr.backward_dx(q, bf16_dev(dY), A, dT, status=st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        f = OL.forward(X, Wdq, t0["A"], t0["B"], spec.s)
+        b = OL.backward(dY, X, Wdq, t0["A"], t0["B"], spec.s)
+        assert OL.rel_fro(host(Y), f["Y"]) <= TOL
+        assert OL.rel_fro(host(dX), b["dX"]) <= TOL
+        assert OL.rel_fro(host(dA), b["dA"]) <= TOL
+        assert OL.rel_fro(host(dB), b["dB"]) <= TOL
