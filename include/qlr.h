@@ -289,7 +289,9 @@ QLR_API int qlr_backward_lora_noalloc(const qlr_qweight* w, const uint16_t* X, c
 /*
  * Input gradient through the frozen quantised weight (QLoRA explainer, "The contribution":
  * backpropagate through the frozen 4-bit weights into the adapters):
- *   dX = bf16( dY dequant(W) + P^T(dT A) )  [M, K]   (+ the previous dX when accumulate != 0)
+ *   dX = bf16( dY dequant(W) + P^T(dT A) )  [M, K]
+ * With accumulate != 0 the previous contents of dX are added to the fp32 result before its one rounding:
+ *   dX = bf16( dY dequant(W) + P^T(dT A) + dX_old )   (how the MLP block's up projection adds onto the gate's)
  * P^T spreads each pooled column over its group with weight 1/group.  Same fused
  * dequant + tcgen05 design as the forward, with the weight tile laid out MN-major.
  */
@@ -306,6 +308,25 @@ QLR_API int qlr_backward_dx(const qlr_qweight* w, const uint16_t* dY, int64_t M,
 QLR_API int qlr_swiglu_forward(const uint16_t* G, const uint16_t* U, uint16_t* H, int64_t n, void* stream);
 QLR_API int qlr_swiglu_backward(const uint16_t* dH, const uint16_t* G, const uint16_t* U, uint16_t* dG, uint16_t* dU,
                         int64_t n, void* stream);
+
+/*
+ * Bound of the pipeline waits (failure detection; the pages have no counterpart).  Every handshake of the
+ * pipelined kernels (fused GEMM, adapter GEMM, decode) waits at most this many SM clock cycles; past it
+ * the kernel raises an abort flag, every role leaves its loop, the CTA waits (with a fixed bound) for its
+ * own TMA copies and tensor-core work still in flight, releases its tensor memory and sets
+ * *status = QLR_ERR_TIMEOUT, so the context stays usable.  The process-wide default is 4e9 cycles (about
+ * 2 s at the B200 boost clock); cycles < 0 restores it.  Applies to the launches that follow the call;
+ * returns the previous bound.  Meant for tests of the timeout path: a short bound makes a healthy kernel
+ * time out too.
+ */
+QLR_API long long qlr_set_wait_limit(long long cycles);
+
+/*
+ * Launches one small kernel that holds tensor memory and waits on a barrier nothing will complete, with
+ * the current wait bound: it must set *status = QLR_ERR_TIMEOUT (status: one device int32, required),
+ * release the tensor memory and return.  A test of the timeout path that needs no fault.
+ */
+QLR_API int qlr_wait_selftest(int32_t* status, void* stream);
 
 /* Number of SMs of the current device (used to size persistent grids); <= 0 on error. */
 QLR_API int qlr_device_sm_count(void);

@@ -15,9 +15,13 @@
 
 namespace qlr {
 
+constexpr long long kDefaultWaitCycles = 4000000000LL;  // ~2 s at the B200 boost clock
+
 __device__ int32_t g_status_sink;
 
 static std::atomic<uint64_t> g_launches{0};
+static std::atomic<long long> g_wait_cycles{kDefaultWaitCycles};
+long long wait_limit_cycles() { return g_wait_cycles.load(std::memory_order_relaxed); }
 void count_launch(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed); }
 
 int32_t* status_or_sink(int32_t* status) {
@@ -223,6 +227,7 @@ int run_adapter(const AdapterGemm& g, int r, int out_mode, float scale, int pool
   p.out = out;
   p.ld_out = ld_out;
   p.status = status;
+  p.wait_cycles = wait_limit_cycles();
   if (p.splits > 1) p.part = reinterpret_cast<float*>(ws);
   if ((rc = cuda_rc(launch_adapter(g.a_src, g.b_src, g.bn, p, maps, st)))) return rc;
   if (p.splits > 1) return cuda_rc(launch_adapter_reduce(p, g.bn, st));
@@ -251,6 +256,10 @@ const char* qlr_error_string(int code) {
 int qlr_version(void) { return 100; }
 
 uint64_t qlr_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+long long qlr_set_wait_limit(long long cycles) {
+  return g_wait_cycles.exchange(cycles < 0 ? kDefaultWaitCycles : cycles, std::memory_order_relaxed);
+}
 
 int qlr_device_sm_count(void) { return device_sm_count(); }
 
@@ -426,6 +435,7 @@ int qlr_forward_base(const qlr_qweight* w, const uint16_t* X, int64_t M, const u
   p.tail_a_rows = N;
   p.tail_a_cols = r;
   p.status = stat;
+  p.wait_cycles = wait_limit_cycles();
   return cuda_rc(launch_gemm(A_DQ_K, B_TMA_K, tok, OUT_BF16_T, 0, p, maps, st));
 }
 
@@ -565,6 +575,7 @@ int qlr_backward_dx(const qlr_qweight* w, const uint16_t* dY, int64_t M, const u
   p.tail_a_cols = pooled ? K / w->group : K;
   p.tail_pool_L = pooled ? w->group : 0;
   p.status = stat;
+  p.wait_cycles = wait_limit_cycles();
   return cuda_rc(launch_gemm(A_DQ_MN, B_TMA_K, tok, OUT_BF16_T, 1, p, maps, st));
 }
 

@@ -17,6 +17,9 @@ Levels levels_for(int bits);
 // Status sink used when the caller passes no status word.
 int32_t* status_or_sink(int32_t* status);
 
+// Bound (SM clock cycles) given to the pipeline waits of the kernels launched next (qlr_set_wait_limit).
+long long wait_limit_cycles();
+
 __device__ __forceinline__ void report(int32_t* status, int32_t code) { atomicExch(status, code); }
 
 // ---- launch wrappers (quantize.cu) ----

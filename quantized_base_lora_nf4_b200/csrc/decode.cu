@@ -48,6 +48,7 @@ struct DecodeParams {
   uint16_t* Y;              // [M, N] bf16
   Levels lv;
   int32_t* status;
+  long long wait_cycles;    // bound of every pipeline wait (SM clock cycles)
 };
 
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
@@ -189,7 +190,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         int sl = 0;
         uint32_t ph = 0;  // ring slot and the parity of its current fill
         for (int s = 0; s < nsteps; ++s) {
-          if (!mbar_wait(&bars->empty[sl], ph ^ 1, abort_flag)) break;
+          if (!mbar_wait(&bars->empty[sl], ph ^ 1, abort_flag, p.wait_cycles)) break;
           uint8_t* slot = gen(kRingAddr + sl * C::kSlot);
           mbar_arrive_expect_tx(&bars->full[sl], nu * C::kUnitCodes + 4 * C::kXQ);
           tma_load_2d(slot, tm_codes, s * 128, static_cast<int32_t>(prow0), &bars->full[sl]);
@@ -199,6 +200,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
           if (++sl == kSlots) {
             sl = 0;
             ph ^= 1;
+          }
+        }
+        // after an abort, the copies still in flight must land before the CTA may exit: wait for the
+        // last fill of every slot (one outstanding fill per slot at most)
+        if (*abort_flag) {
+          for (int k = 0; k < kSlots; ++k) {
+            if (--sl < 0) {
+              sl = kSlots - 1;
+              ph ^= 1;
+            }
+            mbar_drain(&bars->full[sl], ph);
           }
         }
       }
@@ -291,7 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       int sl = 0;
       uint32_t ph = 0;  // ring slot and the parity of its current fill
       for (int s = 0; s < nsteps; ++s) {
-        const bool ok = mbar_wait(&bars->full[sl], ph, abort_flag);
+        const bool ok = mbar_wait(&bars->full[sl], ph, abort_flag, p.wait_cycles);
         if (!__all_sync(0xffffffffu, ok)) break;
         const uint32_t slot = kRingAddr + sl * C::kSlot;  // codes [unit][16 rows][128 B], then the input quarters
         const uint32_t xs = slot + kMaxUnits * C::kUnitCodes;
@@ -428,6 +440,7 @@ cudaError_t launch_decode(const qlr_qweight* w, const uint16_t* X, int64_t M, co
   p.Y = Y;
   p.lv = levels_for(4);
   p.status = status;
+  p.wait_cycles = wait_limit_cycles();
   const int nt = M <= 8 ? 1 : 2;
   CUtensorMap tc_lo, tc_hi, tx;
   if (make_tmap(&tc_lo, w->codes, 1, w->N, w->K / 2, 16 * p.nu_lo, 128, 128)) return cudaErrorInvalidValue;

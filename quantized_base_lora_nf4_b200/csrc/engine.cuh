@@ -180,12 +180,26 @@ __device__ __forceinline__ void dequant_row64(const DqParams& dq, const uint8_t*
 }
 
 // Writes one 32-column chunk of an fp32 accumulator row as bf16 into out^T (out row = D column),
-// transposing through a per-warp 32x32 staging tile so every global store is 16 bytes wide.
+// transposing through a per-warp 32x32 staging tile so every global store is 16 bytes wide.  With
+// `accumulate` the previous bf16 value is added to the fp32 accumulator first and the sum rounded to bf16
+// once (the warp reads 32 consecutive outputs of one row per load).
 __device__ __forceinline__ void store_chunk_bf16_t(const uint32_t (&v)[32], uint16_t* stg, int lane, int dcol0,
                                                    int drow0, const GemmParams& p) {
+  if (p.accumulate) {
+    const int ocol = drow0 + lane;
+    const uint16_t* base = static_cast<const uint16_t*>(p.out) + ocol;
+#pragma unroll 8
+    for (int jj = 0; jj < 32; ++jj) {
+      const int orow = dcol0 + jj;
+      const float old = (orow < p.Nn && ocol < p.Mm) ? bf16_bits_to_f32(base[static_cast<int64_t>(orow) * p.ldo]) : 0.f;
+      stg[jj * 32 + lane] =
+          static_cast<uint16_t>(pack_bf16x2_rn(__fadd_rn(__uint_as_float(v[jj]), old), 0.f) & 0xFFFFu);
+    }
+  } else {
 #pragma unroll
-  for (int jj = 0; jj < 32; ++jj)
-    stg[jj * 32 + lane] = static_cast<uint16_t>(pack_bf16x2_rn(__uint_as_float(v[jj]), 0.f) & 0xFFFFu);
+    for (int jj = 0; jj < 32; ++jj)
+      stg[jj * 32 + lane] = static_cast<uint16_t>(pack_bf16x2_rn(__uint_as_float(v[jj]), 0.f) & 0xFFFFu);
+  }
   __syncwarp();
 #pragma unroll
   for (int t = 0; t < 4; ++t) {
@@ -194,17 +208,8 @@ __device__ __forceinline__ void store_chunk_bf16_t(const uint32_t (&v)[32], uint
     const int orow = dcol0 + jj;              // output row (D column)
     const int ocol = drow0 + part * 8;        // output column (D row)
     if (orow < p.Nn && ocol < p.Mm) {
-      uint4 val = *reinterpret_cast<const uint4*>(stg + jj * 32 + part * 8);
+      const uint4 val = *reinterpret_cast<const uint4*>(stg + jj * 32 + part * 8);
       uint16_t* dst = static_cast<uint16_t*>(p.out) + static_cast<int64_t>(orow) * p.ldo + ocol;
-      if (p.accumulate) {
-        const uint4 old = *reinterpret_cast<const uint4*>(dst);
-        uint32_t* nv = reinterpret_cast<uint32_t*>(&val);
-        const uint32_t* ov = reinterpret_cast<const uint32_t*>(&old);
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          nv[e] = pack_bf16x2_rn(bf16_bits_to_f32(nv[e] & 0xFFFFu) + bf16_bits_to_f32(ov[e] & 0xFFFFu),
-                                 bf16_bits_to_f32(nv[e] >> 16) + bf16_bits_to_f32(ov[e] >> 16));
-      }
       *reinterpret_cast<uint4*>(dst) = val;
     }
   }

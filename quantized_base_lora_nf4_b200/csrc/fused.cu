@@ -193,7 +193,7 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
         for (int ks = 0; ks < nsteps && ok; ++ks) {
           for (int h = 0; h < HALVES; ++h, ++j) {
             const int s = j % NSB;
-            if (!mbar_wait(&bars->b_empty[s], ((j / NSB) & 1) ^ 1, abort_flag)) { ok = false; break; }
+            if (!mbar_wait(&bars->b_empty[s], ((j / NSB) & 1) ^ 1, abort_flag, p.wait_cycles)) { ok = false; break; }
             uint64_t* fb = &bars->b_full[s];
             mbar_arrive_expect_tx(fb, C::kB);
             if (ks < nmain)
@@ -205,8 +205,7 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
       }
       const uint32_t first = j > NSB ? j - NSB : 0;
       for (uint32_t q = first; q < j; ++q) {
-        volatile int never = 0;
-        mbar_wait(&bars->b_full[q % NSB], (q / NSB) & 1, &never);
+        mbar_drain(&bars->b_full[q % NSB], (q / NSB) & 1);
       }
     }
   } else if (warp == kCodesWarp) {
@@ -219,7 +218,7 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
         const int m0 = tile_m0(tile);
         for (int ks = 0; ks < nmain; ks += p.code_steps, ++jc) {
           const int s = static_cast<int>(jc & mask);
-          if (!mbar_wait(&bars->c_empty[s], ((jc >> lg) & 1) ^ 1, abort_flag)) break;
+          if (!mbar_wait(&bars->c_empty[s], ((jc >> lg) & 1) ^ 1, abort_flag, p.wait_cycles)) break;
           uint64_t* fb = &bars->c_full[s];
           mbar_arrive_expect_tx(fb, p.code_box_bytes);
           if (!MN)  // [128 W rows][8 kb bytes per step]
@@ -230,8 +229,7 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
       }
       const uint32_t first = jc > static_cast<uint32_t>(ncs) ? jc - ncs : 0;
       for (uint32_t q = first; q < jc; ++q) {
-        volatile int never = 0;
-        mbar_wait(&bars->c_full[q & mask], (q >> lg) & 1, &never);
+        mbar_drain(&bars->c_full[q & mask], (q >> lg) & 1);
       }
     }
   } else if (warp == kIssuerWarp) {
@@ -249,11 +247,11 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
       for (int tile = blockIdx.x; tile < n_tiles_total && ok; tile += gridDim.x, ++it) {
         const int acc = PAIR ? 0 : (it & 1);
         const uint32_t acc_par = PAIR ? ((it & 1) ^ 1) : (((it >> 1) & 1) ^ 1);
-        if (!mbar_wait(&bars->acc_empty[acc], acc_par, abort_flag)) break;
+        if (!mbar_wait(&bars->acc_empty[acc], acc_par, abort_flag, p.wait_cycles)) break;
         tc_fence_after();
         for (int ks = 0; ks < nsteps && ok; ++ks, ++j) {
           const int sa = j % NSA;
-          if (!mbar_wait(&bars->a_full[sa], (j / NSA) & 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(&bars->a_full[sa], (j / NSA) & 1, abort_flag, p.wait_cycles)) { ok = false; break; }
           const uint64_t ad0 = a_desc0 + static_cast<uint32_t>((sa * C::kA) >> 4);
           int nsub = 4;
           if (ks >= nmain) {
@@ -262,7 +260,7 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
           }
           for (int h = 0; h < HALVES; ++h, ++jb) {
             const int sb = jb % NSB;
-            if (!mbar_wait(&bars->b_full[sb], (jb / NSB) & 1, abort_flag)) { ok = false; break; }
+            if (!mbar_wait(&bars->b_full[sb], (jb / NSB) & 1, abort_flag, p.wait_cycles)) { ok = false; break; }
             tc_fence_after();
             const uint64_t bd0 = b_desc0 + static_cast<uint32_t>((sb * C::kB) >> 4);
             const uint32_t d_tmem = tmem_base + (PAIR ? h : acc) * BN;
@@ -283,8 +281,7 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
         umma_commit(&bars->acc_full[acc]);
       }
       umma_commit(&bars->drain);
-      volatile int never = 0;
-      mbar_wait(&bars->drain, 0, &never);
+      mbar_drain(&bars->drain, 0);
     }
   } else if (warp >= 2 && warp <= 5) {
     // ------------------------------------------------------------------ epilogue
@@ -295,7 +292,7 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
       const int m0 = tile_m0(tile), n0 = tile_n0(tile);
       const int acc = PAIR ? 0 : (it & 1);
       const uint32_t acc_par = PAIR ? (it & 1) : ((it >> 1) & 1);
-      const bool got = mbar_wait(&bars->acc_full[acc], acc_par, abort_flag);
+      const bool got = mbar_wait(&bars->acc_full[acc], acc_par, abort_flag, p.wait_cycles);
       __syncwarp();
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
@@ -367,13 +364,13 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
       const eng::DqConst nxt = have_next ? prefetch() : eng::DqConst{0u, 0u};
 
       const int sa = c_j % NSA;
-      if (!mbar_wait(&bars->a_empty[sa], ((c_j / NSA) & 1) ^ 1, abort_flag)) break;
+      if (!mbar_wait(&bars->a_empty[sa], ((c_j / NSA) & 1) ^ 1, abort_flag, p.wait_cycles)) break;
       uint8_t* st_a = ring_a + sa * C::kA;
       if (c_ks < nmain) {
         const int kb = p.code_bits, lg = p.code_slots_log2;
         const uint32_t box = p.code_steps == 2 ? c_jc >> 1 : c_jc, sub = p.code_steps == 2 ? (c_jc & 1) : 0;
         const int sc = static_cast<int>(box & ((1u << lg) - 1u));
-        if (!mbar_wait(&bars->c_full[sc], (box >> lg) & 1, abort_flag)) break;
+        if (!mbar_wait(&bars->c_full[sc], (box >> lg) & 1, abort_flag, p.wait_cycles)) break;
         const uint8_t* st_c = ring_c + sc * p.code_box_bytes;
         int64_t row, col;
         bool valid;

@@ -41,6 +41,7 @@ struct alignas(8) ABars {
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
+  int ep_ok[4];
   float chunk[4 * 64];
 };
 
@@ -165,7 +166,7 @@ __global__ void __launch_bounds__(kThreadsAdapter, 1)
         const int m0 = tile * 128;
         for (int ks = 0; ks < nsteps; ++ks, ++j) {
           const int s = j % NS;
-          if (!mbar_wait(&bars->empty[s], ((j / NS) & 1) ^ 1, abort_flag)) break;
+          if (!mbar_wait(&bars->empty[s], ((j / NS) & 1) ^ 1, abort_flag, p.wait_cycles)) break;
           uint8_t* st_a = smem + s * C::kStage;
           uint8_t* st_b = st_a + C::kA;
           uint64_t* fb = &bars->full[s];
@@ -187,8 +188,7 @@ __global__ void __launch_bounds__(kThreadsAdapter, 1)
       }
       const uint32_t first = j > NS ? j - NS : 0;
       for (uint32_t qq = first; qq < j; ++qq) {
-        volatile int never = 0;
-        mbar_wait(&bars->full[qq % NS], (qq / NS) & 1, &never);
+        mbar_drain(&bars->full[qq % NS], (qq / NS) & 1);
       }
     }
   } else if (warp == 1) {
@@ -201,12 +201,12 @@ __global__ void __launch_bounds__(kThreadsAdapter, 1)
         int tile, split, kb, nsteps;
         item_coords(item, tile, split, kb, nsteps);
         const int acc = it & 1;
-        if (!mbar_wait(&bars->acc_empty[acc], ((it >> 1) & 1) ^ 1, abort_flag)) break;
+        if (!mbar_wait(&bars->acc_empty[acc], ((it >> 1) & 1) ^ 1, abort_flag, p.wait_cycles)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
         for (int ks = 0; ks < nsteps; ++ks, ++j) {
           const int s = j % NS;
-          if (!mbar_wait(&bars->full[s], (j / NS) & 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(&bars->full[s], (j / NS) & 1, abort_flag, p.wait_cycles)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(smem + s * C::kStage);
           const uint32_t b_addr = a_addr + C::kA;
@@ -229,8 +229,7 @@ __global__ void __launch_bounds__(kThreadsAdapter, 1)
         umma_commit(&bars->acc_full[acc]);  // also for an empty item: the epilogue then reads zeros
       }
       umma_commit(&bars->drain);
-      volatile int never = 0;
-      mbar_wait(&bars->drain, 0, &never);
+      mbar_drain(&bars->drain, 0);
     }
   } else {
     // ------------------------------------------------------------------ epilogue (warps 2..5)
@@ -242,9 +241,18 @@ __global__ void __launch_bounds__(kThreadsAdapter, 1)
       item_coords(item, tile, split, kb, nsteps);
       const int m0 = tile * 128;
       const int acc = it & 1;
-      const bool got = mbar_wait(&bars->acc_full[acc], (it >> 1) & 1, abort_flag);
+      const bool got = mbar_wait(&bars->acc_full[acc], (it >> 1) & 1, abort_flag, p.wait_cycles);
       __syncwarp();
-      if (!__all_sync(0xffffffffu, got)) break;
+      bool all_got = __all_sync(0xffffffffu, got);
+      if (S == 1 && p.out_mode == ADAPTER_COLS_F32 && p.pool_L > 1) {
+        // the pooled store synchronises the four epilogue warps on a named barrier, so they must leave
+        // the loop together: one joint decision after an abort
+        if (lane == 0) bars->ep_ok[q] = all_got ? 1 : 0;
+        named_bar_sync(1, 128);
+        all_got = bars->ep_ok[0] && bars->ep_ok[1] && bars->ep_ok[2] && bars->ep_ok[3];
+        named_bar_sync(1, 128);
+      }
+      if (!all_got) break;
       tc_fence_after();
       float v[BN];
 #pragma unroll

@@ -55,6 +55,7 @@ struct GemmParams {
   int64_t tail_a_rows, tail_a_cols;
   int tail_pool_L;       // input gradient with the pooled adapter: tail row j is A[j, k / L] / L
   int32_t* status;
+  long long wait_cycles; // bound of every pipeline wait (SM clock cycles)
 };
 
 struct GemmMaps {
@@ -82,6 +83,7 @@ struct AdapterParams {
   int64_t ld_out;
   float* part;       // [splits][m_tiles * 128][BN] fp32 (splits > 1)
   int32_t* status;
+  long long wait_cycles;  // bound of every pipeline wait (SM clock cycles)
 };
 
 cudaError_t launch_adapter(int a_src, int b_src, int bn, const AdapterParams& p, const GemmMaps& maps,

@@ -1,7 +1,7 @@
 // Thin inline-PTX wrappers for sm_100a: mbarriers, TMA tile loads, tcgen05 (TMEM
 // allocation, UMMA issue/commit, TMEM loads) and the fences that order them.
-// Every wait is bounded: after ~2 s of SM clock it raises a CTA-wide abort flag and
-// reports QLR_ERR_TIMEOUT through the caller's status word instead of hanging.
+// Every wait is bounded: past its bound (~2 s of SM clock by default) it raises a CTA-wide abort flag and
+// the kernel reports QLR_ERR_TIMEOUT through the caller's status word instead of hanging.
 #pragma once
 #include <cstdint>
 #include <cuda_runtime.h>
@@ -37,24 +37,40 @@ QLR_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-constexpr long long kWaitCycles = 4000000000LL;  // ~2 s at the B200 boost clock
+// Default bound of a pipeline wait: ~2 s at the B200 boost clock.  Each launch carries its own bound
+// (qlr_set_wait_limit changes it for the launches that follow, for tests of the timeout path).
+constexpr long long kWaitCycles = 4000000000LL;
+// Bound of the waits a CTA makes after an abort for its own TMA copies and MMAs still in flight: these
+// always complete, and the CTA must not exit (or free its tensor memory) before they have.
+constexpr long long kDrainCycles = 4000000000LL;
 
-// Waits for the phase with the given parity to complete.  Returns false (and raises
-// *abort) when the bound expires or another role already aborted.  Polls try_wait without a
-// suspend hint: measured on B200, a suspended waiter is not resumed promptly when a TMA
-// transaction or a tcgen05.commit completes the phase, which adds microseconds to every handshake.
-QLR_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+// Waits for the phase with the given parity to complete.  Returns false (and raises *abort) when the
+// bound `limit` (SM clock cycles) expires or another role already aborted.  Polls try_wait without a
+// suspend hint: measured on B200, a suspended waiter is not resumed promptly when a TMA transaction or a
+// tcgen05.commit completes the phase, which adds microseconds to every handshake.
+QLR_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, long long limit) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63) == 0) {
       if (*abort_flag) return false;
-      if (clock64() - t0 > kWaitCycles) {
+      if (clock64() - t0 > limit) {
         *abort_flag = 1;
         return false;
       }
     }
+  }
+}
+
+// Waits for this CTA's own asynchronous work (a TMA copy or the MMAs behind a commit) to land, whatever the
+// abort flag says, with the fixed drain bound.
+QLR_DEV bool mbar_drain(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63) == 0 && clock64() - t0 > kDrainCycles) return false;
   }
 }
 

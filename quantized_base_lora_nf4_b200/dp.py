@@ -38,12 +38,18 @@ class GradBucket:
         self.sizes = [g.numel() for g in self.grads]
         self.flat = torch.empty(sum(self.sizes), dtype=dt, device=dev)
 
-    def start(self, group: Optional[dist.ProcessGroup] = None):
+    def start(self, group: Optional[dist.ProcessGroup] = None, stream=None):
         """Copy the gradients in and start the SUM all-reduce without waiting for it (None when there
-        is nothing to exchange).  With NCCL the collective is ordered after the copies on the current
-        stream and runs beside whatever that stream does next."""
+        is nothing to exchange).  The copies and, with NCCL, the collective are ordered on torch's
+        current stream; `stream` names the CUDA stream the backward ran on when that is another one
+        (the library's calls take an explicit stream), and the current stream then waits for it before
+        the copies, so the exchange never reads gradients the backward has not finished writing."""
         if not dist.is_initialized() or dist.get_world_size(group) == 1:
             return None
+        if stream is not None and self.flat.is_cuda:
+            cur = torch.cuda.current_stream(self.flat.device)
+            if stream != cur:
+                cur.wait_stream(stream)
         off = 0
         for g, n in zip(self.grads, self.sizes):
             self.flat[off:off + n].copy_(g.reshape(-1))
@@ -87,10 +93,11 @@ class OverlappedBuckets:
                 cur, cur_bytes = [], 0
         self.pending: List[Tuple[int, object]] = []
 
-    def layer_done(self, i: int, group: Optional[dist.ProcessGroup] = None) -> None:
+    def layer_done(self, i: int, group: Optional[dist.ProcessGroup] = None, stream=None) -> None:
+        """Layer i's backward has been issued (on `stream`, default torch's current stream)."""
         b = self.start_after.get(i)
         if b is not None:
-            self.pending.append((b, self.buckets[b].start(group)))
+            self.pending.append((b, self.buckets[b].start(group, stream)))
 
     def finish(self) -> None:
         for b, work in self.pending:

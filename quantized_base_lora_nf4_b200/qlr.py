@@ -31,6 +31,7 @@ EXPORTED = (
     "qlr_backward_dx", "qlr_swiglu_forward", "qlr_swiglu_backward", "qlr_device_sm_count", "qlr_lora_down",
     "qlr_forward_base", "qlr_launch_count", "qlr_backward_lora_noalloc", "qlr_lqlora_init_workspace_bytes",
     "qlr_lqlora_init", "qlr_nf_quant_error_workspace_bytes", "qlr_nf_quant_error", "qlr_lqlora_allocate",
+    "qlr_set_wait_limit", "qlr_wait_selftest",
 )
 
 
@@ -87,6 +88,8 @@ def lib() -> ctypes.CDLL:
         "qlr_nf_quant_error_workspace_bytes": (SZ, [I64, I64, I, I, I]),
         "qlr_nf_quant_error": (I, [P, I64, I64, I, I, I, P, P, SZ, P, P]),
         "qlr_lqlora_allocate": (I, [P, P, I, I, I64, I64, P, P]),
+        "qlr_set_wait_limit": (ctypes.c_longlong, [ctypes.c_longlong]),
+        "qlr_wait_selftest": (I, [P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -321,6 +324,17 @@ def forward_base(q: QWeight, X: torch.Tensor, B: torch.Tensor, T_save: torch.Ten
 
 def launch_count() -> int:
     return int(lib().qlr_launch_count())
+
+
+def set_wait_limit(cycles: int) -> int:
+    """Bound (SM clock cycles) of the pipeline waits of the kernels launched next; < 0 restores the
+    default.  Returns the previous bound."""
+    return int(lib().qlr_set_wait_limit(int(cycles)))
+
+
+def wait_selftest(status: torch.Tensor, stream=None) -> None:
+    """A kernel whose wait can only run out: it must set *status to the timeout code and free its tensor memory."""
+    _check(lib().qlr_wait_selftest(_ptr(status), _stream(stream)), "qlr_wait_selftest")
 
 
 def backward_lora(q: QWeight, X: torch.Tensor, dY: torch.Tensor, T_save: torch.Tensor, B: torch.Tensor, s: float,

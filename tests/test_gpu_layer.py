@@ -12,6 +12,30 @@ from tests.gpu_helpers import DEV, bf16_dev, f32_dev, host
 pytestmark = [pytest.mark.gpu, pytest.mark.filterwarnings("ignore::RuntimeWarning")]
 
 TOL = 1e-2
+# a single token row (or weight row) may be off by at most this much relative to its own norm: the
+# whole-tensor bound alone would let one row of 2048 be 45 % wrong
+ROW_TOL = 3e-2
+
+
+def worst_row(got, ref, axis=1):
+    """Largest error of one row (axis=1) or column (axis=0), relative to that row's norm, the norm floored
+    at a tenth of the mean so that a row whose exact value nearly cancels is not judged on its own."""
+    got, ref = np.asarray(got, np.float64), np.asarray(ref, np.float64)
+    num = np.linalg.norm(got - ref, axis=axis)
+    den = np.linalg.norm(ref, axis=axis)
+    den = np.maximum(den, 0.1 * den.mean() + 1e-300)
+    return float((num / den).max())
+
+
+def check_close(got, ref, what):
+    """The relative Frobenius bound on the whole tensor, and the per-row (and, with 8 or more rows,
+    per-column) bound, so an error confined to one token, one weight row, one tile or a ragged tail shows."""
+    got = np.asarray(got, np.float64)
+    assert OL.rel_fro(got, ref) <= TOL, (what, OL.rel_fro(got, ref))
+    if got.ndim == 2 and got.size:
+        assert worst_row(got, ref, 1) <= ROW_TOL, (what, "row", worst_row(got, ref, 1))
+        if got.shape[0] >= 8:
+            assert worst_row(got, ref, 0) <= ROW_TOL, (what, "column", worst_row(got, ref, 0))
 
 
 def quantize_both(qlr, spec, W):
@@ -36,20 +60,20 @@ def run_and_check(qlr, spec, M, seed=0, rows=None, accumulate_check=False):
     sel = slice(None) if rows is None else rows
     Xs, dYs = t["X"][sel], t["dY"][sel]
     f = OL.forward(Xs, Wdq, t["A"], t["B"], spec.s, L)
-    assert OL.rel_fro(host(Y)[sel], f["Y"]) <= TOL
-    assert OL.rel_fro(host(T)[sel], spec.s * f["T"]) <= TOL
+    check_close(host(Y)[sel], f["Y"], "Y")
+    check_close(host(T)[sel], spec.s * f["T"], "T")
     bsel = OL.backward(dYs, Xs, Wdq, t["A"], t["B"], spec.s, L)
-    assert OL.rel_fro(host(dT)[sel], bsel["dT"]) <= TOL
-    assert OL.rel_fro(host(dX)[sel], bsel["dX"]) <= TOL
+    check_close(host(dT)[sel], bsel["dT"], "dT")
+    check_close(host(dX)[sel], bsel["dX"], "dX")
     # adapter gradients reduce over every token: checked in full
     full = bsel if rows is None else OL.backward(t["dY"], t["X"], Wdq, t["A"], t["B"], spec.s, L)
-    assert OL.rel_fro(host(dA), full["dA"]) <= TOL
-    assert OL.rel_fro(host(dB), full["dB"]) <= TOL
+    check_close(host(dA), full["dA"], "dA")
+    check_close(host(dB), full["dB"], "dB")
     if accumulate_check:
         dX2 = dX.clone()
         qlr.backward_dx(q, dY, A, dT, pooled=spec.pooled, dX=dX2, accumulate=True)
         torch.cuda.synchronize()
-        assert OL.rel_fro(host(dX2)[sel], 2 * bsel["dX"]) <= TOL
+        check_close(host(dX2)[sel], 2 * bsel["dX"], "dX accumulated")
     return {"Y": Y, "dX": dX, "dA": dA, "dB": dB}
 
 
@@ -115,10 +139,10 @@ def test_swiglu(cuda_lib):
     H = qlr.swiglu_forward(bf16_dev(G), bf16_dev(U))
     dG, dU = qlr.swiglu_backward(bf16_dev(dH), bf16_dev(G), bf16_dev(U))
     torch.cuda.synchronize()
-    assert OL.rel_fro(host(H), OL.swiglu_forward(G, U)) <= TOL
+    check_close(host(H), OL.swiglu_forward(G, U), "H")
     rg, ru = OL.swiglu_backward(dH, G, U)
-    assert OL.rel_fro(host(dG), rg) <= TOL
-    assert OL.rel_fro(host(dU), ru) <= TOL
+    check_close(host(dG), rg, "dG")
+    check_close(host(dU), ru, "dU")
 
 
 def test_zero_tokens(cuda_lib):
@@ -152,8 +176,8 @@ def test_decode_projection_full_size_sampled_rows(cuda_lib, M):
     Wdq = np.concatenate([Q.dequant_nfk(Q.quantize_nfk(t["W"][r:r + 2], 4, 64, 256)) for r in rows])
     ref = OL.forward(X, np.zeros((2 * len(rows), spec.K)), t["A"], t["B"][sel], spec.s)["Y"] + \
         X.astype(np.float64) @ Wdq.astype(np.float64).T
-    assert OL.rel_fro(Yh[:, sel], ref) <= TOL
-    assert OL.rel_fro(host(T), spec.s * OL.forward(X, np.zeros((1, spec.K)), t["A"], t["B"][:1], spec.s)["T"]) <= TOL
+    check_close(Yh[:, sel], ref, "Y")
+    check_close(host(T), spec.s * OL.forward(X, np.zeros((1, spec.K)), t["A"], t["B"][:1], spec.s)["T"], "T")
 
 
 @pytest.mark.parametrize("M", [1, 5, 16])
@@ -184,7 +208,7 @@ def test_several_tiles_per_cta_without_token_pairs(cuda_lib):
         assert int(st.item()) == 0
         f = OL.forward(X, Wdq, t0["A"], t0["B"], spec.s)
         b = OL.backward(dY, X, Wdq, t0["A"], t0["B"], spec.s)
-        assert OL.rel_fro(host(Y), f["Y"]) <= TOL
-        assert OL.rel_fro(host(dX), b["dX"]) <= TOL
-        assert OL.rel_fro(host(dA), b["dA"]) <= TOL
-        assert OL.rel_fro(host(dB), b["dB"]) <= TOL
+        check_close(host(Y), f["Y"], "Y")
+        check_close(host(dX), b["dX"], "dX")
+        check_close(host(dA), b["dA"], "dA")
+        check_close(host(dB), b["dB"], "dB")

@@ -121,3 +121,48 @@ def test_qalora_merge_bit_exact_and_lossless(cuda_lib):
     np.testing.assert_array_equal(q.zero.cpu().numpy().view(np.uint16), zp.view(np.uint16))
     Wd = qlr.dequant(q)
     np.testing.assert_array_equal(bf16_bits(host(Wd)), bf16_bits(Q.dequant_int4_group(ref, zero=zp)))
+
+
+def _nf_tie_inputs(bits: int, per_pair: int = 6) -> np.ndarray:
+    """fp32 values u between each pair of adjacent levels a < b at the switch from the lower to the upper
+    level: every u whose fp32 distances to a and b are equal (the oracle keeps the lower index), and the
+    last u nearer a and the first u nearer b, found by scanning the fp32 neighbours of the midpoint."""
+    from oracle.codebook import nf_codebook_f32
+    lev = nf_codebook_f32(bits)
+    out = []
+    for a, b in zip(lev[:-1], lev[1:]):
+        mid = np.float32((np.float64(a) + np.float64(b)) / 2)
+        base = int(np.array([mid]).view(np.int32)[0])
+        u = np.arange(base - 512, base + 513, dtype=np.int64).astype(np.int32).view(np.float32)
+        u = np.unique(u[(u > a) & (u < b)])
+        da = np.abs((u - a).astype(np.float32))
+        db = np.abs((u - b).astype(np.float32))
+        out.extend(u[da == db][:per_pair].tolist())
+        below, above = u[da < db], u[da > db]
+        out.extend([below.max(), above.min()])
+    return np.array(out, np.float32)
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+@pytest.mark.parametrize("block,dq", [(64, 256), (128, 0)])
+def test_nf_quantize_ties_bit_exact(cuda_lib, bits, block, dq):
+    """Inputs exactly between two levels in fp32 distance: the GPU's level search must keep the lower index,
+    as the oracle's first-index argmin does.  Blocks with absmax 1 (u = w exactly) and blocks scaled by
+    0.8125 and 3.0 (the division decides which side the quotient falls)."""
+    qlr = cuda_lib
+    ties = _nf_tie_inputs(bits)
+    assert ties.size >= 2 * (2 ** bits - 1)
+    rows = []
+    for c1 in (1.0, 0.8125, 3.0):
+        for start in range(0, ties.size, block - 1):
+            blk = np.zeros(block, np.float32)
+            seg = (ties[start:start + block - 1] * np.float32(c1)).astype(np.float32)
+            blk[0] = np.float32(c1)              # the block's absmax
+            blk[1:1 + seg.size] = seg
+            rows.append(blk)
+    W = np.concatenate(rows)
+    W = np.concatenate([W, np.zeros((-W.size) % 256, np.float32)]).reshape(-1, 256)
+    ref = Q.quantize_nfk(W, bits, block, dq)
+    q = qlr.quantize_nf4(f32_dev(W), bits, block, dq)
+    torch.cuda.synchronize()
+    _compare_nf(q, ref)

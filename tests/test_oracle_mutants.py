@@ -34,6 +34,18 @@ MUTANTS = [
     ("lqlora.py", "U, S, Vt = np.linalg.svd(W64 - deq, full_matrices=False)",
      "U, S, Vt = np.linalg.svd(W64, full_matrices=False)", "test_oracle_lqlora.py"),
     ("allocation.py", "for i in range(m - 1, -1, -1):", "for i in range(m):", "test_oracle_allocation.py"),
+    # the dequantised value's rounding (pinned by literal bf16 ties in test_oracle_dequant_rounding.py)
+    ("quantize.py", "return bf16_rn(vals.reshape(-1)[: N * K]).reshape(N, K)", "return vals.reshape(-1)[: N * K].reshape(N, K)",
+     "test_oracle_dequant_rounding.py"),
+    ("quantize.py", 'vals = levels[q["codes"]].reshape(-1, block) * scales[:, None]   # fp32 * fp32 -> fp32',
+     'vals = (levels[q["codes"]].reshape(-1, block) * e4m3_decode(q["c1_fp8"]).astype(np.float32)[:, None])'
+     '.astype(np.float32) * np.repeat(q["s2"], q["dq_block"])[: q["c1_fp8"].size][:, None]',
+     "test_oracle_dequant_rounding.py"),
+    ("quantize.py", "return bf16_rn(v.reshape(-1)).reshape(N, K)", "return v.reshape(N, K)", "test_oracle_dequant_rounding.py"),
+    ("quantize.py", "v = (d * sc[..., None]).astype(np.float32)",
+     'v = (d.astype(np.float16) * q["scale"][..., None]).astype(np.float32)', "test_oracle_dequant_rounding.py"),
+    ("numerics.py", "r = ((u + np.uint64(0x7FFF) + lsb) & np.uint64(0xFFFF0000)).astype(np.uint32)",
+     "r = (u & np.uint64(0xFFFF0000)).astype(np.uint32)", "test_oracle_dequant_rounding.py"),
 ]
 
 
