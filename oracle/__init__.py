@@ -23,14 +23,17 @@ Modules
   storage   bits-per-parameter and byte accounting of the formats
   lqlora    LQ-LoRA initialisation: alternating truncated SVD and NF-k quantisation
   allocation LQ-LoRA's budgeted (bits, block) choice per matrix (multiple-choice knapsack)
+  loqa      LoQA: gradients of the loss with respect to the INT4 scale and zero point
 
 Parity-pinned: every function is checked in ``tests/test_oracle_*.py`` against
 closed forms, invariants, brute force on tiny inputs, library routines or the
 pages' printed figures (the allocation against exhaustive search and the two
 closed-form ends of the budget; the initialisation against constructed SVDs, an
-exactly low-rank matrix and its zero-iteration case).  The pages print no worked
-example for the two LQ-LoRA parts, so what they pin is the reading of the
-abstract that these modules state, not numbers from the pages.
+exactly low-rank matrix and its zero-iteration case; the LoQA gradients against
+finite differences of the loss, brute force and the pooled-adapter identity of a
+zero-point shift).  The pages print no worked example for the two LQ-LoRA parts
+or for LoQA, so what they pin is the reading of the abstract that these modules
+state, not numbers from the pages.
 """
 
-from . import numerics, codebook, quantize, layer, storage, lqlora, allocation  # noqa: F401
+from . import numerics, codebook, quantize, layer, storage, lqlora, allocation, loqa  # noqa: F401

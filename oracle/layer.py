@@ -42,23 +42,24 @@ def unpool(G: np.ndarray, L: int) -> np.ndarray:
     return np.repeat(f64(G), L, axis=1) / L
 
 
-def forward(X, Wdq, A, B, s: float, L: Optional[int] = None) -> Dict[str, np.ndarray]:
-    X, Wdq, A, B = f64(X), f64(Wdq), f64(A), f64(B)
-    P = pool(X, L) if L else X
+def forward(X, Wdq, A, B, s: float, L: Optional[int] = None, dtype=np.float64) -> Dict[str, np.ndarray]:
+    """dtype: the precision of the products (fp64 for parity; the timed CPU baseline passes fp32)."""
+    X, Wdq, A, B = (np.asarray(a, dtype) for a in (X, Wdq, A, B))
+    P = (pool(X, L).astype(dtype) if L else X)
     T = P @ A.T
     Y = X @ Wdq.T + s * (T @ B.T)
     return {"Y": Y, "T": T}
 
 
-def backward(dY, X, Wdq, A, B, s: float, L: Optional[int] = None) -> Dict[str, np.ndarray]:
-    dY, X, Wdq, A, B = f64(dY), f64(X), f64(Wdq), f64(A), f64(B)
-    P = pool(X, L) if L else X
+def backward(dY, X, Wdq, A, B, s: float, L: Optional[int] = None, dtype=np.float64) -> Dict[str, np.ndarray]:
+    dY, X, Wdq, A, B = (np.asarray(a, dtype) for a in (dY, X, Wdq, A, B))
+    P = (pool(X, L).astype(dtype) if L else X)
     T = P @ A.T
     dT = s * (dY @ B)
     dB = s * (dY.T @ T)
     dA = dT.T @ P
     dTA = dT @ A
-    dX = dY @ Wdq + (unpool(dTA, L) if L else dTA)
+    dX = dY @ Wdq + (unpool(dTA, L).astype(dtype) if L else dTA)
     return {"dX": dX, "dA": dA, "dB": dB, "dT": dT, "T": T}
 
 

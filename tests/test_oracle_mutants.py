@@ -14,8 +14,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 MUTANTS = [
     ("layer.py", "dB = s * (dY.T @ T)", "dB = (dY.T @ T)", "test_oracle_layer.py"),
-    ("layer.py", "dX = dY @ Wdq + (unpool(dTA, L) if L else dTA)",
-     "dX = dY @ Wdq.T + (unpool(dTA, L) if L else dTA)", "test_oracle_layer.py"),
+    ("layer.py", "dX = dY @ Wdq + (unpool(dTA, L).astype(dtype) if L else dTA)",
+     "dX = dY @ Wdq.T + (unpool(dTA, L).astype(dtype) if L else dTA)", "test_oracle_layer.py"),
     ("layer.py", "dG = dH * U * sig * (1.0 + G * (1.0 - sig))", "dG = dH * U * sig * (1.0 - G * (1.0 - sig))",
      "test_oracle_layer.py"),
     ("layer.py", "return X.reshape(M, K // L, L).mean(axis=-1)", "return X.reshape(M, L, K // L).mean(axis=1)",
@@ -46,6 +46,11 @@ MUTANTS = [
      'v = (d.astype(np.float16) * q["scale"][..., None]).astype(np.float32)', "test_oracle_dequant_rounding.py"),
     ("numerics.py", "r = ((u + np.uint64(0x7FFF) + lsb) & np.uint64(0xFFFF0000)).astype(np.uint32)",
      "r = (u & np.uint64(0xFFFF0000)).astype(np.uint32)", "test_oracle_dequant_rounding.py"),
+    # LoQA's scale and zero-point gradients (pinned by finite differences and brute force)
+    ("loqa.py", "dzero = -np.asarray(scale, np.float64) * Gg.sum(axis=-1)", "dzero = np.asarray(scale, np.float64) * Gg.sum(axis=-1)",
+     "test_oracle_loqa.py"),
+    ("loqa.py", "dscale = (Gg * (cg - z[..., None])).sum(axis=-1)", "dscale = (Gg * cg).sum(axis=-1)", "test_oracle_loqa.py"),
+    ("loqa.py", "Gg = G.reshape(N, K // L, L)", "Gg = G.reshape(N, L, K // L).transpose(0, 2, 1)", "test_oracle_loqa.py"),
 ]
 
 
