@@ -243,6 +243,20 @@ QLR_API int qlr_lora_down(const qlr_qweight* w, const uint16_t* X, int64_t M, co
 QLR_API int qlr_forward_base(const qlr_qweight* w, const uint16_t* X, int64_t M, const uint16_t* B, int r,
                              const uint16_t* T_save, uint16_t* Y, int32_t* status, void* stream);
 
+/*
+ * The MLP block's up projection with the SwiGLU gate fused into its epilogue (the LLaMA-7B-shaped MLP:
+ * H = silu(G) * U between the gate/up and down projections).  Same arguments as qlr_forward_base for the up
+ * projection, plus the gate projection's output G (bf16 [M, N], from qlr_forward_base of the gate weight):
+ *   U = bf16( X dequant(W_up)^T + T_up B_up^T )      written to U  [M, N]
+ *   H = bf16( silu(G) * U ),  silu(g) = g / (1 + exp(-g)), fp32 arithmetic on the bf16 G and U
+ * in one launch, so U is never read back.  The SwiGLU arithmetic is the same as qlr_swiglu_forward's, so the
+ * results are bit-identical to qlr_forward_base followed by qlr_swiglu_forward.  Decode-sized calls (the
+ * decode kernel's conditions) run the two steps as two launches.  N a multiple of 8.
+ */
+QLR_API int qlr_forward_swiglu(const qlr_qweight* w_up, const uint16_t* X, int64_t M, const uint16_t* B_up, int r,
+                               const uint16_t* T_up, const uint16_t* G, uint16_t* U, uint16_t* H, int32_t* status,
+                               void* stream);
+
 /* Number of kernels this library has launched in this process (all devices, all streams). */
 QLR_API uint64_t qlr_launch_count(void);
 
@@ -261,6 +275,22 @@ QLR_API size_t qlr_backward_lora_workspace_bytes(const qlr_qweight* w, int64_t M
 QLR_API int qlr_backward_lora(const qlr_qweight* w, const uint16_t* X, const uint16_t* dY, const uint16_t* T_save,
                       const uint16_t* B, int64_t M, int r, float s, int pooled, float* dA, float* dB,
                       uint16_t* dT_out, void* workspace, size_t workspace_bytes, int32_t* status, void* stream);
+
+/*
+ * The two halves of qlr_backward_lora, for callers that overlap them with the input gradient: dT (which
+ * qlr_backward_dx needs) first, then dB and dA (which nothing in the step waits for) on a second stream that
+ * waits for dT, beside qlr_backward_dx on the first.  Same arithmetic and results as qlr_backward_lora; each
+ * takes the workspace of qlr_backward_lora_workspace_bytes (calls that may run at the same time need
+ * separate workspaces).
+ *   qlr_backward_lora_dT     dT = bf16( s dY B )                              (no pooled variant is needed)
+ *   qlr_backward_lora_dAdB   dB = dY^T T_save,  dA = dT^T P(X)   from the dT of qlr_backward_lora_dT
+ */
+QLR_API int qlr_backward_lora_dT(const qlr_qweight* w, const uint16_t* dY, int64_t M, const uint16_t* B, int r,
+                                 float s, uint16_t* dT_out, void* workspace, size_t workspace_bytes, int32_t* status,
+                                 void* stream);
+QLR_API int qlr_backward_lora_dAdB(const qlr_qweight* w, const uint16_t* X, const uint16_t* dY, const uint16_t* T_save,
+                                   const uint16_t* dT, int64_t M, int r, int pooled, float* dA, float* dB,
+                                   void* workspace, size_t workspace_bytes, int32_t* status, void* stream);
 
 /* Size in bytes of the scratch array built into the library for qlr_backward_lora_noalloc: one per
  * GPU that loads the library, held until the process exits. */
@@ -287,6 +317,22 @@ QLR_API int qlr_backward_lora_noalloc(const qlr_qweight* w, const uint16_t* X, c
                                       void* stream);
 
 /*
+ * LoQA: gradients of the loss with respect to the quantiser's own parameters (LoQA abstract: the scale and
+ * the zero point of a quantised model are fine-tuned, through a form of the quantisation operator that works
+ * with LoRA and equals the original).  Read on the group-wise INT4 format: the dequantised weight is
+ * W[o, k] = scale[o, g] (code[o, k] - zero[o, g]), g = k / group, with the codes frozen; the bf16 rounding of
+ * W is passed straight through.  With G = dY^T X (the gradient with respect to W, never formed in memory):
+ *   dscale[o, g] = sum_{k in g} G[o, k] (code[o, k] - zero[o, g])      fp32 [N, K / group]
+ *   dzero[o, g]  = -scale[o, g] sum_{k in g} G[o, k]                    fp32 [N, K / group]
+ * A tcgen05 GEMM forms 128 x 256 tiles of G in tensor memory (the tokens are the reduction) and its epilogue
+ * reduces them group by group with the codes.  Each result is one fixed-order sum (deterministic).
+ *   w       QLR_FMT_INT4G, group 32, 64 or 128;  N a multiple of 8;  K a multiple of the group.
+ *   X bf16 [M, K], dY bf16 [M, N] (device, row-major, 16-byte aligned);  M = 0 writes zeros.
+ */
+QLR_API int qlr_loqa_grad(const qlr_qweight* w, const uint16_t* X, const uint16_t* dY, int64_t M, float* dscale,
+                          float* dzero, int32_t* status, void* stream);
+
+/*
  * Input gradient through the frozen quantised weight (QLoRA explainer, "The contribution":
  * backpropagate through the frozen 4-bit weights into the adapters):
  *   dX = bf16( dY dequant(W) + P^T(dT A) )  [M, K]
@@ -299,6 +345,18 @@ QLR_API size_t qlr_backward_dx_workspace_bytes(const qlr_qweight* w, int64_t M, 
 QLR_API int qlr_backward_dx(const qlr_qweight* w, const uint16_t* dY, int64_t M, const uint16_t* A, const uint16_t* dT,
                     int r, int pooled, int accumulate, uint16_t* dX, void* workspace, size_t workspace_bytes,
                     int32_t* status, void* stream);
+
+/*
+ * The MLP block's down-projection input gradient with the SwiGLU backward fused into its epilogue: with
+ * dH = bf16( dY dequant(W_down) + dT A )  [M, K]  (K = the down weight's inputs = the gate/up outputs), which
+ * is never stored, writes
+ *   dG = bf16( dH U sig(G) (1 + G (1 - sig(G))) ),   dU = bf16( dH silu(G) )     bf16 [M, K]
+ * from the forward's G and U.  Same arithmetic as qlr_backward_dx followed by qlr_swiglu_backward, so the
+ * results are bit-identical to that pair; dH's write and read are saved.  No pooled adapter; K a multiple of 8.
+ */
+QLR_API int qlr_backward_dx_swiglu(const qlr_qweight* w_down, const uint16_t* dY, int64_t M, const uint16_t* A,
+                                   const uint16_t* dT, int r, const uint16_t* G, const uint16_t* U, uint16_t* dG,
+                                   uint16_t* dU, int32_t* status, void* stream);
 
 /*
  * SwiGLU between the gate/up and down projections of an MLP block (the LLaMA-7B-shaped

@@ -388,8 +388,13 @@ int qlr_lora_down(const qlr_qweight* w, const uint16_t* X, int64_t M, const uint
   return run_adapter(g, r, ADAPTER_ROWS_BF16, s, 1, T_save, r, ws, stat, st);
 }
 
-int qlr_forward_base(const qlr_qweight* w, const uint16_t* X, int64_t M, const uint16_t* B, int r,
-                     const uint16_t* T_save, uint16_t* Y, int32_t* status, void* stream) {
+namespace {
+
+// Y = X dequant(W)^T + T_save B^T with the given epilogue (EPI_SWIGLU_FWD: Y is U and H = silu(G) U is
+// written beside it; a decode-sized call runs the decode kernel and then the standalone SwiGLU kernel).
+int forward_base_impl(const qlr_qweight* w, const uint16_t* X, int64_t M, const uint16_t* B, int r,
+                      const uint16_t* T_save, uint16_t* Y, int epi, const uint16_t* G, uint16_t* H, int32_t* status,
+                      void* stream) {
   int rc = check_gemm_weight(w);
   if (rc) return rc;
   if ((rc = check_rank(r))) return rc;
@@ -402,7 +407,10 @@ int qlr_forward_base(const qlr_qweight* w, const uint16_t* X, int64_t M, const u
   int32_t* stat = status_or_sink(status);
   const int64_t N = w->N, K = w->K;
   // a few tokens of a 4-bit NF weight: the HBM-bound decode kernel
-  if (decode_supported(w, M)) return cuda_rc(launch_decode(w, X, M, B, r, T_save, Y, stat, st));
+  if (decode_supported(w, M)) {
+    if ((rc = cuda_rc(launch_decode(w, X, M, B, r, T_save, Y, stat, st)))) return rc;
+    return epi == EPI_SWIGLU_FWD ? cuda_rc(launch_swiglu_fwd(G, Y, H, M * N, st)) : QLR_OK;
+  }
   // Y = X dequant(W)^T + T_save B^T: fused dequant + tcgen05, computed as Y^T tiles (W rows on TMEM lanes)
   const int tok = M >= 512 ? 512 : (M >= 192 ? 256 : 64);  // tokens per tile
   const int bn_tok = tok == 512 ? 256 : tok;                // tokens per activation stage
@@ -430,6 +438,9 @@ int qlr_forward_base(const qlr_qweight* w, const uint16_t* X, int64_t M, const u
   p.out = Y;
   p.ldo = N;
   p.accumulate = 0;
+  p.epi = epi;
+  p.aux_g = G;
+  p.aux_out = H;
   p.dq = dq_params(w);
   p.tail_a = B;
   p.tail_a_rows = N;
@@ -437,6 +448,22 @@ int qlr_forward_base(const qlr_qweight* w, const uint16_t* X, int64_t M, const u
   p.status = stat;
   p.wait_cycles = wait_limit_cycles();
   return cuda_rc(launch_gemm(A_DQ_K, B_TMA_K, tok, OUT_BF16_T, 0, p, maps, st));
+}
+
+}  // namespace
+
+int qlr_forward_base(const qlr_qweight* w, const uint16_t* X, int64_t M, const uint16_t* B, int r,
+                     const uint16_t* T_save, uint16_t* Y, int32_t* status, void* stream) {
+  return forward_base_impl(w, X, M, B, r, T_save, Y, EPI_STORE, nullptr, nullptr, status, stream);
+}
+
+int qlr_forward_swiglu(const qlr_qweight* w_up, const uint16_t* X, int64_t M, const uint16_t* B_up, int r,
+                       const uint16_t* T_up, const uint16_t* G, uint16_t* U, uint16_t* H, int32_t* status,
+                       void* stream) {
+  if (M > 0 && (!G || !H)) return QLR_ERR_ARG;
+  if (!aligned16(G) || !aligned16(H)) return QLR_ERR_ALIGN;
+  if (w_up && w_up->N % 8) return QLR_ERR_SHAPE;
+  return forward_base_impl(w_up, X, M, B_up, r, T_up, U, EPI_SWIGLU_FWD, G, H, status, stream);
 }
 
 int qlr_forward(const qlr_qweight* w, const uint16_t* X, int64_t M, const uint16_t* A, const uint16_t* B, int r,
@@ -465,40 +492,41 @@ size_t qlr_backward_lora_workspace_bytes(const qlr_qweight* w, int64_t M, int r,
   return a > b ? (a > c ? a : c) : (b > c ? b : c);
 }
 
-int qlr_backward_lora(const qlr_qweight* w, const uint16_t* X, const uint16_t* dY, const uint16_t* T_save,
-                      const uint16_t* B, int64_t M, int r, float s, int pooled, float* dA, float* dB,
-                      uint16_t* dT_out, void* workspace, size_t workspace_bytes, int32_t* status, void* stream) {
+namespace {
+
+// Shared validation of the adapter-gradient calls; fills *need with the workspace size.
+int check_backward_lora(const qlr_qweight* w, int64_t M, int r, int pooled, const void* workspace,
+                        size_t workspace_bytes) {
   int rc = check_gemm_weight(w);
   if (rc) return rc;
   if ((rc = check_rank(r))) return rc;
   if (M < 0) return QLR_ERR_ARG;
-  if (!dA || !dB) return QLR_ERR_ARG;
-  if (M > 0 && (!X || !dY || !T_save || !B || !dT_out)) return QLR_ERR_ARG;
-  if (!aligned16(X) || !aligned16(dY) || !aligned16(T_save) || !aligned16(B) || !aligned16(dA) || !aligned16(dB) ||
-      !aligned16(dT_out))
-    return QLR_ERR_ALIGN;
   if (pooled && w->fmt != QLR_FMT_INT4G) return QLR_ERR_UNSUPPORTED;
   if (pooled && (w->K / w->group) % 8) return QLR_ERR_SHAPE;
-  cudaStream_t st = as_stream(stream);
-  const int64_t N = w->N, K = w->K;
-  const int64_t Ka = pooled ? K / w->group : K;
-  if (M == 0) {
-    // no tokens: the gradients are zero
-    if (cudaMemsetAsync(dA, 0, size_t(r) * Ka * 4, st) != cudaSuccess) return QLR_ERR_CUDA;
-    return cuda_rc(cudaMemsetAsync(dB, 0, size_t(N) * r * 4, st));
-  }
   if (M > (int64_t(1) << 30)) return QLR_ERR_SHAPE;
+  if (M == 0) return QLR_OK;
   const size_t need = qlr_backward_lora_workspace_bytes(w, M, r, pooled);
   if (need && (!workspace || workspace_bytes < need)) return QLR_ERR_WORKSPACE;
   if (need && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return QLR_ERR_ALIGN;
+  return QLR_OK;
+}
+
+int run_dT(const qlr_qweight* w, const uint16_t* dY, int64_t M, const uint16_t* B, int r, float s, uint16_t* dT_out,
+           void* workspace, int32_t* status, cudaStream_t st) {
+  // dT = bf16(s dY B)
+  AdapterGemm g{A_TMA_K, B_TMA_MN, adapter_bn(r), M, w->N, dY, M, w->N, B, w->N, r};
+  return run_adapter(g, r, ADAPTER_ROWS_BF16, s, 1, dT_out, r, static_cast<uint8_t*>(workspace),
+                     status_or_sink(status), st);
+}
+
+int run_dAdB(const qlr_qweight* w, const uint16_t* X, const uint16_t* dY, const uint16_t* T_save, const uint16_t* dT,
+             int64_t M, int r, int pooled, float* dA, float* dB, void* workspace, int32_t* status, cudaStream_t st) {
+  const int64_t N = w->N, K = w->K;
+  const int64_t Ka = pooled ? K / w->group : K;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   int32_t* stat = status_or_sink(status);
   const int bn = adapter_bn(r);
-  // dT = bf16(s dY B)
-  {
-    AdapterGemm g{A_TMA_K, B_TMA_MN, bn, M, N, dY, M, N, B, N, r};
-    if ((rc = run_adapter(g, r, ADAPTER_ROWS_BF16, s, 1, dT_out, r, ws, stat, st))) return rc;
-  }
+  int rc;
   // dB = dY^T T_save  (rows of D are output features, reduction over tokens)
   {
     AdapterGemm g{A_TMA_MN, B_TMA_MN, bn, N, M, dY, M, N, T_save, M, r};
@@ -506,13 +534,58 @@ int qlr_backward_lora(const qlr_qweight* w, const uint16_t* X, const uint16_t* d
   }
   // pooled adapter: dA = dT^T P(X) from the group means of X
   if (pooled && pooled_adapter_supported(K, w->group, r))
-    return cuda_rc(launch_pooled_dA(X, M, K, w->group, dT_out, r, dA, reinterpret_cast<float*>(ws), st));
+    return cuda_rc(launch_pooled_dA(X, M, K, w->group, dT, r, dA, reinterpret_cast<float*>(ws), st));
   // dA^T = X^T dT over all K inputs; the pooled adapter sums each group of L inputs and divides by L
-  {
-    AdapterGemm g{A_TMA_MN, B_TMA_MN, bn, K, M, X, M, K, dT_out, M, r};
-    if ((rc = run_adapter(g, r, ADAPTER_COLS_F32, 1.0f, pooled ? w->group : 1, dA, Ka, ws, stat, st))) return rc;
-  }
-  return QLR_OK;
+  AdapterGemm g{A_TMA_MN, B_TMA_MN, bn, K, M, X, M, K, dT, M, r};
+  return run_adapter(g, r, ADAPTER_COLS_F32, 1.0f, pooled ? w->group : 1, dA, Ka, ws, stat, st);
+}
+
+int zero_grads(const qlr_qweight* w, int r, int pooled, float* dA, float* dB, cudaStream_t st) {
+  const int64_t Ka = pooled ? w->K / w->group : w->K;
+  if (cudaMemsetAsync(dA, 0, size_t(r) * Ka * 4, st) != cudaSuccess) return QLR_ERR_CUDA;
+  return cuda_rc(cudaMemsetAsync(dB, 0, size_t(w->N) * r * 4, st));
+}
+
+}  // namespace
+
+int qlr_backward_lora(const qlr_qweight* w, const uint16_t* X, const uint16_t* dY, const uint16_t* T_save,
+                      const uint16_t* B, int64_t M, int r, float s, int pooled, float* dA, float* dB,
+                      uint16_t* dT_out, void* workspace, size_t workspace_bytes, int32_t* status, void* stream) {
+  int rc = check_backward_lora(w, M, r, pooled, workspace, workspace_bytes);
+  if (rc) return rc;
+  if (!dA || !dB) return QLR_ERR_ARG;
+  if (M > 0 && (!X || !dY || !T_save || !B || !dT_out)) return QLR_ERR_ARG;
+  if (!aligned16(X) || !aligned16(dY) || !aligned16(T_save) || !aligned16(B) || !aligned16(dA) || !aligned16(dB) ||
+      !aligned16(dT_out))
+    return QLR_ERR_ALIGN;
+  cudaStream_t st = as_stream(stream);
+  if (M == 0) return zero_grads(w, r, pooled, dA, dB, st);  // no tokens: the gradients are zero
+  if ((rc = run_dT(w, dY, M, B, r, s, dT_out, workspace, status, st))) return rc;
+  return run_dAdB(w, X, dY, T_save, dT_out, M, r, pooled, dA, dB, workspace, status, st);
+}
+
+int qlr_backward_lora_dT(const qlr_qweight* w, const uint16_t* dY, int64_t M, const uint16_t* B, int r, float s,
+                         uint16_t* dT_out, void* workspace, size_t workspace_bytes, int32_t* status, void* stream) {
+  int rc = check_backward_lora(w, M, r, 0, workspace, workspace_bytes);
+  if (rc) return rc;
+  if (M == 0) return QLR_OK;
+  if (!dY || !B || !dT_out) return QLR_ERR_ARG;
+  if (!aligned16(dY) || !aligned16(B) || !aligned16(dT_out)) return QLR_ERR_ALIGN;
+  return run_dT(w, dY, M, B, r, s, dT_out, workspace, status, as_stream(stream));
+}
+
+int qlr_backward_lora_dAdB(const qlr_qweight* w, const uint16_t* X, const uint16_t* dY, const uint16_t* T_save,
+                           const uint16_t* dT, int64_t M, int r, int pooled, float* dA, float* dB, void* workspace,
+                           size_t workspace_bytes, int32_t* status, void* stream) {
+  int rc = check_backward_lora(w, M, r, pooled, workspace, workspace_bytes);
+  if (rc) return rc;
+  if (!dA || !dB) return QLR_ERR_ARG;
+  if (M > 0 && (!X || !dY || !T_save || !dT)) return QLR_ERR_ARG;
+  if (!aligned16(X) || !aligned16(dY) || !aligned16(T_save) || !aligned16(dT) || !aligned16(dA) || !aligned16(dB))
+    return QLR_ERR_ALIGN;
+  cudaStream_t st = as_stream(stream);
+  if (M == 0) return zero_grads(w, r, pooled, dA, dB, st);
+  return run_dAdB(w, X, dY, T_save, dT, M, r, pooled, dA, dB, workspace, status, st);
 }
 
 // ---- backward: input gradient --------------------------------------------------------------------
@@ -525,9 +598,13 @@ size_t qlr_backward_dx_workspace_bytes(const qlr_qweight* w, int64_t M, int r, i
   return 0;  // the pooled adapter's group expansion is formed while the tail rows are copied
 }
 
-int qlr_backward_dx(const qlr_qweight* w, const uint16_t* dY, int64_t M, const uint16_t* A, const uint16_t* dT,
-                    int r, int pooled, int accumulate, uint16_t* dX, void* workspace, size_t workspace_bytes,
-                    int32_t* status, void* stream) {
+namespace {
+
+// dX = dY dequant(W) + P^T(dT A) with the given epilogue (EPI_SWIGLU_BWD: dX is dH, never stored; dG and dU
+// are written from G and U).
+int backward_dx_impl(const qlr_qweight* w, const uint16_t* dY, int64_t M, const uint16_t* A, const uint16_t* dT,
+                     int r, int pooled, int accumulate, uint16_t* dX, int epi, const uint16_t* G, const uint16_t* U,
+                     uint16_t* dU, int32_t* status, void* stream) {
   int rc = check_gemm_weight(w);
   if (rc) return rc;
   if ((rc = check_rank(r))) return rc;
@@ -538,8 +615,6 @@ int qlr_backward_dx(const qlr_qweight* w, const uint16_t* dY, int64_t M, const u
   if (pooled && w->fmt != QLR_FMT_INT4G) return QLR_ERR_UNSUPPORTED;
   if (M == 0) return QLR_OK;
   if (M > (int64_t(1) << 30)) return QLR_ERR_SHAPE;
-  (void)workspace;
-  (void)workspace_bytes;
   cudaStream_t st = as_stream(stream);
   int32_t* stat = status_or_sink(status);
   const int64_t N = w->N, K = w->K;
@@ -569,6 +644,10 @@ int qlr_backward_dx(const qlr_qweight* w, const uint16_t* dY, int64_t M, const u
   p.out = dX;
   p.ldo = K;
   p.accumulate = accumulate ? 1 : 0;
+  p.epi = epi;
+  p.aux_g = G;
+  p.aux_u = U;
+  p.aux_out = dU;
   p.dq = dq_params(w);
   p.tail_a = At;
   p.tail_a_rows = r;
@@ -577,6 +656,26 @@ int qlr_backward_dx(const qlr_qweight* w, const uint16_t* dY, int64_t M, const u
   p.status = stat;
   p.wait_cycles = wait_limit_cycles();
   return cuda_rc(launch_gemm(A_DQ_MN, B_TMA_K, tok, OUT_BF16_T, 1, p, maps, st));
+}
+
+}  // namespace
+
+int qlr_backward_dx(const qlr_qweight* w, const uint16_t* dY, int64_t M, const uint16_t* A, const uint16_t* dT,
+                    int r, int pooled, int accumulate, uint16_t* dX, void* workspace, size_t workspace_bytes,
+                    int32_t* status, void* stream) {
+  (void)workspace;
+  (void)workspace_bytes;
+  return backward_dx_impl(w, dY, M, A, dT, r, pooled, accumulate, dX, EPI_STORE, nullptr, nullptr, nullptr, status,
+                          stream);
+}
+
+int qlr_backward_dx_swiglu(const qlr_qweight* w_down, const uint16_t* dY, int64_t M, const uint16_t* A,
+                           const uint16_t* dT, int r, const uint16_t* G, const uint16_t* U, uint16_t* dG, uint16_t* dU,
+                           int32_t* status, void* stream) {
+  if (M > 0 && (!G || !U || !dU)) return QLR_ERR_ARG;
+  if (!aligned16(G) || !aligned16(U) || !aligned16(dU)) return QLR_ERR_ALIGN;
+  if (w_down && w_down->K % 8) return QLR_ERR_SHAPE;
+  return backward_dx_impl(w_down, dY, M, A, dT, r, 0, 0, dG, EPI_SWIGLU_BWD, G, U, dU, status, stream);
 }
 
 // ---- SwiGLU ---------------------------------------------------------------------------------------

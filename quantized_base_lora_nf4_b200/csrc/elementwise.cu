@@ -6,6 +6,7 @@
 #include "common.cuh"
 #include "gemm.cuh"
 #include "ptx.cuh"
+#include "swiglu.cuh"
 
 namespace qlr {
 
@@ -13,8 +14,6 @@ namespace {
 
 __device__ __forceinline__ float lo_f(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float hi_f(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
-
-__device__ __forceinline__ float sigmoidf_(float g) { return 1.0f / (1.0f + expf(-g)); }
 
 __global__ void swiglu_fwd_kernel(const uint4* __restrict__ G, const uint4* __restrict__ U, uint4* __restrict__ H,
                                   int64_t n8) {
@@ -27,10 +26,7 @@ __global__ void swiglu_fwd_kernel(const uint4* __restrict__ G, const uint4* __re
     uint32_t hv[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const float g0 = lo_f(gv[j]), g1 = hi_f(gv[j]);
-      const float h0 = g0 * sigmoidf_(g0) * lo_f(uv[j]);
-      const float h1 = g1 * sigmoidf_(g1) * hi_f(uv[j]);
-      hv[j] = pack_bf16x2_rn(h0, h1);
+      hv[j] = pack_bf16x2_rn(swiglu_h(lo_f(gv[j]), lo_f(uv[j])), swiglu_h(hi_f(gv[j]), hi_f(uv[j])));
     }
     H[i] = make_uint4(hv[0], hv[1], hv[2], hv[3]);
   }
@@ -53,9 +49,7 @@ __global__ void swiglu_bwd_kernel(const uint4* __restrict__ dH, const uint4* __r
         const float dh = h ? hi_f(dv[j]) : lo_f(dv[j]);
         const float gg = h ? hi_f(gv[j]) : lo_f(gv[j]);
         const float uu = h ? hi_f(uv[j]) : lo_f(uv[j]);
-        const float sg = sigmoidf_(gg);
-        rg[h] = dh * uu * sg * (1.0f + gg * (1.0f - sg));
-        ru[h] = dh * gg * sg;
+        swiglu_grads(dh, gg, uu, rg[h], ru[h]);
       }
       og[j] = pack_bf16x2_rn(rg[0], rg[1]);
       ou[j] = pack_bf16x2_rn(ru[0], ru[1]);

@@ -8,6 +8,7 @@
 
 #include "gemm.cuh"
 #include "ptx.cuh"
+#include "swiglu.cuh"
 
 namespace qlr {
 namespace eng {
@@ -209,8 +210,39 @@ __device__ __forceinline__ void store_chunk_bf16_t(const uint32_t (&v)[32], uint
     const int ocol = drow0 + part * 8;        // output column (D row)
     if (orow < p.Nn && ocol < p.Mm) {
       const uint4 val = *reinterpret_cast<const uint4*>(stg + jj * 32 + part * 8);
-      uint16_t* dst = static_cast<uint16_t*>(p.out) + static_cast<int64_t>(orow) * p.ldo + ocol;
-      *reinterpret_cast<uint4*>(dst) = val;
+      const int64_t off = static_cast<int64_t>(orow) * p.ldo + ocol;
+      uint16_t* dst = static_cast<uint16_t*>(p.out) + off;
+      if (p.epi == EPI_STORE) {
+        *reinterpret_cast<uint4*>(dst) = val;
+      } else if (p.epi == EPI_SWIGLU_FWD) {  // val = U; H = silu(G) U
+        *reinterpret_cast<uint4*>(dst) = val;
+        const uint4 g4 = *reinterpret_cast<const uint4*>(p.aux_g + off);
+        const uint32_t gv[4] = {g4.x, g4.y, g4.z, g4.w}, uv[4] = {val.x, val.y, val.z, val.w};
+        uint32_t hv[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          hv[e] = pack_bf16x2_rn(swiglu_h(bf16_bits_to_f32(gv[e] & 0xFFFFu), bf16_bits_to_f32(uv[e] & 0xFFFFu)),
+                                 swiglu_h(bf16_bits_to_f32(gv[e] >> 16), bf16_bits_to_f32(uv[e] >> 16)));
+        *reinterpret_cast<uint4*>(p.aux_out + off) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+      } else {  // val = dH (bf16, as a stored dH would be); dG to out, dU to aux_out
+        const uint4 g4 = *reinterpret_cast<const uint4*>(p.aux_g + off);
+        const uint4 u4 = *reinterpret_cast<const uint4*>(p.aux_u + off);
+        const uint32_t dv[4] = {val.x, val.y, val.z, val.w}, gv[4] = {g4.x, g4.y, g4.z, g4.w},
+                       uv[4] = {u4.x, u4.y, u4.z, u4.w};
+        uint32_t og[4], ou[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float g0, u0, g1, u1;
+          swiglu_grads(bf16_bits_to_f32(dv[e] & 0xFFFFu), bf16_bits_to_f32(gv[e] & 0xFFFFu),
+                       bf16_bits_to_f32(uv[e] & 0xFFFFu), g0, u0);
+          swiglu_grads(bf16_bits_to_f32(dv[e] >> 16), bf16_bits_to_f32(gv[e] >> 16), bf16_bits_to_f32(uv[e] >> 16), g1,
+                       u1);
+          og[e] = pack_bf16x2_rn(g0, g1);
+          ou[e] = pack_bf16x2_rn(u0, u1);
+        }
+        *reinterpret_cast<uint4*>(dst) = make_uint4(og[0], og[1], og[2], og[3]);
+        *reinterpret_cast<uint4*>(p.aux_out + off) = make_uint4(ou[0], ou[1], ou[2], ou[3]);
+      }
     }
   }
   __syncwarp();

@@ -16,6 +16,7 @@ enum ASrc : int {
 };
 enum BSrc : int { B_TMA_K = 0, B_TMA_MN = 1 };
 enum OutMode : int { OUT_BF16_T = 0, OUT_F32_D = 1 };
+enum EpiMode : int { EPI_STORE = 0, EPI_SWIGLU_FWD = 1, EPI_SWIGLU_BWD = 2 };
 
 struct DqParams {
   int fmt, bits, block, dq_block, group;
@@ -44,6 +45,13 @@ struct GemmParams {
   void* out;             // OUT_BF16_T: bf16 [Nn, ldo] receiving D^T; OUT_F32_D: fp32 [splits][m_tiles*128][ldo]
   int64_t ldo;
   int accumulate;        // OUT_BF16_T: add the previous contents of out
+  // epilogue: EPI_STORE writes D^T to out; EPI_SWIGLU_FWD writes it (U) to out and H = silu(G) U to aux_out
+  // (G read from aux_g); EPI_SWIGLU_BWD treats it as dH (never stored) and writes dG to out, dU to aux_out
+  // (G, U read from aux_g, aux_u).  Every auxiliary tensor has the layout of out.
+  int epi;
+  const uint16_t* aux_g;
+  const uint16_t* aux_u;
+  uint16_t* aux_out;
   DqParams dq;
   // codes ring of the fused kernel: one TMA box per slot covering code_steps main steps (2 for 3-bit
   // codes along K, whose 24-byte runs are not a legal box width), 2^code_slots_log2 slots of

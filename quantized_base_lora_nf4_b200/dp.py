@@ -40,16 +40,19 @@ class GradBucket:
 
     def start(self, group: Optional[dist.ProcessGroup] = None, stream=None):
         """Copy the gradients in and start the SUM all-reduce without waiting for it (None when there
-        is nothing to exchange).  The copies and, with NCCL, the collective are ordered on torch's
-        current stream; `stream` names the CUDA stream the backward ran on when that is another one
-        (the library's calls take an explicit stream), and the current stream then waits for it before
-        the copies, so the exchange never reads gradients the backward has not finished writing."""
+        is nothing to exchange).  The copies and, with NCCL, the collective are ordered after the work
+        already issued on `stream`: the CUDA stream the gradients were computed on (the library's calls
+        take an explicit stream), torch's current stream when None.  They are issued on that stream, so
+        the exchange never reads gradients the backward has not finished writing and does not hold up
+        the other streams."""
         if not dist.is_initialized() or dist.get_world_size(group) == 1:
             return None
         if stream is not None and self.flat.is_cuda:
-            cur = torch.cuda.current_stream(self.flat.device)
-            if stream != cur:
-                cur.wait_stream(stream)
+            with torch.cuda.stream(stream):
+                return self._start(group)
+        return self._start(group)
+
+    def _start(self, group):
         off = 0
         for g, n in zip(self.grads, self.sizes):
             self.flat[off:off + n].copy_(g.reshape(-1))

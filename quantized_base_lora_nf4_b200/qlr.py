@@ -31,7 +31,8 @@ EXPORTED = (
     "qlr_backward_dx", "qlr_swiglu_forward", "qlr_swiglu_backward", "qlr_device_sm_count", "qlr_lora_down",
     "qlr_forward_base", "qlr_launch_count", "qlr_backward_lora_noalloc", "qlr_lqlora_init_workspace_bytes",
     "qlr_lqlora_init", "qlr_nf_quant_error_workspace_bytes", "qlr_nf_quant_error", "qlr_lqlora_allocate",
-    "qlr_set_wait_limit", "qlr_wait_selftest",
+    "qlr_set_wait_limit", "qlr_wait_selftest", "qlr_loqa_grad", "qlr_forward_swiglu", "qlr_backward_dx_swiglu",
+    "qlr_backward_lora_dT", "qlr_backward_lora_dAdB",
 )
 
 
@@ -90,6 +91,11 @@ def lib() -> ctypes.CDLL:
         "qlr_lqlora_allocate": (I, [P, P, I, I, I64, I64, P, P]),
         "qlr_set_wait_limit": (ctypes.c_longlong, [ctypes.c_longlong]),
         "qlr_wait_selftest": (I, [P, P]),
+        "qlr_loqa_grad": (I, [QP, P, P, I64, P, P, P, P]),
+        "qlr_forward_swiglu": (I, [QP, P, I64, P, I, P, P, P, P, P, P]),
+        "qlr_backward_dx_swiglu": (I, [QP, P, I64, P, P, I, P, P, P, P, P, P]),
+        "qlr_backward_lora_dT": (I, [QP, P, I64, P, I, F, P, P, SZ, P, P]),
+        "qlr_backward_lora_dAdB": (I, [QP, P, P, P, P, I64, I, I, P, P, P, SZ, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -322,6 +328,34 @@ def forward_base(q: QWeight, X: torch.Tensor, B: torch.Tensor, T_save: torch.Ten
     return Y
 
 
+def forward_swiglu(q_up: QWeight, X: torch.Tensor, B_up: torch.Tensor, T_up: torch.Tensor, G: torch.Tensor,
+                   U: Optional[torch.Tensor] = None, H: Optional[torch.Tensor] = None,
+                   status: Optional[torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Up projection U and the SwiGLU H = silu(G) * U in one launch (G: the gate projection's output)."""
+    M = X.shape[0]
+    if U is None:
+        U = torch.empty((M, q_up.N), dtype=torch.bfloat16, device=X.device)
+    if H is None:
+        H = torch.empty_like(U)
+    _check(lib().qlr_forward_swiglu(q_up.ref(), _ptr(X), M, _ptr(B_up), B_up.shape[1], _ptr(T_up), _ptr(G), _ptr(U),
+                                    _ptr(H), _ptr(status), _stream(stream)), "qlr_forward_swiglu")
+    return U, H
+
+
+def backward_dx_swiglu(q_down: QWeight, dY: torch.Tensor, A: torch.Tensor, dT: torch.Tensor, G: torch.Tensor,
+                       U: torch.Tensor, dG: Optional[torch.Tensor] = None, dU: Optional[torch.Tensor] = None,
+                       status: Optional[torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """The down projection's input gradient dH turned into (dG, dU) in its epilogue (dH never stored)."""
+    M = dY.shape[0]
+    if dG is None:
+        dG = torch.empty((M, q_down.K), dtype=torch.bfloat16, device=dY.device)
+    if dU is None:
+        dU = torch.empty_like(dG)
+    _check(lib().qlr_backward_dx_swiglu(q_down.ref(), _ptr(dY), M, _ptr(A), _ptr(dT), A.shape[0], _ptr(G), _ptr(U),
+                                        _ptr(dG), _ptr(dU), _ptr(status), _stream(stream)), "qlr_backward_dx_swiglu")
+    return dG, dU
+
+
 def launch_count() -> int:
     return int(lib().qlr_launch_count())
 
@@ -358,6 +392,54 @@ def backward_lora(q: QWeight, X: torch.Tensor, dY: torch.Tensor, T_save: torch.T
                                    int(pooled), _ptr(dA), _ptr(dB), _ptr(dT), _ptr(w), w.numel(), _ptr(status),
                                    _stream(stream)), "qlr_backward_lora")
     return dA, dB, dT
+
+
+def loqa_grad(q: QWeight, X: torch.Tensor, dY: torch.Tensor, dscale: Optional[torch.Tensor] = None,
+              dzero: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None, stream=None):
+    """LoQA: gradients of the loss with respect to the INT4 weight's scale and zero point, fp32 [N, K/group]."""
+    G = q.K // q.group
+    dev = X.device
+    if dscale is None:
+        dscale = torch.empty((q.N, G), dtype=torch.float32, device=dev)
+    if dzero is None:
+        dzero = torch.empty((q.N, G), dtype=torch.float32, device=dev)
+    _check(lib().qlr_loqa_grad(q.ref(), _ptr(X), _ptr(dY), X.shape[0], _ptr(dscale), _ptr(dzero), _ptr(status),
+                               _stream(stream)), "qlr_loqa_grad")
+    return dscale, dzero
+
+
+def backward_lora_dT(q: QWeight, dY: torch.Tensor, B: torch.Tensor, s: float, dT: Optional[torch.Tensor] = None,
+                     ws: Optional[Workspace] = None, status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """First half of backward_lora: dT = bf16(s dY B)."""
+    M, r = dY.shape[0], B.shape[1]
+    if dT is None:
+        dT = torch.empty((M, r), dtype=torch.bfloat16, device=dY.device)
+    qs = q.struct()
+    need = lib().qlr_backward_lora_workspace_bytes(ctypes.byref(qs), M, r, 0)
+    w = (ws or Workspace(dY.device)).get(need)
+    _check(lib().qlr_backward_lora_dT(ctypes.byref(qs), _ptr(dY), M, _ptr(B), r, float(s), _ptr(dT), _ptr(w), w.numel(),
+                                      _ptr(status), _stream(stream)), "qlr_backward_lora_dT")
+    return dT
+
+
+def backward_lora_dAdB(q: QWeight, X: torch.Tensor, dY: torch.Tensor, T_save: torch.Tensor, dT: torch.Tensor,
+                       pooled: bool = False, dA: Optional[torch.Tensor] = None, dB: Optional[torch.Tensor] = None,
+                       ws: Optional[Workspace] = None, status: Optional[torch.Tensor] = None, stream=None):
+    """Second half of backward_lora: dB = dY^T T_save and dA = dT^T P(X)."""
+    M, r = X.shape[0], dT.shape[1]
+    dev = X.device
+    Ka = q.K // q.group if pooled else q.K
+    if dA is None:
+        dA = torch.empty((r, Ka), dtype=torch.float32, device=dev)
+    if dB is None:
+        dB = torch.empty((q.N, r), dtype=torch.float32, device=dev)
+    qs = q.struct()
+    need = lib().qlr_backward_lora_workspace_bytes(ctypes.byref(qs), M, r, int(pooled))
+    w = (ws or Workspace(dev)).get(need)
+    _check(lib().qlr_backward_lora_dAdB(ctypes.byref(qs), _ptr(X), _ptr(dY), _ptr(T_save), _ptr(dT), M, r, int(pooled),
+                                        _ptr(dA), _ptr(dB), _ptr(w), w.numel(), _ptr(status), _stream(stream)),
+           "qlr_backward_lora_dAdB")
+    return dA, dB
 
 
 def backward_dx(q: QWeight, dY: torch.Tensor, A: torch.Tensor, dT: torch.Tensor, pooled: bool = False,

@@ -212,3 +212,37 @@ def test_several_tiles_per_cta_without_token_pairs(cuda_lib):
         check_close(host(dX), b["dX"], "dX")
         check_close(host(dA), b["dA"], "dA")
         check_close(host(dB), b["dB"], "dB")
+
+
+@pytest.mark.parametrize("pooled", [False, True])
+def test_split_adapter_backward_on_two_streams_bit_identical(cuda_lib, pooled):
+    """dT on one stream, then dB and dA on a second stream that waits for it (beside the input gradient on the
+    first): the same kernels as backward_lora in one call, so the same bits."""
+    qlr = cuda_lib
+    if pooled:
+        spec = LinearSpec("w", 1024, 2048, "int4g", group=32, r=16, s=1.0, pooled=True)
+    else:
+        spec = LinearSpec("w", 1536, 1024, "nfk", 3, 128, 256, r=64, s=0.25)
+    M = 700
+    t = linear_tensors(spec, M, seed=12)
+    q, _ = quantize_both(qlr, spec, t["W"])
+    X, A, B, dY = bf16_dev(t["X"]), bf16_dev(t["A"]), bf16_dev(t["B"]), bf16_dev(t["dY"])
+    _, T = qlr.forward(q, X, A, B, spec.s, pooled=pooled)
+    dA0, dB0, dT0 = qlr.backward_lora(q, X, dY, T, B, spec.s, pooled=pooled)
+    dX0 = qlr.backward_dx(q, dY, A, dT0, pooled=pooled)
+    main = torch.cuda.current_stream()
+    side = torch.cuda.Stream()
+    st = qlr.new_status(DEV)
+    dT = qlr.backward_lora_dT(q, dY, B, spec.s, status=st)
+    ev = torch.cuda.Event()
+    ev.record(main)
+    side.wait_event(ev)
+    dA, dB = qlr.backward_lora_dAdB(q, X, dY, T, dT, pooled=pooled, status=st, stream=side)
+    dX = qlr.backward_dx(q, dY, A, dT, pooled=pooled, status=st)
+    main.wait_stream(side)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    for a, b in ((dT, dT0), (dX, dX0)):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    for a, b in ((dA, dA0), (dB, dB0)):
+        assert torch.equal(a.view(torch.int32), b.view(torch.int32))

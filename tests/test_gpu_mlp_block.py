@@ -16,7 +16,9 @@ from tests.test_gpu_layer import check_close, quantize_both
 pytestmark = [pytest.mark.gpu, pytest.mark.filterwarnings("ignore::RuntimeWarning")]
 
 
-def run_block(qlr, specs, M, seed, rows=None):
+def run_block(qlr, specs, M, seed, rows=None, fused=False):
+    """The block on the GPU (fused: SwiGLU inside the up projection's and the down projection's input-gradient
+    epilogues) checked against the oracle's chain; returns every device result."""
     gs, us, ds = specs
     ts = [linear_tensors(s, M, seed=seed, matrix_index=i, with_x=(i == 0), with_dy=(i == 2)) for i, s in enumerate(specs)]
     X = ts[0]["X"]
@@ -30,14 +32,21 @@ def run_block(qlr, specs, M, seed, rows=None):
     Tg = qlr.lora_down(qs[0], Xd, A[0], gs.s, status=st)
     Tu = qlr.lora_down(qs[1], Xd, A[1], us.s, status=st)
     G = qlr.forward_base(qs[0], Xd, B[0], Tg, status=st)
-    U = qlr.forward_base(qs[1], Xd, B[1], Tu, status=st)
-    H = qlr.swiglu_forward(G, U)
+    if fused:
+        U, H = qlr.forward_swiglu(qs[1], Xd, B[1], Tu, G, status=st)
+    else:
+        U = qlr.forward_base(qs[1], Xd, B[1], Tu, status=st)
+        H = qlr.swiglu_forward(G, U)
     Td = qlr.lora_down(qs[2], H, A[2], ds.s, status=st)
     Y = qlr.forward_base(qs[2], H, B[2], Td, status=st)
     # backward
     dAd, dBd, dTd = qlr.backward_lora(qs[2], H, dOutd, Td, B[2], ds.s, status=st)
-    dH = qlr.backward_dx(qs[2], dOutd, A[2], dTd, status=st)
-    dG, dU = qlr.swiglu_backward(dH, G, U)
+    if fused:
+        dH = None
+        dG, dU = qlr.backward_dx_swiglu(qs[2], dOutd, A[2], dTd, G, U, status=st)
+    else:
+        dH = qlr.backward_dx(qs[2], dOutd, A[2], dTd, status=st)
+        dG, dU = qlr.swiglu_backward(dH, G, U)
     dAg, dBg, dTg = qlr.backward_lora(qs[0], Xd, dG, Tg, B[0], gs.s, status=st)
     dX = qlr.backward_dx(qs[0], dG, A[0], dTg, status=st)
     dAu, dBu, dTu = qlr.backward_lora(qs[1], Xd, dU, Tu, B[1], us.s, status=st)
@@ -57,13 +66,16 @@ def run_block(qlr, specs, M, seed, rows=None):
     y = OL.forward(h[sel], Wdq[2], ts[2]["A"], ts[2]["B"], ds.s)["Y"]
     check_close(host(Y)[sel], y, "Y")
     check_close(host(H)[sel], h[sel], "H")
-    check_close(host(dH)[sel], bd["dX"][sel], "dH")
+    if dH is not None:
+        check_close(host(dH)[sel], bd["dX"][sel], "dH")
     check_close(host(dG)[sel], dg[sel], "dG")
     check_close(host(dU)[sel], du[sel], "dU")
     check_close(host(dX)[sel], (bg["dX"] + bu["dX"])[sel], "dX = gate's + up's")
     for got, ref, what in ((dAd, bd["dA"], "dA down"), (dBd, bd["dB"], "dB down"), (dAg, bg["dA"], "dA gate"),
                            (dBg, bg["dB"], "dB gate"), (dAu, bu["dA"], "dA up"), (dBu, bu["dB"], "dB up")):
         check_close(host(got), ref, what)
+    return {"Y": Y, "G": G, "U": U, "H": H, "dG": dG, "dU": dU, "dX": dX, "dAd": dAd, "dBd": dBd, "dAg": dAg,
+            "dBg": dBg, "dAu": dAu, "dBu": dBu}
 
 
 def test_mlp_block_reduced_ragged(cuda_lib):
@@ -81,3 +93,26 @@ def test_mlp_block_full_size_sampled_rows(cuda_lib):
     wl = workload("mlp7b")
     rows = np.sort(np.random.default_rng(5).choice(wl.M, 96, replace=False))
     run_block(cuda_lib, wl.linears, wl.M, seed=0, rows=rows)
+
+
+@pytest.mark.parametrize("M", [300, 8])
+def test_mlp_block_swiglu_fused_bit_identical(cuda_lib, M):
+    """The SwiGLU fused into the up projection's epilogue (forward) and the down projection's input-gradient
+    epilogue (backward) gives exactly the bits of the separate SwiGLU kernels (one shared definition of the
+    arithmetic), and matches the oracle.  8 tokens: the up projection runs the decode kernel, then SwiGLU."""
+    s = 16.0 / 64.0
+    # the decode kernel (8 tokens) needs K a multiple of 256: gate/up K = 512, down K = 768
+    specs = (LinearSpec("gate", 768, 512, "nfk", 4, 64, 256, r=16, s=s),
+             LinearSpec("up", 768, 512, "nfk", 4, 64, 256, r=16, s=s),
+             LinearSpec("down", 512, 768, "nfk", 4, 64, 256, r=16, s=s))
+    a = run_block(cuda_lib, specs, M, seed=43)
+    b = run_block(cuda_lib, specs, M, seed=43, fused=True)
+    for k, v in a.items():
+        assert torch.equal(v.view(torch.int16) if v.dtype == torch.bfloat16 else v.view(torch.int32),
+                           b[k].view(torch.int16) if b[k].dtype == torch.bfloat16 else b[k].view(torch.int32)), k
+
+
+def test_mlp_block_full_size_fused(cuda_lib):
+    wl = workload("mlp7b")
+    rows = np.sort(np.random.default_rng(6).choice(wl.M, 64, replace=False))
+    run_block(cuda_lib, wl.linears, wl.M, seed=0, rows=rows, fused=True)
