@@ -488,7 +488,9 @@ def summarize(res, world, peaks, peak_kind):
             "fused_forward": step_fwd, "fused_input_gradient": step_dx,
             "adapter_and_rest": ms - step_fwd - step_dx,
             "fused_forward_TFLOPs": sum(fwd_fl) / (step_fwd / 1e3) / 1e12,
-            "fused_input_gradient_TFLOPs": sum(dx_fl) / (step_dx / 1e3) / 1e12},
+            "fused_input_gradient_TFLOPs": sum(dx_fl) / (step_dx / 1e3) / 1e12,
+            # per launch, in launch order (the MLP block's input gradients run down, gate, up)
+            **({"fused_forward_per_launch": fwd_per, "fused_input_gradient_per_launch": dx_per} if n_lin <= 8 else {})},
         "gpu_launches": res["launches"], "gpu_launches_per_step": res["launches"] / steps,
         "clocks": res["clocks"],
         "e2e": {"value": world * M / (res["e2e_ms_per_step"] / 1e3), "unit": "tokens/s",

@@ -62,7 +62,7 @@ struct FCfg {
   static constexpr int kC = 4096;
   static constexpr int NSA = BN >= 256 ? 3 : 4;
   static constexpr int NSC = 8;
-  static constexpr int kStaging = 4 * 32 * 32 * 2;
+  static constexpr int kStaging = 4 * 32 * 32 * 4;  // per epilogue warp a 32 x 32 fp32 tile
   static constexpr int kFixed = kStaging + 2048;
   static constexpr int kBudget = 227 * 1024 - kFixed - NSA * kA - NSC * kC;
   static constexpr int NSB = (kBudget / kB) > 8 ? 8 : (kBudget / kB);
@@ -178,20 +178,34 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
   tc_fence_after();
   const uint32_t tmem_base = bars->tmem_base;
 
-  const int n_tiles_total = p.m_tiles * p.n_tiles;
+  // Work items: tiles of 128 weight rows x TOK tokens in row-major tile order.  With token pairs, the tiles
+  // from p.full_items on (the last, partial wave of a launch with more tiles than CTAs) are each split
+  // into two items of BN tokens, one per half, so that they spread over more CTAs.
+  const int n_items = p.n_items;
   const int nmain = p.n_main, ntail = p.n_tail, nsteps = nmain + ntail;
-  auto tile_m0 = [&](int tile) { return (tile / p.n_tiles) * 128; };
-  auto tile_n0 = [&](int tile) { return (tile % p.n_tiles) * TOK; };
+  auto item_of = [&](int item, int& m0, int& n0, int& halves) {
+    int tile = item, half = 0;
+    halves = HALVES;
+    if (PAIR && item >= p.full_items) {
+      const int hi = item - p.full_items;
+      tile = p.full_items + (hi >> 1);
+      half = hi & 1;
+      halves = 1;
+    }
+    m0 = (tile / p.n_tiles) * 128;
+    n0 = (tile % p.n_tiles) * TOK + half * BN;
+  };
 
   if (warp == kActWarp) {
     // ------------------------------------------------------------------ activation producer
     if (lane == 0) {
       uint32_t j = 0;
-      for (int tile = blockIdx.x; tile < n_tiles_total && !*abort_flag; tile += gridDim.x) {
-        const int n0 = tile_n0(tile);
+      for (int item = blockIdx.x; item < n_items && !*abort_flag; item += gridDim.x) {
+        int m0, n0, halves;
+        item_of(item, m0, n0, halves);
         bool ok = true;
         for (int ks = 0; ks < nsteps && ok; ++ks) {
-          for (int h = 0; h < HALVES; ++h, ++j) {
+          for (int h = 0; h < halves; ++h, ++j) {
             const int s = j % NSB;
             if (!mbar_wait(&bars->b_empty[s], ((j / NSB) & 1) ^ 1, abort_flag, p.wait_cycles)) { ok = false; break; }
             uint64_t* fb = &bars->b_full[s];
@@ -214,8 +228,9 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
       const int lg = p.code_slots_log2, ncs = 1 << lg, kb = p.code_bits;
       const uint32_t mask = static_cast<uint32_t>(ncs - 1);
       uint32_t jc = 0;  // boxes
-      for (int tile = blockIdx.x; tile < n_tiles_total && !*abort_flag; tile += gridDim.x) {
-        const int m0 = tile_m0(tile);
+      for (int item = blockIdx.x; item < n_items && !*abort_flag; item += gridDim.x) {
+        int m0, n0, halves;
+        item_of(item, m0, n0, halves);
         for (int ks = 0; ks < nmain; ks += p.code_steps, ++jc) {
           const int s = static_cast<int>(jc & mask);
           if (!mbar_wait(&bars->c_empty[s], ((jc >> lg) & 1) ^ 1, abort_flag, p.wait_cycles)) break;
@@ -244,7 +259,9 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
       const uint64_t b_desc0 = smem_desc(smem_u32(ring_b), 16, 1024, kSw128);
       constexpr uint32_t kAk = MN ? (2048 >> 4) : (32 >> 4), kBk = 32 >> 4;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < n_tiles_total && ok; tile += gridDim.x, ++it) {
+      for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++it) {
+        int m0, n0, halves;
+        item_of(item, m0, n0, halves);
         const int acc = PAIR ? 0 : (it & 1);
         const uint32_t acc_par = PAIR ? ((it & 1) ^ 1) : (((it >> 1) & 1) ^ 1);
         if (!mbar_wait(&bars->acc_empty[acc], acc_par, abort_flag, p.wait_cycles)) break;
@@ -258,7 +275,7 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
             const int rem = p.r_tail - (ks - nmain) * 64;
             nsub = rem >= 64 ? 4 : (rem + 15) / 16;
           }
-          for (int h = 0; h < HALVES; ++h, ++jb) {
+          for (int h = 0; h < halves; ++h, ++jb) {
             const int sb = jb % NSB;
             if (!mbar_wait(&bars->b_full[sb], (jb / NSB) & 1, abort_flag, p.wait_cycles)) { ok = false; break; }
             tc_fence_after();
@@ -286,18 +303,19 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
   } else if (warp >= 2 && warp <= 5) {
     // ------------------------------------------------------------------ epilogue
     const int q = warp & 3;
-    uint16_t* stg = reinterpret_cast<uint16_t*>(staging) + q * 32 * 32;
+    float* stg = reinterpret_cast<float*>(staging) + q * 32 * 32;
     int it = 0;
-    for (int tile = blockIdx.x; tile < n_tiles_total; tile += gridDim.x, ++it) {
-      const int m0 = tile_m0(tile), n0 = tile_n0(tile);
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it) {
+      int m0, n0, halves;
+      item_of(item, m0, n0, halves);
       const int acc = PAIR ? 0 : (it & 1);
       const uint32_t acc_par = PAIR ? (it & 1) : ((it >> 1) & 1);
-      const bool got = mbar_wait(&bars->acc_full[acc], acc_par, abort_flag, p.wait_cycles);
+      const bool got = mbar_wait_pause(&bars->acc_full[acc], acc_par, abort_flag, p.wait_cycles);
       __syncwarp();
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
 #pragma unroll 1
-      for (int c = 0; c < TOK / 32; ++c) {  // PAIR: accumulator columns 0..2*BN-1 are tokens n0 .. n0+2*BN-1
+      for (int c = 0; c < halves * BN / 32; ++c) {  // PAIR: accumulator columns 0..2*BN-1 are tokens n0 .. n0+2*BN-1
         uint32_t v[32];
         tmem_ld_32x32b_x32(tmem_base + (PAIR ? 0 : acc * BN) + c * 32 + ((q * 32) << 16), v);
         tmem_ld_wait();
@@ -324,15 +342,21 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
       }
     };
     // cursor over the CTA's step sequence; j counts every step, jc the main (dequantised) ones
-    int tile = blockIdx.x, ks = 0;
-    int tm0 = tile < n_tiles_total ? tile_m0(tile) : 0;
+    int item = blockIdx.x, ks = 0;
+    int tm0 = 0;
+    auto item_m0 = [&](int it_) {
+      int m0, n0, halves;
+      item_of(it_, m0, n0, halves);
+      return m0;
+    };
+    if (item < n_items) tm0 = item_m0(item);
     uint32_t j = 0, jc = 0;
     auto seek = [&]() -> bool {  // advance to the next step with (j & 1) == grp
-      while (tile < n_tiles_total) {
+      while (item < n_items) {
         if (ks >= nsteps) {
-          tile += gridDim.x;
+          item += gridDim.x;
           ks = 0;
-          if (tile < n_tiles_total) tm0 = tile_m0(tile);
+          if (item < n_items) tm0 = item_m0(item);
           continue;
         }
         if (static_cast<int>(j & 1) == grp) return true;
@@ -423,8 +447,8 @@ cudaError_t launch_fused_variant(const GemmParams& p, const GemmMaps& maps, cuda
   auto kern = fused_kernel<A_SRC, BN, PAIR>;
   const cudaError_t attr_err = ensure_max_dynamic_smem(kern, C::kSmem + 1024);
   if (attr_err != cudaSuccess) return attr_err;
-  const int tiles = p.m_tiles * p.n_tiles;
-  const int grid = tiles < device_sm_count() ? tiles : device_sm_count();
+  const int items = p.n_items;
+  const int grid = items < device_sm_count() ? items : device_sm_count();
   return launch_pdl(kern, dim3(grid), dim3(kThreadsFused), C::kSmem + 1024, st, p, maps);
 }
 

@@ -41,6 +41,9 @@ struct GemmParams {
   int n_tail;            // 64-wide reduction steps of the tail (only with splits == 1)
   int r_tail;            // reduction extent of the tail (its last step may be partial)
   int m_tiles, n_tiles;
+  // fused kernels' work items: n_items in all; with token pairs, tiles from full_items on are split into
+  // two items of one half each (n_items = full_items + 2 (m_tiles n_tiles - full_items))
+  int n_items, full_items;
   int b_atom;            // MN-major B: elements per swizzle atom row (16, 32 or 64)
   void* out;             // OUT_BF16_T: bf16 [Nn, ldo] receiving D^T; OUT_F32_D: fp32 [splits][m_tiles*128][ldo]
   int64_t ldo;

@@ -48,12 +48,49 @@ constexpr long long kDrainCycles = 4000000000LL;
 // bound `limit` (SM clock cycles) expires or another role already aborted.  Polls try_wait without a
 // suspend hint: measured on B200, a suspended waiter is not resumed promptly when a TMA transaction or a
 // tcgen05.commit completes the phase, which adds microseconds to every handshake.
+QLR_DEV bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounds below this are test bounds: polled with the non-blocking test_wait, so that 64 polls take a
+// fixed, short time (a try_wait may suspend the thread until the phase completes).
+constexpr long long kShortWaitCycles = 1000000LL;
+
 QLR_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, long long limit) {
-  if (mbar_try_wait(bar, parity)) return true;
+  const bool short_bound = limit < kShortWaitCycles;
+  if (short_bound ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (short_bound ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity)) return true;
     if ((it & 63) == 0) {
+      if (*abort_flag) return false;
+      if (clock64() - t0 > limit) {
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+
+// As mbar_wait, for a role that waits long and is not on the critical path (the epilogue, waiting for a
+// whole tile's accumulation): a 128 ns pause between polls leaves the issue slots of its warp scheduler to
+// the MMA issuer that shares it.  Not for the TMA producers: a late refill of a shallow ring stalls the MMAs.
+QLR_DEV bool mbar_wait_pause(uint64_t* bar, uint32_t parity, volatile int* abort_flag, long long limit) {
+  const bool short_bound = limit < kShortWaitCycles;
+  if (short_bound ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  for (uint32_t it = 1;; ++it) {
+    __nanosleep(128);
+    if (short_bound ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity)) return true;
+    if ((it & 15) == 0) {
       if (*abort_flag) return false;
       if (clock64() - t0 > limit) {
         *abort_flag = 1;

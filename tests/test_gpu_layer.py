@@ -246,3 +246,12 @@ def test_split_adapter_backward_on_two_streams_bit_identical(cuda_lib, pooled):
         assert torch.equal(a.view(torch.int16), b.view(torch.int16))
     for a, b in ((dA, dA0), (dB, dB0)):
         assert torch.equal(a.view(torch.int32), b.view(torch.int32))
+
+
+@pytest.mark.parametrize("N,K", [(11008, 512), (512, 11008)])
+def test_last_wave_split_into_half_tiles(cuda_lib, N, K):
+    """2048 tokens over 86 row tiles give 344 tiles of 128 x 512 on 148 SMs: the 48 tiles of the last wave
+    are split into 96 half tiles of 256 tokens (forward for N = 11008, input gradient for K = 11008)."""
+    spec = LinearSpec("w", N, K, "nfk", 4, 64, 256, r=16, s=0.5)
+    rows = np.sort(np.random.default_rng(N).choice(2048, 160, replace=False))
+    run_and_check(cuda_lib, spec, 2048, seed=17, rows=rows)
