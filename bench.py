@@ -239,7 +239,7 @@ class Layer:
         self.ws_s = qlr.Workspace(dev)  # the adapter gradients' second stream
 
 
-def run_ours(args, wl_name, rank, world, dev, steps, warmup, e2e_steps=None):
+def run_ours(args, wl_name, rank, world, dev, steps, warmup, e2e_steps=None, swiglu_fused=False):
     """Times `steps` training steps of workload `wl_name` (after `warmup` untimed ones) with CUDA events on
     the stream the kernels run on, L2 flushed before each step; then the same step end to end from pinned
     host memory.  Returns the measurements (time is the max over ranks)."""
@@ -252,7 +252,7 @@ def run_ours(args, wl_name, rank, world, dev, steps, warmup, e2e_steps=None):
     wl = workload(wl_name, args.seed)
     M = wl.M
     seed = args.seed
-    Hm = dG = dU = None
+    Hm = dHm = dG = dU = None
     if wl.kind == "mlp":
         gate_s, up_s, down_s = wl.linears
         gate = Layer(qlr, gate_s, M, seed, rank, dev)
@@ -260,7 +260,7 @@ def run_ours(args, wl_name, rank, world, dev, steps, warmup, e2e_steps=None):
         Hm = torch.empty((M, gate_s.N), dtype=torch.bfloat16, device=dev)
         down = Layer(qlr, down_s, M, seed + 2, rank, dev, X=Hm)
         layers = [gate, up, down]
-        dG, dU = torch.empty_like(Hm), torch.empty_like(Hm)
+        dHm, dG, dU = torch.empty_like(Hm), torch.empty_like(Hm), torch.empty_like(Hm)
     elif wl.kind == "stack":
         layers = [Layer(qlr, spec, M, seed * 100003 + i, rank, dev, on_device=True) for i, spec in enumerate(wl.linears)]
         torch.cuda.synchronize()
@@ -317,14 +317,20 @@ def run_ours(args, wl_name, rank, world, dev, steps, warmup, e2e_steps=None):
             qlr.lora_down(gate.q, gate.X, gate.A, gate.spec.s, T_save=gate.T, ws=gate.ws)
             qlr.lora_down(up.q, up.X, up.A, up.spec.s, T_save=up.T, ws=up.ws)
             fwd_base(gate, record)
-            # the up projection with the SwiGLU gate in its epilogue: U and H = silu(G) U in one launch
-            timed(record, fwd_ev, lambda: qlr.forward_swiglu(up.q, up.X, up.B, up.T, gate.Y, U=up.Y, H=Hm))
+            if swiglu_fused:  # the up projection with the SwiGLU gate in its epilogue: U and H in one launch
+                timed(record, fwd_ev, lambda: qlr.forward_swiglu(up.q, up.X, up.B, up.T, gate.Y, U=up.Y, H=Hm))
+            else:
+                fwd_base(up, record)
+                qlr.swiglu_forward(gate.Y, up.Y, H=Hm)
             qlr.lora_down(down.q, Hm, down.A, down.spec.s, T_save=down.T, ws=down.ws)
             fwd_base(down, record)
-            # the down projection's input gradient dH turned into (dG, dU) in its epilogue
             adapter_bwd(down, down.dY, X=Hm)
-            timed(record, dx_ev, lambda: qlr.backward_dx_swiglu(down.q, down.dY, down.A, down.dT, gate.Y, up.Y,
-                                                                dG=dG, dU=dU))
+            if swiglu_fused:  # the down projection's input gradient dH turned into (dG, dU) in its epilogue
+                timed(record, dx_ev, lambda: qlr.backward_dx_swiglu(down.q, down.dY, down.A, down.dT, gate.Y, up.Y,
+                                                                    dG=dG, dU=dU))
+            else:
+                timed(record, dx_ev, lambda: qlr.backward_dx(down.q, down.dY, down.A, down.dT, dX=dHm, ws=down.ws_x))
+                qlr.swiglu_backward(dHm, gate.Y, up.Y, dG=dG, dU=dU)
             lin_bwd(gate, dG, gate.dX, record)
             lin_bwd(up, dU, gate.dX, record, accumulate=True)
         else:  # one linear, or every linear of the stack in turn
@@ -846,8 +852,8 @@ def main():
     if world == 1 and not args.no_extra and args.workload == "lqlora":
         # the other configurations, each in its own timed run on the same GPU (not part of `value`)
         extra = {}
-        for name in ("qalora", "mlp7b"):
-            r = run_ours(args, name, 0, 1, dev, steps=10, warmup=3, e2e_steps=5)
+        for name, fused in (("qalora", False), ("mlp7b", False), ("mlp7b_swiglu_fused", True)):
+            r = run_ours(args, name.split("_")[0], 0, 1, dev, steps=10, warmup=3, e2e_steps=5, swiglu_fused=fused)
             ss = summarize(r, 1, peaks, peak_kind)
             extra[name] = {"workload": workload_desc(r["wl"]), "tokens_per_s": ss["value"],
                            "ms_per_step": ss["ms_per_step"], "tflops": ss["tflops"],

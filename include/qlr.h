@@ -164,8 +164,10 @@ QLR_API int qlr_dequant(const qlr_qweight* w, uint16_t* W_out, int32_t* status, 
  *           factors and cuSOLVER's work area; about 4 N K floats).
  * The SVD is cuSOLVER's single-precision gesvd, loaded at run time; without it the call returns
  * QLR_ERR_UNSUPPORTED (iters = 0 needs no solver).  This is an offline, once-per-weight call: it
- * synchronises the stream (the factorisation's status is read back after every SVD) and creates its
- * solver handle per call.  Singular vectors are unique up to sign, so A and B may differ in sign from
+ * synchronises the stream (the factorisation's status is read back after every SVD).  The solver handle is
+ * created once per device, on the first call made while that device is current (the solver allocates a
+ * little device memory for it then), and kept until the process exits; make that first call outside any
+ * stream capture.  Singular vectors are unique up to sign, so A and B may differ in sign from
  * another implementation's; their product does not.
  */
 QLR_API size_t qlr_lqlora_init_workspace_bytes(int64_t N, int64_t K, int r);

@@ -181,11 +181,34 @@ __device__ __forceinline__ void dequant_row64(const DqParams& dq, const uint8_t*
 }
 
 // Writes one 32-column chunk of an fp32 accumulator row as bf16 into out^T (out row = D column),
-// transposing through a per-warp 32 x 32 fp32 staging tile so that every global access is 16 bytes wide
-// (a thread handles 8 consecutive outputs of one row).  Every output is rounded to bf16 once: with
-// `accumulate`, after the previous bf16 value has been added to the fp32 result.
-__device__ __forceinline__ void store_chunk_bf16_t(const uint32_t (&v)[32], float* stg, int lane, int dcol0,
+// transposing through a per-warp 32 x 32 bf16 staging tile so that every global store is 16 bytes wide.
+__device__ __forceinline__ void store_chunk_bf16_t(const uint32_t (&v)[32], uint16_t* stg, int lane, int dcol0,
                                                    int drow0, const GemmParams& p) {
+#pragma unroll
+  for (int jj = 0; jj < 32; ++jj)
+    stg[jj * 32 + lane] = static_cast<uint16_t>(pack_bf16x2_rn(__uint_as_float(v[jj]), 0.f) & 0xFFFFu);
+  __syncwarp();
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    const int idx = t * 32 + lane;
+    const int jj = idx >> 2, part = idx & 3;
+    const int orow = dcol0 + jj;              // output row (D column)
+    const int ocol = drow0 + part * 8;        // output column (D row)
+    if (orow < p.Nn && ocol < p.Mm) {
+      const uint4 val = *reinterpret_cast<const uint4*>(stg + jj * 32 + part * 8);
+      *reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + static_cast<int64_t>(orow) * p.ldo + ocol) = val;
+    }
+  }
+  __syncwarp();
+}
+
+// As store_chunk_bf16_t, staged in fp32 for the outputs that need the unrounded value or more than a store
+// (a thread handles 8 consecutive outputs of one row): with `accumulate` the previous bf16 value is added to
+// the fp32 result before its one rounding; EPI_SWIGLU_FWD stores the result U and H = silu(G) U;
+// EPI_SWIGLU_BWD treats the result as dH and stores dG and dU instead.
+template <int EPI>
+__device__ __forceinline__ void store_chunk_f32_t(const uint32_t (&v)[32], float* stg, int lane, int dcol0, int drow0,
+                                                  const GemmParams& p) {
 #pragma unroll
   for (int jj = 0; jj < 32; ++jj) stg[jj * 32 + lane] = __uint_as_float(v[jj]);
   __syncwarp();
@@ -201,7 +224,7 @@ __device__ __forceinline__ void store_chunk_bf16_t(const uint32_t (&v)[32], floa
       float f[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
       const int64_t off = static_cast<int64_t>(orow) * p.ldo + ocol;
       uint16_t* dst = static_cast<uint16_t*>(p.out) + off;
-      if (p.accumulate) {
+      if (EPI == EPI_STORE && p.accumulate) {
         const uint4 o4 = *reinterpret_cast<const uint4*>(dst);
         const uint32_t ov[4] = {o4.x, o4.y, o4.z, o4.w};
 #pragma unroll
@@ -213,11 +236,10 @@ __device__ __forceinline__ void store_chunk_bf16_t(const uint32_t (&v)[32], floa
       uint32_t w[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) w[e] = pack_bf16x2_rn(f[2 * e], f[2 * e + 1]);
-      const uint4 val = make_uint4(w[0], w[1], w[2], w[3]);
-      if (p.epi == EPI_STORE) {
-        *reinterpret_cast<uint4*>(dst) = val;
-      } else if (p.epi == EPI_SWIGLU_FWD) {  // val = U; H = silu(G) U
-        *reinterpret_cast<uint4*>(dst) = val;
+      if (EPI == EPI_STORE) {
+        *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+      } else if (EPI == EPI_SWIGLU_FWD) {  // w = U; H = silu(G) U
+        *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
         const uint4 g4 = *reinterpret_cast<const uint4*>(p.aux_g + off);
         const uint32_t gv[4] = {g4.x, g4.y, g4.z, g4.w};
         uint32_t hv[4];
@@ -226,7 +248,7 @@ __device__ __forceinline__ void store_chunk_bf16_t(const uint32_t (&v)[32], floa
           hv[e] = pack_bf16x2_rn(swiglu_h(bf16_bits_to_f32(gv[e] & 0xFFFFu), bf16_bits_to_f32(w[e] & 0xFFFFu)),
                                  swiglu_h(bf16_bits_to_f32(gv[e] >> 16), bf16_bits_to_f32(w[e] >> 16)));
         *reinterpret_cast<uint4*>(p.aux_out + off) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-      } else {  // val = dH (bf16, as a stored dH would be); dG to out, dU to aux_out
+      } else {  // w = dH (bf16, as a stored dH would be); dG to out, dU to aux_out
         const uint4 g4 = *reinterpret_cast<const uint4*>(p.aux_g + off);
         const uint4 u4 = *reinterpret_cast<const uint4*>(p.aux_u + off);
         const uint32_t gv[4] = {g4.x, g4.y, g4.z, g4.w}, uv[4] = {u4.x, u4.y, u4.z, u4.w};

@@ -116,7 +116,8 @@ __device__ __forceinline__ void copy_row64_pooled(const uint16_t* src_row, bool 
 
 // PAIR: one tile covers 2 x BN tokens with both TMEM accumulators, so every dequantised weight
 // stage feeds twice the MMA work (the epilogue then does not overlap the next tile's main loop).
-template <int A_SRC, int BN, bool PAIR>
+// EPI: EPI_STORE (with a run-time accumulate flag), EPI_SWIGLU_FWD or EPI_SWIGLU_BWD (see GemmParams).
+template <int A_SRC, int BN, bool PAIR, int EPI>
 __global__ void __launch_bounds__(kThreadsFused, 1)
     fused_kernel(const __grid_constant__ GemmParams p, const __grid_constant__ GemmMaps maps) {
   using C = FCfg<BN>;
@@ -205,7 +206,9 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
         item_of(item, m0, n0, halves);
         bool ok = true;
         for (int ks = 0; ks < nsteps && ok; ++ks) {
-          for (int h = 0; h < halves; ++h, ++j) {
+#pragma unroll
+          for (int h = 0; h < HALVES; ++h) {
+            if (h >= halves) break;
             const int s = j % NSB;
             if (!mbar_wait(&bars->b_empty[s], ((j / NSB) & 1) ^ 1, abort_flag, p.wait_cycles)) { ok = false; break; }
             uint64_t* fb = &bars->b_full[s];
@@ -214,6 +217,7 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
               tma_load_2d(ring_b + s * C::kB, &maps.b, ks * 64, n0 + h * BN, fb);
             else
               tma_load_2d(ring_b + s * C::kB, &maps.b_tail, (ks - nmain) * 64, n0 + h * BN, fb);
+            ++j;
           }
         }
       }
@@ -275,7 +279,9 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
             const int rem = p.r_tail - (ks - nmain) * 64;
             nsub = rem >= 64 ? 4 : (rem + 15) / 16;
           }
-          for (int h = 0; h < halves; ++h, ++jb) {
+#pragma unroll
+          for (int h = 0; h < HALVES; ++h) {
+            if (h >= halves) break;
             const int sb = jb % NSB;
             if (!mbar_wait(&bars->b_full[sb], (jb / NSB) & 1, abort_flag, p.wait_cycles)) { ok = false; break; }
             tc_fence_after();
@@ -290,6 +296,7 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
                 umma_bf16_ss(d_tmem, ad0 + kk * kAk, bd0 + kk * kBk, kIdesc, (ks > 0 || kk > 0) ? 1u : 0u);
             }
             umma_commit(&bars->b_empty[sb]);
+            ++jb;
           }
           if (!ok) break;
           umma_commit(&bars->a_empty[sa]);
@@ -303,7 +310,8 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
   } else if (warp >= 2 && warp <= 5) {
     // ------------------------------------------------------------------ epilogue
     const int q = warp & 3;
-    float* stg = reinterpret_cast<float*>(staging) + q * 32 * 32;
+    uint16_t* stg = reinterpret_cast<uint16_t*>(staging) + q * 32 * 32;
+    float* stgf = reinterpret_cast<float*>(staging) + q * 32 * 32;
     int it = 0;
     for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it) {
       int m0, n0, halves;
@@ -319,7 +327,10 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
         uint32_t v[32];
         tmem_ld_32x32b_x32(tmem_base + (PAIR ? 0 : acc * BN) + c * 32 + ((q * 32) << 16), v);
         tmem_ld_wait();
-        eng::store_chunk_bf16_t(v, stg, lane, n0 + c * 32, m0 + q * 32, p);
+        if (EPI == EPI_STORE && !p.accumulate)
+          eng::store_chunk_bf16_t(v, stg, lane, n0 + c * 32, m0 + q * 32, p);
+        else
+          eng::store_chunk_f32_t<EPI>(v, stgf, lane, n0 + c * 32, m0 + q * 32, p);
       }
       tc_fence_before();
       mbar_arrive(&bars->acc_empty[acc]);
@@ -441,10 +452,10 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
   if (threadIdx.x == 0 && bars->abort_flag) report(p.status, QLR_ERR_TIMEOUT);
 }
 
-template <int A_SRC, int BN, bool PAIR>
+template <int A_SRC, int BN, bool PAIR, int EPI>
 cudaError_t launch_fused_variant(const GemmParams& p, const GemmMaps& maps, cudaStream_t st) {
   using C = FCfg<BN>;
-  auto kern = fused_kernel<A_SRC, BN, PAIR>;
+  auto kern = fused_kernel<A_SRC, BN, PAIR, EPI>;
   const cudaError_t attr_err = ensure_max_dynamic_smem(kern, C::kSmem + 1024);
   if (attr_err != cudaSuccess) return attr_err;
   const int items = p.n_items;
@@ -454,15 +465,28 @@ cudaError_t launch_fused_variant(const GemmParams& p, const GemmMaps& maps, cuda
 
 }  // namespace
 
-// bn = tokens per tile: 512 (paired 256-column accumulators), 256 or 64.
+namespace {
+template <int A_SRC, int EPI>
+cudaError_t launch_fused_epi(int bn, const GemmParams& p, const GemmMaps& maps, cudaStream_t st) {
+  if (bn == 512) return launch_fused_variant<A_SRC, 256, true, EPI>(p, maps, st);
+  if (bn == 256) return launch_fused_variant<A_SRC, 256, false, EPI>(p, maps, st);
+  if (bn == 64) return launch_fused_variant<A_SRC, 64, false, EPI>(p, maps, st);
+  return cudaErrorNotSupported;
+}
+}  // namespace
+
+// bn = tokens per tile: 512 (paired 256-column accumulators), 256 or 64; the epilogue mode is p.epi (the
+// SwiGLU forward only with the forward, the SwiGLU backward only with the input gradient).
 cudaError_t launch_fused(int a_src, int bn, const GemmParams& p, const GemmMaps& maps, cudaStream_t st) {
   if (p.splits != 1) return cudaErrorNotSupported;
-  if (a_src == A_DQ_K && bn == 512) return launch_fused_variant<A_DQ_K, 256, true>(p, maps, st);
-  if (a_src == A_DQ_K && bn == 256) return launch_fused_variant<A_DQ_K, 256, false>(p, maps, st);
-  if (a_src == A_DQ_K && bn == 64) return launch_fused_variant<A_DQ_K, 64, false>(p, maps, st);
-  if (a_src == A_DQ_MN && bn == 512) return launch_fused_variant<A_DQ_MN, 256, true>(p, maps, st);
-  if (a_src == A_DQ_MN && bn == 256) return launch_fused_variant<A_DQ_MN, 256, false>(p, maps, st);
-  if (a_src == A_DQ_MN && bn == 64) return launch_fused_variant<A_DQ_MN, 64, false>(p, maps, st);
+  if (a_src == A_DQ_K) {
+    if (p.epi == EPI_STORE) return launch_fused_epi<A_DQ_K, EPI_STORE>(bn, p, maps, st);
+    if (p.epi == EPI_SWIGLU_FWD) return launch_fused_epi<A_DQ_K, EPI_SWIGLU_FWD>(bn, p, maps, st);
+  }
+  if (a_src == A_DQ_MN) {
+    if (p.epi == EPI_STORE) return launch_fused_epi<A_DQ_MN, EPI_STORE>(bn, p, maps, st);
+    if (p.epi == EPI_SWIGLU_BWD) return launch_fused_epi<A_DQ_MN, EPI_SWIGLU_BWD>(bn, p, maps, st);
+  }
   return cudaErrorNotSupported;
 }
 

@@ -175,15 +175,27 @@ LqLayout lq_layout(int64_t N, int64_t K, int r, int lwork) {
   return L;
 }
 
+// One solver handle per device, created on the first call made while that device is current and kept for
+// the life of the process (the handle's own small device allocation happens once, not per call).
+cusolverDnHandle_t device_handle() {
+  static std::mutex mu;
+  static cusolverDnHandle_t handles[64] = {nullptr};
+  const Solver& sv = solver();
+  if (!sv.ok) return nullptr;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!handles[dev] && sv.create(&handles[dev]) != CUSOLVER_STATUS_SUCCESS) handles[dev] = nullptr;
+  return handles[dev];
+}
+
 int gesvd_lwork(int64_t N, int64_t K, int* lwork) {
   const Solver& sv = solver();
   if (!sv.ok) return QLR_ERR_UNSUPPORTED;
-  cusolverDnHandle_t h = nullptr;
-  if (sv.create(&h) != CUSOLVER_STATUS_SUCCESS) return QLR_ERR_CUDA;
+  cusolverDnHandle_t h = device_handle();
+  if (!h) return QLR_ERR_CUDA;
   const int m = static_cast<int>(N > K ? N : K), n = static_cast<int>(N > K ? K : N);
-  const cusolverStatus_t st = sv.buffer_size(h, m, n, lwork);
-  sv.destroy(h);
-  return st == CUSOLVER_STATUS_SUCCESS ? QLR_OK : QLR_ERR_CUDA;
+  return sv.buffer_size(h, m, n, lwork) == CUSOLVER_STATUS_SUCCESS ? QLR_OK : QLR_ERR_CUDA;
 }
 
 int check_lq_args(int64_t N, int64_t K, int bits, int block, int dq_block, int r, int iters) {
@@ -247,8 +259,8 @@ extern "C" int qlr_lqlora_init(const float* W, int64_t N, int64_t K, int bits, i
   const bool wide = K >= N;
   const int m = static_cast<int>(wide ? K : N), n = static_cast<int>(wide ? N : K);
 
-  cusolverDnHandle_t h = nullptr;
-  if (sv.create(&h) != CUSOLVER_STATUS_SUCCESS) return QLR_ERR_CUDA;
+  cusolverDnHandle_t h = device_handle();
+  if (!h) return QLR_ERR_CUDA;
   rc = QLR_OK;
   for (int t = 0; t < iters && rc == QLR_OK; ++t) {
     // the residual to factor: W (t = 0), else W - dequant(Q_t)
@@ -293,6 +305,5 @@ extern "C" int qlr_lqlora_init(const float* W, int64_t N, int64_t K, int bits, i
     if (cudaGetLastError() != cudaSuccess || cudaStreamSynchronize(st) != cudaSuccess) rc = QLR_ERR_CUDA;
   }
   cudaStreamSynchronize(st);
-  sv.destroy(h);
   return rc;
 }

@@ -60,8 +60,9 @@ QLR_DEV bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounds below this are test bounds: polled with the non-blocking test_wait, so that 64 polls take a
-// fixed, short time (a try_wait may suspend the thread until the phase completes).
+// Bounds below this are test bounds: polled with the non-blocking test_wait and the clock read after every
+// poll, so that a wait not complete at once runs out (a try_wait may suspend the thread until the phase
+// completes, and a wait then never sees its bound).
 constexpr long long kShortWaitCycles = 1000000LL;
 
 QLR_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, long long limit) {
@@ -70,7 +71,7 @@ QLR_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
   const long long t0 = clock64();
   for (uint32_t it = 1;; ++it) {
     if (short_bound ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity)) return true;
-    if ((it & 63) == 0) {
+    if (short_bound || (it & 63) == 0) {
       if (*abort_flag) return false;
       if (clock64() - t0 > limit) {
         *abort_flag = 1;
@@ -90,7 +91,7 @@ QLR_DEV bool mbar_wait_pause(uint64_t* bar, uint32_t parity, volatile int* abort
   for (uint32_t it = 1;; ++it) {
     __nanosleep(128);
     if (short_bound ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity)) return true;
-    if ((it & 15) == 0) {
+    if (short_bound || (it & 15) == 0) {
       if (*abort_flag) return false;
       if (clock64() - t0 > limit) {
         *abort_flag = 1;
