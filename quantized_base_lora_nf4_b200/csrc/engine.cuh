@@ -206,11 +206,14 @@ __device__ __forceinline__ void store_chunk_bf16_t(const uint32_t (&v)[32], uint
 // (a thread handles 8 consecutive outputs of one row): with `accumulate` the previous bf16 value is added to
 // the fp32 result before its one rounding; EPI_SWIGLU_FWD stores the result U and H = silu(G) U;
 // EPI_SWIGLU_BWD treats the result as dH and stores dG and dU instead.
+// The staging tile keeps row jj's column c at jj * 32 + (c ^ 4 (jj mod 8)): the XOR moves whole 16-byte
+// groups, so both the column writes (one row per loop step, a lane per column) and the 16-byte row reads
+// spread over all 32 banks.
 template <int EPI>
 __device__ __forceinline__ void store_chunk_f32_t(const uint32_t (&v)[32], float* stg, int lane, int dcol0, int drow0,
                                                   const GemmParams& p) {
 #pragma unroll
-  for (int jj = 0; jj < 32; ++jj) stg[jj * 32 + lane] = __uint_as_float(v[jj]);
+  for (int jj = 0; jj < 32; ++jj) stg[jj * 32 + (lane ^ ((jj & 7) << 2))] = __uint_as_float(v[jj]);
   __syncwarp();
 #pragma unroll
   for (int t = 0; t < 4; ++t) {
@@ -219,8 +222,9 @@ __device__ __forceinline__ void store_chunk_f32_t(const uint32_t (&v)[32], float
     const int orow = dcol0 + jj;              // output row (D column)
     const int ocol = drow0 + part * 8;        // output column (D row)
     if (orow < p.Nn && ocol < p.Mm) {
-      const float4 f0 = *reinterpret_cast<const float4*>(stg + jj * 32 + part * 8);
-      const float4 f1 = *reinterpret_cast<const float4*>(stg + jj * 32 + part * 8 + 4);
+      const int sw = (jj & 7) << 2;
+      const float4 f0 = *reinterpret_cast<const float4*>(stg + jj * 32 + ((part * 8) ^ sw));
+      const float4 f1 = *reinterpret_cast<const float4*>(stg + jj * 32 + ((part * 8 + 4) ^ sw));
       float f[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
       const int64_t off = static_cast<int64_t>(orow) * p.ldo + ocol;
       uint16_t* dst = static_cast<uint16_t*>(p.out) + off;

@@ -19,6 +19,7 @@
 // accumulators (2 x BN fp32 columns) overlap each tile's epilogue with the next tile's main loop.
 // Every wait is bounded; a wait that runs out aborts the CTA and reports QLR_ERR_TIMEOUT.
 #include <mutex>
+#include <type_traits>
 
 #include "engine.cuh"
 
@@ -205,21 +206,27 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
         int m0, n0, halves;
         item_of(item, m0, n0, halves);
         bool ok = true;
-        for (int ks = 0; ks < nsteps && ok; ++ks) {
+        auto loads = [&](auto nh_tag) {
+          constexpr int NH = decltype(nh_tag)::value;
+          for (int ks = 0; ks < nsteps && ok; ++ks) {
 #pragma unroll
-          for (int h = 0; h < HALVES; ++h) {
-            if (h >= halves) break;
-            const int s = j % NSB;
-            if (!mbar_wait(&bars->b_empty[s], ((j / NSB) & 1) ^ 1, abort_flag, p.wait_cycles)) { ok = false; break; }
-            uint64_t* fb = &bars->b_full[s];
-            mbar_arrive_expect_tx(fb, C::kB);
-            if (ks < nmain)
-              tma_load_2d(ring_b + s * C::kB, &maps.b, ks * 64, n0 + h * BN, fb);
-            else
-              tma_load_2d(ring_b + s * C::kB, &maps.b_tail, (ks - nmain) * 64, n0 + h * BN, fb);
-            ++j;
+            for (int h = 0; h < NH; ++h) {
+              const int s = j % NSB;
+              if (!mbar_wait(&bars->b_empty[s], ((j / NSB) & 1) ^ 1, abort_flag, p.wait_cycles)) { ok = false; break; }
+              uint64_t* fb = &bars->b_full[s];
+              mbar_arrive_expect_tx(fb, C::kB);
+              if (ks < nmain)
+                tma_load_2d(ring_b + s * C::kB, &maps.b, ks * 64, n0 + h * BN, fb);
+              else
+                tma_load_2d(ring_b + s * C::kB, &maps.b_tail, (ks - nmain) * 64, n0 + h * BN, fb);
+              ++j;
+            }
           }
-        }
+        };
+        if (halves == HALVES)
+          loads(std::integral_constant<int, HALVES>{});
+        else
+          loads(std::integral_constant<int, 1>{});
       }
       const uint32_t first = j > NSB ? j - NSB : 0;
       for (uint32_t q = first; q < j; ++q) {
@@ -270,37 +277,45 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
         const uint32_t acc_par = PAIR ? ((it & 1) ^ 1) : (((it >> 1) & 1) ^ 1);
         if (!mbar_wait(&bars->acc_empty[acc], acc_par, abort_flag, p.wait_cycles)) break;
         tc_fence_after();
-        for (int ks = 0; ks < nsteps && ok; ++ks, ++j) {
-          const int sa = j % NSA;
-          if (!mbar_wait(&bars->a_full[sa], (j / NSA) & 1, abort_flag, p.wait_cycles)) { ok = false; break; }
-          const uint64_t ad0 = a_desc0 + static_cast<uint32_t>((sa * C::kA) >> 4);
-          int nsub = 4;
-          if (ks >= nmain) {
-            const int rem = p.r_tail - (ks - nmain) * 64;
-            nsub = rem >= 64 ? 4 : (rem + 15) / 16;
-          }
-#pragma unroll
-          for (int h = 0; h < HALVES; ++h) {
-            if (h >= halves) break;
-            const int sb = jb % NSB;
-            if (!mbar_wait(&bars->b_full[sb], (jb / NSB) & 1, abort_flag, p.wait_cycles)) { ok = false; break; }
-            tc_fence_after();
-            const uint64_t bd0 = b_desc0 + static_cast<uint32_t>((sb * C::kB) >> 4);
-            const uint32_t d_tmem = tmem_base + (PAIR ? h : acc) * BN;
-            if (nsub == 4) {
-#pragma unroll
-              for (int kk = 0; kk < 4; ++kk)
-                umma_bf16_ss(d_tmem, ad0 + kk * kAk, bd0 + kk * kBk, kIdesc, (ks > 0 || kk > 0) ? 1u : 0u);
-            } else {
-              for (int kk = 0; kk < nsub; ++kk)
-                umma_bf16_ss(d_tmem, ad0 + kk * kAk, bd0 + kk * kBk, kIdesc, (ks > 0 || kk > 0) ? 1u : 0u);
+        // the step loop with the activation stages per step (halves) as a compile-time count: a split tail
+        // item runs the one-stage copy, everything else the unrolled full one
+        auto steps = [&](auto nh_tag) {
+          constexpr int NH = decltype(nh_tag)::value;
+          for (int ks = 0; ks < nsteps && ok; ++ks, ++j) {
+            const int sa = j % NSA;
+            if (!mbar_wait(&bars->a_full[sa], (j / NSA) & 1, abort_flag, p.wait_cycles)) { ok = false; break; }
+            const uint64_t ad0 = a_desc0 + static_cast<uint32_t>((sa * C::kA) >> 4);
+            int nsub = 4;
+            if (ks >= nmain) {
+              const int rem = p.r_tail - (ks - nmain) * 64;
+              nsub = rem >= 64 ? 4 : (rem + 15) / 16;
             }
-            umma_commit(&bars->b_empty[sb]);
-            ++jb;
+#pragma unroll
+            for (int h = 0; h < NH; ++h) {
+              const int sb = jb % NSB;
+              if (!mbar_wait(&bars->b_full[sb], (jb / NSB) & 1, abort_flag, p.wait_cycles)) { ok = false; break; }
+              tc_fence_after();
+              const uint64_t bd0 = b_desc0 + static_cast<uint32_t>((sb * C::kB) >> 4);
+              const uint32_t d_tmem = tmem_base + (PAIR ? h : acc) * BN;
+              if (nsub == 4) {
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                  umma_bf16_ss(d_tmem, ad0 + kk * kAk, bd0 + kk * kBk, kIdesc, (ks > 0 || kk > 0) ? 1u : 0u);
+              } else {
+                for (int kk = 0; kk < nsub; ++kk)
+                  umma_bf16_ss(d_tmem, ad0 + kk * kAk, bd0 + kk * kBk, kIdesc, (ks > 0 || kk > 0) ? 1u : 0u);
+              }
+              umma_commit(&bars->b_empty[sb]);
+              ++jb;
+            }
+            if (!ok) break;
+            umma_commit(&bars->a_empty[sa]);
           }
-          if (!ok) break;
-          umma_commit(&bars->a_empty[sa]);
-        }
+        };
+        if (halves == HALVES)
+          steps(std::integral_constant<int, HALVES>{});
+        else
+          steps(std::integral_constant<int, 1>{});
         if (!ok) break;
         umma_commit(&bars->acc_full[acc]);
       }

@@ -44,34 +44,26 @@ constexpr long long kWaitCycles = 4000000000LL;
 // always complete, and the CTA must not exit (or free its tensor memory) before they have.
 constexpr long long kDrainCycles = 4000000000LL;
 
+// Bounds below this are test bounds: the clock is read after every poll, so that a wait that is not
+// complete within one try_wait runs out (with checks every 64 polls, a try_wait that suspends the thread
+// until the phase completes lets short waits finish before their bound is ever looked at).  The loop is
+// the same either way: a second loop or a branch inside the MMA issuer's wait measurably slowed the
+// fused kernels.
+constexpr long long kShortWaitCycles = 1000000LL;
+
 // Waits for the phase with the given parity to complete.  Returns false (and raises *abort) when the
 // bound `limit` (SM clock cycles) expires or another role already aborted.  Polls try_wait without a
 // suspend hint: measured on B200, a suspended waiter is not resumed promptly when a TMA transaction or a
 // tcgen05.commit completes the phase, which adds microseconds to every handshake.
-QLR_DEV bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Bounds below this are test bounds: polled with the non-blocking test_wait and the clock read after every
-// poll, so that a wait not complete at once runs out (a try_wait may suspend the thread until the phase
-// completes, and a wait then never sees its bound).
-constexpr long long kShortWaitCycles = 1000000LL;
 
 QLR_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, long long limit) {
-  const bool short_bound = limit < kShortWaitCycles;
-  if (short_bound ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity)) return true;
+  if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
+  // the bound is checked every 64 polls, or after every poll under a test bound
+  const uint32_t mask = limit < kShortWaitCycles ? 0u : 63u;
   for (uint32_t it = 1;; ++it) {
-    if (short_bound ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity)) return true;
-    if (short_bound || (it & 63) == 0) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & mask) == 0) {
       if (*abort_flag) return false;
       if (clock64() - t0 > limit) {
         *abort_flag = 1;
@@ -85,13 +77,13 @@ QLR_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
 // whole tile's accumulation): a 128 ns pause between polls leaves the issue slots of its warp scheduler to
 // the MMA issuer that shares it.  Not for the TMA producers: a late refill of a shallow ring stalls the MMAs.
 QLR_DEV bool mbar_wait_pause(uint64_t* bar, uint32_t parity, volatile int* abort_flag, long long limit) {
-  const bool short_bound = limit < kShortWaitCycles;
-  if (short_bound ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity)) return true;
+  if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
+  const uint32_t mask = limit < kShortWaitCycles ? 0u : 15u;
   for (uint32_t it = 1;; ++it) {
     __nanosleep(128);
-    if (short_bound ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity)) return true;
-    if (short_bound || (it & 15) == 0) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & mask) == 0) {
       if (*abort_flag) return false;
       if (clock64() - t0 > limit) {
         *abort_flag = 1;
