@@ -61,10 +61,15 @@ def parse():
 
 
 # ------------------------------------------------------------------------------------------ accounting
-def flush_l2(buf):
+def flush_l2(buf, lead_ms: float = 1.0):
     """Evict the step's data from L2: write a buffer larger than L2, then read it back, so that the
-    timed step neither hits in L2 nor pays for writing back the flush's own dirty lines."""
+    timed step neither hits in L2 nor pays for writing back the flush's own dirty lines.  First the stream
+    spins for `lead_ms` on the device, so that the host enqueues the flush, the start event and the whole
+    timed step while the GPU is still busy: the events then time the GPU's work, with no gaps where it
+    waits for the host to launch the next kernel (the small workloads launch faster than Python can)."""
     import torch
+    if lead_ms > 0:
+        torch.cuda._sleep(int(lead_ms * 2.0e6))  # ~2e6 SM cycles per ms at the B200's clocks
     buf.zero_()
     return buf.view(torch.int32).amax()
 

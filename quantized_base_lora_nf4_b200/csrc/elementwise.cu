@@ -70,29 +70,83 @@ __global__ void expand_kernel(const uint16_t* __restrict__ A, int r, int64_t K, 
   Aexp[i] = static_cast<uint16_t>(pack_bf16x2_rn(v, 0.f) & 0xFFFFu);
 }
 
-// Split-order sum of an adapter GEMM's parts + its output transform, one thread per output element.
-__global__ void adapter_reduce_kernel(const AdapterParams p, int bn) {
+// Split-order sum of an adapter GEMM's parts + its output transform, row outputs (T_save, dT: bf16 scaled;
+// dB: fp32): a thread sums four consecutive columns of one row, every split's 16 bytes loaded before any
+// addition, and adds them in split order (deterministic, and the same sums as one column per thread).
+__global__ void __launch_bounds__(256) adapter_reduce_rows_kernel(const AdapterParams p, int bn) {
   pdl_launch_dependents();
   pdl_wait();
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int q = p.r / 4;  // float4 groups per row
+  if (i >= static_cast<int64_t>(p.Mm) * q) return;
+  const int64_t m = i / q;
+  const int j = static_cast<int>(i - m * q) * 4;
   const int64_t split_stride = static_cast<int64_t>(p.m_tiles) * 128 * bn;
-  if (i >= static_cast<int64_t>(p.Mm) * p.r) return;
-  int64_t m, j;
-  if (p.out_mode == ADAPTER_COLS_F32) {  // consecutive threads walk output columns (coalesced stores)
-    j = i / p.Mm;
-    m = i % p.Mm;
-  } else {
-    m = i / p.r;
-    j = i % p.r;
+  const float* src = p.part + m * bn + j;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  int s = 0;
+  for (; s + 4 <= p.splits; s += 4) {  // four splits' loads in flight, summed in order
+    float4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) v[u] = __ldg(reinterpret_cast<const float4*>(src + (s + u) * split_stride));
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      acc.x += v[u].x;
+      acc.y += v[u].y;
+      acc.z += v[u].z;
+      acc.w += v[u].w;
+    }
   }
-  float acc = 0.f;
-  for (int s = 0; s < p.splits; ++s) acc += p.part[s * split_stride + m * bn + j];
-  if (p.out_mode == ADAPTER_ROWS_BF16)
-    static_cast<uint16_t*>(p.out)[m * p.ld_out + j] = static_cast<uint16_t>(pack_bf16x2_rn(p.scale * acc, 0.f) & 0xFFFFu);
-  else if (p.out_mode == ADAPTER_ROWS_F32)
-    static_cast<float*>(p.out)[m * p.ld_out + j] = acc;
-  else
-    static_cast<float*>(p.out)[j * p.ld_out + m] = acc;
+  for (; s < p.splits; ++s) {
+    const float4 v = __ldg(reinterpret_cast<const float4*>(src + s * split_stride));
+    acc.x += v.x;
+    acc.y += v.y;
+    acc.z += v.z;
+    acc.w += v.w;
+  }
+  if (p.out_mode == ADAPTER_ROWS_BF16) {
+    uint2 w;
+    w.x = pack_bf16x2_rn(p.scale * acc.x, p.scale * acc.y);
+    w.y = pack_bf16x2_rn(p.scale * acc.z, p.scale * acc.w);
+    *reinterpret_cast<uint2*>(static_cast<uint16_t*>(p.out) + m * p.ld_out + j) = w;
+  } else {
+    *reinterpret_cast<float4*>(static_cast<float*>(p.out) + m * p.ld_out + j) = acc;
+  }
+}
+
+// The transposed output out[j, m] (dA^T, unpooled): a CTA takes 32 rows m, sums their splits (coalesced
+// 16-byte loads of whole rows, split order), turns the 32 x r tile in shared memory and writes each column
+// j as 32 consecutive floats.
+__global__ void __launch_bounds__(256) adapter_reduce_cols_kernel(const AdapterParams p, int bn) {
+  __shared__ float tile[32][65];
+  pdl_launch_dependents();
+  pdl_wait();
+  const int64_t m0 = static_cast<int64_t>(blockIdx.x) * 32;
+  const int64_t split_stride = static_cast<int64_t>(p.m_tiles) * 128 * bn;
+  const int q = p.r / 4;
+  for (int e = threadIdx.x; e < 32 * q; e += blockDim.x) {
+    const int row = e / q, j = (e - row * q) * 4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (m0 + row < p.Mm) {
+      const float* src = p.part + (m0 + row) * bn + j;
+      for (int s = 0; s < p.splits; ++s) {
+        const float4 v = __ldg(reinterpret_cast<const float4*>(src + s * split_stride));
+        acc.x += v.x;
+        acc.y += v.y;
+        acc.z += v.z;
+        acc.w += v.w;
+      }
+    }
+    tile[row][j] = acc.x;
+    tile[row][j + 1] = acc.y;
+    tile[row][j + 2] = acc.z;
+    tile[row][j + 3] = acc.w;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < 32 * p.r; e += blockDim.x) {
+    const int j = e >> 5, row = e & 31;
+    if (m0 + row < p.Mm) static_cast<float*>(p.out)[static_cast<int64_t>(j) * p.ld_out + m0 + row] = tile[row][j];
+  }
 }
 
 // The pooled transposed output out[j, g] = (sum of the L rows of group g) / L: a block of 256 threads
@@ -190,9 +244,13 @@ cudaError_t launch_adapter_reduce(const AdapterParams& p, int bn, cudaStream_t s
     const int64_t blocks = (static_cast<int64_t>(p.Mm) + 255) / 256 * p.r;
     return launch_pdl(adapter_reduce_pooled_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st, p, bn);
   }
-  const int64_t n = static_cast<int64_t>(p.Mm) * p.r;
-  if (n == 0) return cudaSuccess;
-  return launch_pdl(adapter_reduce_kernel, dim3(static_cast<unsigned>((n + 255) / 256)), dim3(256), 0, st, p, bn);
+  if (p.Mm == 0) return cudaSuccess;
+  if (p.out_mode == ADAPTER_COLS_F32) {
+    const int64_t blocks = (static_cast<int64_t>(p.Mm) + 31) / 32;
+    return launch_pdl(adapter_reduce_cols_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st, p, bn);
+  }
+  const int64_t n = static_cast<int64_t>(p.Mm) * (p.r / 4);
+  return launch_pdl(adapter_reduce_rows_kernel, dim3(static_cast<unsigned>((n + 255) / 256)), dim3(256), 0, st, p, bn);
 }
 
 cudaError_t launch_swiglu_fwd(const uint16_t* G, const uint16_t* U, uint16_t* H, int64_t n, cudaStream_t st) {

@@ -9,7 +9,7 @@
 // Warp roles: 0 TMA producer (ring of A+B stages), 1 TMEM allocator + single-thread tcgen05.mma
 // issuer, 2..5 epilogue.  Two TMEM accumulators overlap an item's epilogue with the next item's main
 // loop.  Without a split the epilogue applies the output transform directly; with one, each item's
-// fp32 tile goes to the workspace and `adapter_reduce_kernel` (elementwise.cu) sums the parts in
+// fp32 tile goes to the workspace and a reduction kernel (elementwise.cu) sums the parts in
 // split order (deterministic) and applies the transform with one thread per output.
 #include <cudaTypedefs.h>
 
