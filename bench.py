@@ -612,8 +612,9 @@ def run_lqlora_init(args, dev, iters: int = 2):
     alloc = run_lqlora_allocation(args, dev, wl)
     return {"metric": "LQ-LoRA initialisation time per matrix (ms), whole call", "per_shape": out,
             "stack_projection_s": stack_s, "stack_matrices": len(wl.linears), "allocation": alloc,
-            "note": "truncated SVD: single-precision cuSOLVER gesvd on the full matrix; residual, rank-r "
-                    "subtraction, factor split and quantisation in this library's kernels"}
+            "note": "truncated SVD: top-r eigenpairs of the smaller-side Gram matrix (fp32 cuBLAS syrk + "
+                    "cuSOLVER syevdx) and one projection GEMM; residual, rank-r subtraction, factor split and "
+                    "quantisation in this library's kernels"}
 
 
 def run_lqlora_allocation(args, dev, wl):

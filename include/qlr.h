@@ -160,15 +160,17 @@ QLR_API int qlr_dequant(const qlr_qweight* w, uint16_t* W_out, int32_t* status, 
  *   out     NF-k weight descriptor with buffers sized by qlr_qweight_part_bytes (fmt, bits, block,
  *           dq_block, N, K must match the arguments); codes and constants are written.
  *   r       1 .. 64 and <= min(N, K);  s > 0;  iters 0 .. 64.
- *   workspace  qlr_lqlora_init_workspace_bytes(N, K, r) bytes, 256-byte aligned (residual, the SVD
- *           factors and cuSOLVER's work area; about 4 N K floats).
- * The SVD is cuSOLVER's single-precision gesvd, loaded at run time; without it the call returns
- * QLR_ERR_UNSUPPORTED (iters = 0 needs no solver).  This is an offline, once-per-weight call: it
- * synchronises the stream (the factorisation's status is read back after every SVD).  The solver handle is
- * created once per device, on the first call made while that device is current (the solver allocates a
- * little device memory for it then), and kept until the process exits; make that first call outside any
- * stream capture.  Singular vectors are unique up to sign, so A and B may differ in sign from
- * another implementation's; their product does not.
+ *   workspace  qlr_lqlora_init_workspace_bytes(N, K, r) bytes, 256-byte aligned (residual, Gram
+ *           matrix, factors and the eigensolver's work area; about N K + min(N, K)^2 floats).
+ * The truncated SVD comes from the r largest eigenpairs of the Gram matrix on the smaller side
+ * (R^T R when K <= N, else R R^T) and one projection of R onto them; the Gram matrix and the projection
+ * are single-precision cuBLAS products and the eigenpairs cuSOLVER's syevdx (index range), both loaded
+ * at run time; without them the call returns QLR_ERR_UNSUPPORTED (iters = 0 needs neither).  This is
+ * an offline, once-per-weight call: it synchronises the stream (the eigensolver's status is read back
+ * every iteration).  The solver and BLAS handles are created once per device, on the first call made
+ * while that device is current (the libraries allocate a little device memory for them then), and
+ * kept until the process exits; make that first call outside any stream capture.  Singular vectors are
+ * unique up to sign, so A and B may differ in sign from another implementation's; their product does not.
  */
 QLR_API size_t qlr_lqlora_init_workspace_bytes(int64_t N, int64_t K, int r);
 QLR_API int qlr_lqlora_init(const float* W, int64_t N, int64_t K, int bits, int block, int dq_block, int r, float s,

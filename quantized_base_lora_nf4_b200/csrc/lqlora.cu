@@ -6,10 +6,16 @@
 //                              Q_t = NF-k quantisation of (W - L_t)
 // with the adapter A = bf16(sqrt(S_r) V_r^T), B = bf16(U_r sqrt(S_r) / s), so s B A = L_T.
 //
-// Residuals, the rank-r subtraction, the factor split and the quantisation run in this library's
-// kernels; the SVD is cuSOLVER's gesvd (a library factorisation), loaded with dlopen on first use so
-// that the library itself has no link-time dependency on it.  An offline, once-per-weight step.
+// The rank-r truncated SVD of the residual R [N, K] comes from the r largest eigenpairs of its Gram
+// matrix on the smaller side: with n = min(N, K), G = R^T R (K <= N) or R R^T (N < K), G = V S^2 V^T,
+// so the top-r right (or left) singular vectors are G's top-r eigenvectors and the other factor is
+// R V_r / S_r (or R^T U_r / S_r).  Only r of the n eigenpairs are computed, instead of a full SVD of R.
+// G and the projection are plain single-precision library GEMMs (cuBLAS), the eigenpairs a library
+// eigensolver (cuSOLVER syevdx, index range n - r + 1 .. n); both are loaded with dlopen on first use, so
+// the library itself has no link-time dependency on them.  Residuals, the rank-r subtraction, the factor
+// split and the quantisation run in this library's kernels.  An offline, once-per-weight step.
 #include <cuda_fp8.h>
+#include <cublas_v2.h>
 #include <cusolverDn.h>
 #include <dlfcn.h>
 
@@ -23,13 +29,16 @@ namespace qlr {
 
 namespace {
 
-// ---- cuSOLVER, resolved at run time ------------------------------------------------------------
+// ---- cuSOLVER and cuBLAS, resolved at run time --------------------------------------------------
 struct Solver {
   decltype(&cusolverDnCreate) create = nullptr;
-  decltype(&cusolverDnDestroy) destroy = nullptr;
   decltype(&cusolverDnSetStream) set_stream = nullptr;
-  decltype(&cusolverDnSgesvd_bufferSize) buffer_size = nullptr;
-  decltype(&cusolverDnSgesvd) gesvd = nullptr;
+  decltype(&cusolverDnSsyevdx_bufferSize) evd_buffer = nullptr;
+  decltype(&cusolverDnSsyevdx) evd = nullptr;
+  decltype(&cublasCreate_v2) blas_create = nullptr;
+  decltype(&cublasSetStream_v2) blas_set_stream = nullptr;
+  decltype(&cublasSsyrk_v2) syrk = nullptr;
+  decltype(&cublasSgemm_v2) gemm = nullptr;
   bool ok = false;
 };
 
@@ -39,13 +48,18 @@ const Solver& solver() {
   std::call_once(once, [] {
     void* h = dlopen("libcusolver.so.11", RTLD_NOW | RTLD_LOCAL);
     if (!h) h = dlopen("libcusolver.so", RTLD_NOW | RTLD_LOCAL);
-    if (!h) return;
+    void* b = dlopen("libcublas.so.12", RTLD_NOW | RTLD_LOCAL);
+    if (!b) b = dlopen("libcublas.so", RTLD_NOW | RTLD_LOCAL);
+    if (!h || !b) return;
     s.create = reinterpret_cast<decltype(s.create)>(dlsym(h, "cusolverDnCreate"));
-    s.destroy = reinterpret_cast<decltype(s.destroy)>(dlsym(h, "cusolverDnDestroy"));
     s.set_stream = reinterpret_cast<decltype(s.set_stream)>(dlsym(h, "cusolverDnSetStream"));
-    s.buffer_size = reinterpret_cast<decltype(s.buffer_size)>(dlsym(h, "cusolverDnSgesvd_bufferSize"));
-    s.gesvd = reinterpret_cast<decltype(s.gesvd)>(dlsym(h, "cusolverDnSgesvd"));
-    s.ok = s.create && s.destroy && s.set_stream && s.buffer_size && s.gesvd;
+    s.evd_buffer = reinterpret_cast<decltype(s.evd_buffer)>(dlsym(h, "cusolverDnSsyevdx_bufferSize"));
+    s.evd = reinterpret_cast<decltype(s.evd)>(dlsym(h, "cusolverDnSsyevdx"));
+    s.blas_create = reinterpret_cast<decltype(s.blas_create)>(dlsym(b, "cublasCreate_v2"));
+    s.blas_set_stream = reinterpret_cast<decltype(s.blas_set_stream)>(dlsym(b, "cublasSetStream_v2"));
+    s.syrk = reinterpret_cast<decltype(s.syrk)>(dlsym(b, "cublasSsyrk_v2"));
+    s.gemm = reinterpret_cast<decltype(s.gemm)>(dlsym(b, "cublasSgemm_v2"));
+    s.ok = s.create && s.set_stream && s.evd_buffer && s.evd && s.blas_create && s.blas_set_stream && s.syrk && s.gemm;
   });
   return s;
 }
@@ -58,41 +72,36 @@ __global__ void residual_kernel(const float* __restrict__ W, int64_t n, const nf
     R[i] = __fsub_rn(W[i], nfk::dequant_at(v, i));
 }
 
-// column-major copy (N x K, leading dimension N) of the row-major N x K matrix R
-__global__ void transpose_kernel(const float* __restrict__ R, int64_t N, int64_t K, float* __restrict__ T) {
-  __shared__ float tile[32][33];
-  const int64_t i0 = static_cast<int64_t>(blockIdx.y) * 32, k0 = static_cast<int64_t>(blockIdx.x) * 32;
-  for (int y = threadIdx.y; y < 32; y += blockDim.y) {
-    const int64_t i = i0 + y, k = k0 + threadIdx.x;
-    if (i < N && k < K) tile[y][threadIdx.x] = R[i * K + k];
-  }
-  __syncthreads();
-  for (int y = threadIdx.y; y < 32; y += blockDim.y) {
-    const int64_t k = k0 + y, i = i0 + threadIdx.x;
-    if (i < N && k < K) T[k * N + i] = tile[threadIdx.x][y];
-  }
-}
-
-// Ur[i][c] = U_R[i][c] sqrt(S[c]) (N x r), Vr[c][k] = sqrt(S[c]) V_R^T[c][k] (r x K), both row-major.
-// wide (K >= N): gesvd factored R^T (K x N) = U' S V'^T, so U_R = V' (from VT, ld N), V_R^T = U'^T (from U, ld K);
-// else: gesvd factored R (N x K) = U S V^T, so U_R = U (ld N), V_R^T = VT (ld K).
-__global__ void factors_kernel(const float* __restrict__ U, const float* __restrict__ VT, const float* __restrict__ S,
-                               int64_t N, int64_t K, int r, int wide, float* __restrict__ Ur, float* __restrict__ Vr) {
+// The rank-r factors from the Gram matrix's top eigenpairs, split as Ur = U_r sqrt(S_r) [N, r] and
+// Vr = sqrt(S_r) V_r^T [r, K], both row-major, components in descending order.  E holds the eigenvectors
+// (column-major, leading dimension n, ascending eigenvalues lam[0 .. r-1]); P the projection of R onto
+// them (column-major): tall (K <= N, n = K): E = V_r, P = R V_r = U_r S_r [N x r, ld N];
+// wide (N < K, n = N): E = U_r, P = R^T U_r = V_r S_r [K x r, ld K].  s_c = sqrt(lam_c).
+__global__ void gram_factors_kernel(const float* __restrict__ E, const float* __restrict__ lam,
+                                    const float* __restrict__ P, int64_t N, int64_t K, int r, int tall,
+                                    float* __restrict__ Ur, float* __restrict__ Vr) {
   const int64_t nu = N * r, total = nu + static_cast<int64_t>(r) * K;
   for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < total;
        e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    int c_out;
+    int64_t pos;  // row i of Ur, or column k of Vr
     if (e < nu) {
-      const int64_t i = e / r;
-      const int c = static_cast<int>(e - i * r);
-      const float u = wide ? VT[c + i * N] : U[i + c * N];
-      Ur[e] = u * sqrtf(S[c]);
+      pos = e / r;
+      c_out = static_cast<int>(e - pos * r);
     } else {
       const int64_t f = e - nu;
-      const int c = static_cast<int>(f / K);
-      const int64_t k = f - static_cast<int64_t>(c) * K;
-      const float v = wide ? U[k + static_cast<int64_t>(c) * K] : VT[c + k * K];
-      Vr[f] = sqrtf(S[c]) * v;
+      c_out = static_cast<int>(f / K);
+      pos = f - static_cast<int64_t>(c_out) * K;
     }
+    const int c = r - 1 - c_out;                       // the eigensolver's ascending order
+    const float sq = sqrtf(sqrtf(fmaxf(lam[c], 0.f)));  // sqrt(s_c)
+    const float inv = sq > 0.f ? 1.0f / sq : 0.f;
+    float v;
+    if (e < nu)  // Ur[i][c_out]
+      v = tall ? P[pos + static_cast<int64_t>(c) * N] * inv : E[pos + static_cast<int64_t>(c) * N] * sq;
+    else         // Vr[c_out][k]
+      v = tall ? E[pos + static_cast<int64_t>(c) * K] * sq : P[pos + static_cast<int64_t>(c) * K] * inv;
+    (e < nu ? Ur : Vr)[e < nu ? e : e - nu] = v;
   }
 }
 
@@ -149,11 +158,11 @@ unsigned grid_of(int64_t n) {
 inline size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct LqLayout {
-  size_t R, T, S, U, VT, Ur, Vr, rwork, info, work, total;
+  size_t R, G, lam, P, Ur, Vr, info, work, total;
 };
 
 LqLayout lq_layout(int64_t N, int64_t K, int r, int lwork) {
-  const int64_t m = N > K ? N : K, n = N > K ? K : N;
+  const int64_t n = N < K ? N : K, m = N < K ? K : N;
   LqLayout L;
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -162,40 +171,49 @@ LqLayout lq_layout(int64_t N, int64_t K, int r, int lwork) {
     return at;
   };
   L.R = take(static_cast<size_t>(N) * K * 4);
-  L.T = take(N > K ? static_cast<size_t>(N) * K * 4 : 0);
-  L.S = take(static_cast<size_t>(n) * 4);
-  L.U = take(static_cast<size_t>(m) * n * 4);
-  L.VT = take(static_cast<size_t>(n) * n * 4);
+  L.G = take(static_cast<size_t>(n) * n * 4);
+  L.lam = take(static_cast<size_t>(n) * 4);
+  L.P = take(static_cast<size_t>(m) * r * 4);
   L.Ur = take(static_cast<size_t>(N) * r * 4);
   L.Vr = take(static_cast<size_t>(r) * K * 4);
-  L.rwork = take(static_cast<size_t>(n) * 4);
   L.info = take(4);
   L.work = take(static_cast<size_t>(lwork) * 4);
   L.total = off;
   return L;
 }
 
-// One solver handle per device, created on the first call made while that device is current and kept for
-// the life of the process (the handle's own small device allocation happens once, not per call).
-cusolverDnHandle_t device_handle() {
+// One solver and one BLAS handle per device, created on the first call made while that device is current
+// and kept for the life of the process (their own small device allocations happen once, not per call).
+struct Handles {
+  cusolverDnHandle_t sol = nullptr;
+  cublasHandle_t blas = nullptr;
+};
+
+const Handles* device_handles() {
   static std::mutex mu;
-  static cusolverDnHandle_t handles[64] = {nullptr};
+  static Handles hs[64];
   const Solver& sv = solver();
   if (!sv.ok) return nullptr;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
   std::lock_guard<std::mutex> lock(mu);
-  if (!handles[dev] && sv.create(&handles[dev]) != CUSOLVER_STATUS_SUCCESS) handles[dev] = nullptr;
-  return handles[dev];
+  Handles& h = hs[dev];
+  if (!h.sol && sv.create(&h.sol) != CUSOLVER_STATUS_SUCCESS) h.sol = nullptr;
+  if (!h.blas && sv.blas_create(&h.blas) != CUBLAS_STATUS_SUCCESS) h.blas = nullptr;
+  return (h.sol && h.blas) ? &h : nullptr;
 }
 
-int gesvd_lwork(int64_t N, int64_t K, int* lwork) {
+int evd_lwork(int64_t N, int64_t K, int r, int* lwork) {
   const Solver& sv = solver();
   if (!sv.ok) return QLR_ERR_UNSUPPORTED;
-  cusolverDnHandle_t h = device_handle();
+  const Handles* h = device_handles();
   if (!h) return QLR_ERR_CUDA;
-  const int m = static_cast<int>(N > K ? N : K), n = static_cast<int>(N > K ? K : N);
-  return sv.buffer_size(h, m, n, lwork) == CUSOLVER_STATUS_SUCCESS ? QLR_OK : QLR_ERR_CUDA;
+  const int n = static_cast<int>(N < K ? N : K);
+  int meig = 0;
+  return sv.evd_buffer(h->sol, CUSOLVER_EIG_MODE_VECTOR, CUSOLVER_EIG_RANGE_I, CUBLAS_FILL_MODE_LOWER, n, nullptr, n, 0.f,
+                       0.f, n - r + 1, n, &meig, nullptr, lwork) == CUSOLVER_STATUS_SUCCESS
+             ? QLR_OK
+             : QLR_ERR_CUDA;
 }
 
 int check_lq_args(int64_t N, int64_t K, int bits, int block, int dq_block, int r, int iters) {
@@ -215,7 +233,7 @@ using namespace qlr;
 extern "C" size_t qlr_lqlora_init_workspace_bytes(int64_t N, int64_t K, int r) {
   if (N <= 0 || K <= 0 || r < 1 || r > 64) return 0;
   int lwork = 0;
-  if (gesvd_lwork(N, K, &lwork) != QLR_OK) return 0;
+  if (evd_lwork(N, K, r, &lwork) != QLR_OK) return 0;
   return lq_layout(N, K, r, lwork).total;
 }
 
@@ -241,48 +259,55 @@ extern "C" int qlr_lqlora_init(const float* W, int64_t N, int64_t K, int bits, i
   const Solver& sv = solver();
   if (!sv.ok) return QLR_ERR_UNSUPPORTED;
   int lwork = 0;
-  if ((rc = gesvd_lwork(N, K, &lwork))) return rc;
+  if ((rc = evd_lwork(N, K, r, &lwork))) return rc;
   const LqLayout L = lq_layout(N, K, r, lwork);
   if (!workspace || workspace_bytes < L.total) return QLR_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(workspace) & 255u) return QLR_ERR_ALIGN;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   float* R = reinterpret_cast<float*>(ws + L.R);
-  float* T = reinterpret_cast<float*>(ws + L.T);
-  float* S = reinterpret_cast<float*>(ws + L.S);
-  float* U = reinterpret_cast<float*>(ws + L.U);
-  float* VT = reinterpret_cast<float*>(ws + L.VT);
+  float* G = reinterpret_cast<float*>(ws + L.G);
+  float* lam = reinterpret_cast<float*>(ws + L.lam);
+  float* P = reinterpret_cast<float*>(ws + L.P);
   float* Ur = reinterpret_cast<float*>(ws + L.Ur);
   float* Vr = reinterpret_cast<float*>(ws + L.Vr);
-  float* rwork = reinterpret_cast<float*>(ws + L.rwork);
   int* info = reinterpret_cast<int*>(ws + L.info);
   float* work = reinterpret_cast<float*>(ws + L.work);
-  const bool wide = K >= N;
-  const int m = static_cast<int>(wide ? K : N), n = static_cast<int>(wide ? N : K);
+  // R row-major [N, K] is, column-major, Rc = R^T [K x N] with leading dimension K
+  const bool tall = K <= N;
+  const int n = static_cast<int>(tall ? K : N), Ni = static_cast<int>(N), Ki = static_cast<int>(K);
+  const float one = 1.f, zero = 0.f;
 
-  cusolverDnHandle_t h = device_handle();
+  const Handles* h = device_handles();
   if (!h) return QLR_ERR_CUDA;
+  if (sv.set_stream(h->sol, st) != CUSOLVER_STATUS_SUCCESS || sv.blas_set_stream(h->blas, st) != CUBLAS_STATUS_SUCCESS)
+    return QLR_ERR_CUDA;
   rc = QLR_OK;
   for (int t = 0; t < iters && rc == QLR_OK; ++t) {
     // the residual to factor: W (t = 0), else W - dequant(Q_t)
-    if (t == 0) {
-      if (cudaMemcpyAsync(R, W, static_cast<size_t>(N) * K * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess) {
-        rc = QLR_ERR_CUDA;
-        break;
-      }
-    } else {
+    const float* Rt = W;
+    if (t > 0) {
       count_launch();
       residual_kernel<<<grid_of(N * K), 256, 0, st>>>(W, N * K, nfk::view_of(out), R);
+      Rt = R;
     }
-    // column-major operand with at least as many rows as columns
-    float* Acm = R;  // row-major N x K read as column-major K x N (ld K)
-    if (!wide) {
-      count_launch();
-      transpose_kernel<<<dim3(static_cast<unsigned>((K + 31) / 32), static_cast<unsigned>((N + 31) / 32)), dim3(32, 8), 0,
-                         st>>>(R, N, K, T);
-      Acm = T;  // column-major N x K (ld N)
+    // Gram matrix on the smaller side (lower triangle): tall G = Rc Rc^T = R^T R [K x K];
+    // wide G = Rc^T Rc = R R^T [N x N]
+    if (sv.syrk(h->blas, CUBLAS_FILL_MODE_LOWER, tall ? CUBLAS_OP_N : CUBLAS_OP_T, n, tall ? Ni : Ki, &one, Rt, Ki,
+                &zero, G, n) != CUBLAS_STATUS_SUCCESS) {
+      rc = QLR_ERR_CUDA;
+      break;
     }
-    if (sv.set_stream(h, st) != CUSOLVER_STATUS_SUCCESS ||
-        sv.gesvd(h, 'S', 'S', m, n, Acm, m, S, U, m, VT, n, work, lwork, rwork, info) != CUSOLVER_STATUS_SUCCESS) {
+    // its r largest eigenpairs (ascending; eigenvectors in G's first r columns)
+    int meig = 0;
+    if (sv.evd(h->sol, CUSOLVER_EIG_MODE_VECTOR, CUSOLVER_EIG_RANGE_I, CUBLAS_FILL_MODE_LOWER, n, G, n, 0.f, 0.f,
+               n - r + 1, n, &meig, lam, work, lwork, info) != CUSOLVER_STATUS_SUCCESS ||
+        meig != r) {
+      rc = QLR_ERR_CUDA;
+      break;
+    }
+    // the other side's factor: tall P = R V_r = Rc^T E [N x r]; wide P = R^T U_r = Rc E [K x r]
+    if (sv.gemm(h->blas, tall ? CUBLAS_OP_T : CUBLAS_OP_N, CUBLAS_OP_N, tall ? Ni : Ki, r, n, &one, Rt, Ki, G, n, &zero,
+                P, tall ? Ni : Ki) != CUBLAS_STATUS_SUCCESS) {
       rc = QLR_ERR_CUDA;
       break;
     }
@@ -293,7 +318,8 @@ extern "C" int qlr_lqlora_init(const float* W, int64_t N, int64_t K, int bits, i
       break;
     }
     count_launch(2);
-    factors_kernel<<<grid_of(N * r + static_cast<int64_t>(r) * K), 256, 0, st>>>(U, VT, S, N, K, r, wide ? 1 : 0, Ur, Vr);
+    gram_factors_kernel<<<grid_of(N * r + static_cast<int64_t>(r) * K), 256, 0, st>>>(G, lam, P, N, K, r, tall ? 1 : 0,
+                                                                                         Ur, Vr);
     lowrank_sub_kernel<<<dim3(static_cast<unsigned>((K + kLrTile - 1) / kLrTile),
                               static_cast<unsigned>((N + kLrTile - 1) / kLrTile)),
                          256, 0, st>>>(W, Ur, Vr, N, K, r, R);
