@@ -110,6 +110,17 @@ QLR_API int64_t qlr_qweight_part_bytes(int fmt, int64_t N, int64_t K, int bits, 
  * distribution per bin.)  `out` is HOST memory of 2^bits floats. */
 QLR_API int qlr_nf_levels(int bits, float* out);
 
+/* The decision table the NF-k quantiser uses for its nearest-level search (QLoRA explainer,
+ * "Background: what is quantization?": each normalised weight u = fp32(w / absmax) in [-1, 1] takes
+ * the nearest level; ties go to the lower index).  For fixed levels that choice is a step function of
+ * u, so it is fixed by 2^bits - 1 fp32 thresholds.  The table splits [-1, 1] into 33 cells, cell
+ * k = round-half-even(16 u) + 16 (computed as the bits of fma(u, 16, 1.5 * 2^23 + 16) minus those of
+ * 1.5 * 2^23), each holding at most one threshold:  code(u) = base[k] + (u >= threshold[k]), with
+ * threshold[k] = +inf for a cell without one.  `threshold` and `base` are HOST arrays of 33 entries.
+ * Returns QLR_ERR_ARG for bits outside 2 .. 4 and QLR_ERR_UNSUPPORTED if a cell would hold two
+ * thresholds (it does not for the NF-2/3/4 levels of qlr_nf_levels).  Pure host arithmetic. */
+QLR_API int qlr_nf_decision_table(int bits, float* threshold, int32_t* base);
+
 /*
  * Blockwise NF-k quantisation with optional double quantisation of the constants.
  * (QLoRA explainer, "Background: what is quantization?", "Innovation 1", the page's code

@@ -286,6 +286,17 @@ int qlr_nf_levels(int bits, float* out) {
   return QLR_OK;
 }
 
+int qlr_nf_decision_table(int bits, float* threshold, int32_t* base) {
+  if (!threshold || !base || bits < 2 || bits > 4) return QLR_ERR_ARG;
+  NfTable tab;
+  if (!nf_decision_table(bits, &tab)) return QLR_ERR_UNSUPPORTED;
+  for (int k = 0; k < 33; ++k) {
+    threshold[k] = tab.t[k];
+    base[k] = tab.base[k];
+  }
+  return QLR_OK;
+}
+
 int64_t qlr_qweight_part_bytes(int fmt, int64_t N, int64_t K, int bits, int block, int dq_block, int group,
                                int part) {
   if (N <= 0 || K <= 0) return QLR_ERR_ARG;

@@ -14,6 +14,15 @@ struct Levels {
 void nf_levels_f32(int k, float* out);
 Levels levels_for(int bits);
 
+// Nearest-level decision of the NF-k quantiser as a table over 33 cells of width 1/16 on [-1, 1]:
+// cell k = round-half-even(16 u) + 16, code(u) = base[k] + (u >= t[k]) (t[k] = +inf: no threshold).
+struct NfTable {
+  float t[33];
+  int32_t base[33];
+};
+// Builds the table of levels_for(bits) (cached); false when a cell would hold two thresholds.
+bool nf_decision_table(int bits, NfTable* out);
+
 // Status sink used when the caller passes no status word.
 int32_t* status_or_sink(int32_t* status);
 

@@ -4,6 +4,11 @@
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
 
+#include <cmath>
+#include <cstring>
+#include <limits>
+#include <mutex>
+
 #include "common.cuh"
 #include "ptx.cuh"
 
@@ -11,66 +16,72 @@ namespace qlr {
 
 namespace {
 
-// First index of the minimum of fp32 |u - level| over the ascending levels s_lv[0 .. 2^bits - 1], with
-// s_lv[0] = -1 <= u <= 1 = s_lv[last].  A binary search finds the largest i with s_lv[i] <= u; only
-// levels i and i + 1 can then be nearest (for j < i, u - s_lv[j] > u - s_lv[i] and fp32 rounding is
-// monotone; a rounding tie would need an ulp of at least the level spacing, impossible for |u| <= 1),
-// and a tie between the two goes to i, the lower index.
-__device__ __forceinline__ int nearest_level(float u, const float* s_lv, int bits) {
-  int i = 0;
-  for (int step = 1 << (bits - 1); step > 0; step >>= 1)
-    if (u >= s_lv[i + step]) i += step;
-  const int last = (1 << bits) - 1;
-  if (i == last) return last;
-  const float d0 = fabsf(__fsub_rn(u, s_lv[i]));
-  const float d1 = fabsf(__fsub_rn(u, s_lv[i + 1]));
-  return d1 < d0 ? i + 1 : i;
+// u = fp32(x / m) for every x of one block or group with a single correctly rounded reciprocal
+// y = RN(1/m) per block: q = RN(x y) lies within an ulp of x / m, the remainder x - q m is exact in one
+// fma, and RN(q + (x - q m) y) is the correctly rounded quotient (P. Markstein, "Computation of
+// elementary functions on the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990).  The
+// argument needs every intermediate in the normal range: callers take this path only for divisors in
+// [2^-64, 2^64] (and, for the INT4 groups, |x| < 2^64), where quotients of magnitude 2^-24 and up --
+// the only ones whose exact value can change a code -- keep every step normal.
+constexpr float kDivLo = 0x1p-64f, kDivHi = 0x1p64f;
+
+__device__ __forceinline__ float div_rn_by(float x, float m, float y) {
+  const float q = __fmul_rn(x, y);
+  const float rem = fmaf(-q, m, x);
+  return fmaf(rem, y, q);
+}
+
+// Nearest NF level of u in [-1, 1] from the host-built decision table (common.cuh): the cell
+// k = round-half-even(16 u) + 16 is the integer part of fma(u, 16, 1.5 * 2^23 + 16), and the cell holds
+// at most one threshold.  A NaN u (non-finite input, reported separately) lands in the last cell.
+__device__ __forceinline__ int nf_code(float u, const float2* s_tab) {
+  const float t = fmaf(u, 16.0f, 12582928.0f);
+  const uint32_t k = min(__float_as_uint(t) - 0x4B400000u, 32u);
+  const float2 e = s_tab[k];
+  return __float_as_int(e.y) + (u >= e.x ? 1 : 0);
 }
 
 // NF-k blockwise quantisation (QLoRA explainer: "Background: what is quantization?",
 // "Innovation 1: 4-bit NormalFloat (NF4)", "Innovation 2: Double Quantization").
-// One CTA per group of 256 first-level blocks (the double-quantisation group).  Each thread owns
-// 8 consecutive inputs per chunk (two 16-byte loads); every load of the CTA is issued before any
-// arithmetic, the BLOCK / 8 threads of a block combine their absmax with shuffles, and the codes
-// of a thread leave as one 32-bit (k = 4) or 16-bit (k = 2) store, or as 3-bit planes assembled over
-// four adjacent lanes (32 codes).
-constexpr int kNfThreads = 512;
+// One CTA of 256 threads per group of 256 first-level blocks (the double-quantisation group).  A thread
+// owns 8 consecutive inputs per chunk (two 16-byte loads) and walks BLOCK / 8 chunks, two at a time with
+// the next two already in flight; the BLOCK / 8 threads of a block combine their absmax with shuffles,
+// and the codes of a thread leave as one 32-bit (k = 4) or 16-bit (k = 2) store, or as 3-bit planes
+// assembled over four adjacent lanes (32 codes).
+constexpr int kNfThreads = 256;
+constexpr int kNfUnroll = 2;  // chunks per thread per step
 
-template <int BLOCK>
+template <int BLOCK, int BITS>
 __global__ void __launch_bounds__(kNfThreads) quantize_nfk_kernel(
-    const float* __restrict__ W, int64_t n_blocks, int bits, int dq_block, Levels lv, int zero_code,
+    const float* __restrict__ W, int64_t n_blocks, int dq_block, const __grid_constant__ NfTable tab, int zero_code,
     uint8_t* __restrict__ codes, float* __restrict__ c1_out, uint8_t* __restrict__ c1_fp8,
     float* __restrict__ s2_out, int32_t* status) {
   constexpr int TPB = BLOCK / 8;                         // threads per block: 8 or 16
-  constexpr int CH = 256 * BLOCK / (kNfThreads * 8);     // chunks per thread: 4 or 8
+  constexpr int NCH = 256 * BLOCK / (kNfThreads * 8);    // chunks per thread: 8 or 16
+  constexpr int NIT = NCH / kNfUnroll;
   __shared__ float s_c1[256];
   __shared__ float s_red[kNfThreads / 32];
-  __shared__ float s_lv[16];
+  __shared__ float2 s_tab[33];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  if (tid < 16) s_lv[tid] = lv.v[tid];
+  if (tid < 33) s_tab[tid] = make_float2(tab.t[tid], __int_as_float(tab.base[tid]));
   const int64_t blk0 = static_cast<int64_t>(blockIdx.x) * 256;
   const int nblk = static_cast<int>((n_blocks - blk0) < 256 ? (n_blocks - blk0) : 256);
-  const int64_t e0 = blk0 * BLOCK;  // first input of this CTA
-  const float4* src = reinterpret_cast<const float4*>(W + e0);
-  float4 v[CH][2];
-#pragma unroll
-  for (int c = 0; c < CH; ++c) {
+  const float4* src = reinterpret_cast<const float4*>(W + blk0 * BLOCK);
+  auto load = [&](int c, float4 (&v)[2]) {
     const int e = c * kNfThreads + tid;  // 8-input chunk index within the CTA
     if (e / TPB < nblk) {
-      v[c][0] = __ldg(src + 2 * e);
-      v[c][1] = __ldg(src + 2 * e + 1);
+      v[0] = __ldg(src + 2 * e);
+      v[1] = __ldg(src + 2 * e + 1);
     } else {
-      v[c][0] = v[c][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+      v[0] = v[1] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-  }
-  __syncthreads();  // s_lv
+  };
   bool bad = false;
-#pragma unroll
-  for (int c = 0; c < CH; ++c) {
+  auto quantize_chunk = [&](int c, const float4 (&v)[2]) {
     const int e = c * kNfThreads + tid;
     const int lb = e / TPB;           // block within the CTA (uniform over the block's threads)
     const bool valid = lb < nblk;
-    const float x[8] = {v[c][0].x, v[c][0].y, v[c][0].z, v[c][0].w, v[c][1].x, v[c][1].y, v[c][1].z, v[c][1].w};
+    const float x[8] = {v[0].x, v[0].y, v[0].z, v[0].w, v[1].x, v[1].y, v[1].z, v[1].w};
     float m = 0.f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -80,21 +91,30 @@ __global__ void __launch_bounds__(kNfThreads) quantize_nfk_kernel(
 #pragma unroll
     for (int o = TPB / 2; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     if (valid && (tid & (TPB - 1)) == 0) s_c1[lb] = m;
+    float u[8];
+    if (m >= kDivLo && m <= kDivHi) {
+      const float y = __frcp_rn(m);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) u[i] = div_rn_by(x[i], m, y);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) u[i] = __fdiv_rn(x[i], m);
+    }
     int code[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) code[i] = (m == 0.f) ? zero_code : nearest_level(__fdiv_rn(x[i], m), s_lv, bits);
+    for (int i = 0; i < 8; ++i) code[i] = (m == 0.f) ? zero_code : nf_code(u[i], s_tab);
     const int64_t chunk = blk0 * TPB + e;  // global 8-input chunk index
-    if (bits == 4) {
+    if constexpr (BITS == 4) {
       uint32_t word = 0;
 #pragma unroll
       for (int i = 0; i < 8; ++i) word |= static_cast<uint32_t>(code[i]) << (4 * i);
       if (valid) reinterpret_cast<uint32_t*>(codes)[chunk] = word;
-    } else if (bits == 2) {
+    } else if constexpr (BITS == 2) {
       uint32_t half = 0;
 #pragma unroll
       for (int i = 0; i < 8; ++i) half |= static_cast<uint32_t>(code[i]) << (2 * i);
       if (valid) reinterpret_cast<uint16_t*>(codes)[chunk] = static_cast<uint16_t>(half);
-    } else {  // bits == 3: lanes 4q .. 4q+3 hold 32 consecutive codes; plane word p, bit t = bit p of code t
+    } else {  // 3 bits: lanes 4q .. 4q+3 hold 32 consecutive codes; plane word p, bit t = bit p of code t
       const int q = lane & 3;
       uint32_t pl[3];
 #pragma unroll
@@ -112,6 +132,26 @@ __global__ void __launch_bounds__(kNfThreads) quantize_nfk_kernel(
         words[0] = pl[0];
         words[1] = pl[1];
         words[2] = pl[2];
+      }
+    }
+  };
+  float4 cur[kNfUnroll][2], nxt[kNfUnroll][2];
+#pragma unroll
+  for (int j = 0; j < kNfUnroll; ++j) load(j, cur[j]);
+  __syncthreads();  // s_tab
+#pragma unroll
+  for (int it = 0; it < NIT; ++it) {
+    if (it + 1 < NIT) {
+#pragma unroll
+      for (int j = 0; j < kNfUnroll; ++j) load((it + 1) * kNfUnroll + j, nxt[j]);
+    }
+#pragma unroll
+    for (int j = 0; j < kNfUnroll; ++j) quantize_chunk(it * kNfUnroll + j, cur[j]);
+    if (it + 1 < NIT) {
+#pragma unroll
+      for (int j = 0; j < kNfUnroll; ++j) {
+        cur[j][0] = nxt[j][0];
+        cur[j][1] = nxt[j][1];
       }
     }
   }
@@ -177,11 +217,22 @@ __global__ void __launch_bounds__(256) quantize_int4g_kernel(const float* __rest
   const float sc = __half2float(sc16);
   float z = 0.f;
   if (sc > 0.f) z = __fadd_rn(fminf(fmaxf(rintf(__fdiv_rn(-lo, sc)), 0.f), 15.f), 0.0f);  // +0, never -0
+  // x / sc through one reciprocal per group (div_rn_by); a group with an input of magnitude 2^64 or more,
+  // or whose fp16 scale overflowed, takes the plain division
+  float u[8];
+  if (sc <= 65504.f && fmaxf(-lo, hi) < kDivHi) {
+    const float y = sc > 0.f ? __frcp_rn(sc) : 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) u[e] = div_rn_by(x[e], sc, y);
+  } else {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) u[e] = __fdiv_rn(x[e], sc);
+  }
   uint32_t word = 0;
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
     int c = 0;
-    if (sc > 0.f) c = static_cast<int>(fminf(fmaxf(rintf(__fadd_rn(__fdiv_rn(x[e], sc), z)), 0.f), 15.f));
+    if (sc > 0.f) c = static_cast<int>(fminf(fmaxf(rintf(__fadd_rn(u[e], z)), 0.f), 15.f));
     word |= static_cast<uint32_t>(c) << (4 * e);  // element 2j in the low nibble of byte j
   }
   reinterpret_cast<uint32_t*>(codes)[t] = word;
@@ -267,22 +318,130 @@ __global__ void merge_kernel(const uint16_t* __restrict__ A, const uint16_t* __r
 
 }  // namespace
 
+namespace {
+
+template <int BLOCK>
+cudaError_t launch_nfk_block(const float* W, int64_t n_blocks, int bits, int dq_block, const NfTable& tab, int zc,
+                             const qlr_qweight* out, int32_t* status, cudaStream_t st) {
+  const unsigned grid = static_cast<unsigned>((n_blocks + 255) / 256);
+  count_launch();
+  switch (bits) {
+    case 2:
+      quantize_nfk_kernel<BLOCK, 2><<<grid, kNfThreads, 0, st>>>(W, n_blocks, dq_block, tab, zc, out->codes, out->c1,
+                                                                 out->c1_fp8, out->s2, status);
+      break;
+    case 3:
+      quantize_nfk_kernel<BLOCK, 3><<<grid, kNfThreads, 0, st>>>(W, n_blocks, dq_block, tab, zc, out->codes, out->c1,
+                                                                 out->c1_fp8, out->s2, status);
+      break;
+    default:
+      quantize_nfk_kernel<BLOCK, 4><<<grid, kNfThreads, 0, st>>>(W, n_blocks, dq_block, tab, zc, out->codes, out->c1,
+                                                                 out->c1_fp8, out->s2, status);
+      break;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+// ---- the nearest-level decision table (host) ---------------------------------------------------
+namespace {
+
+uint32_t bits_of(float f) {
+  uint32_t b;
+  std::memcpy(&b, &f, 4);
+  return b;
+}
+float float_of(uint32_t b) {
+  float f;
+  std::memcpy(&f, &b, 4);
+  return f;
+}
+// fp32 values in increasing order as integers (-0 and +0 both map to 0)
+int64_t ordinal(float f) {
+  const uint32_t b = bits_of(f);
+  return (b >> 31) ? -static_cast<int64_t>(b & 0x7FFFFFFFu) : static_cast<int64_t>(b);
+}
+float from_ordinal(int64_t o) {
+  return o < 0 ? float_of(static_cast<uint32_t>(-o) | 0x80000000u) : float_of(static_cast<uint32_t>(o));
+}
+// the rule itself: first index of the smallest fp32 |u - level|
+int nearest_by_rule(float u, const float* lv, int n) {
+  int best = 0;
+  float bd = std::fabs(u - lv[0]);
+  for (int j = 1; j < n; ++j) {
+    const float d = std::fabs(u - lv[j]);
+    if (d < bd) {
+      bd = d;
+      best = j;
+    }
+  }
+  return best;
+}
+// the device's cell of u (same fma, correctly rounded on both sides)
+int cell_of(float u) { return static_cast<int>(bits_of(std::fma(u, 16.0f, 12582928.0f)) - 0x4B400000u); }
+// smallest u of [-1, 1] where a predicate that is false below some point and true above it holds
+template <class Pred>
+int64_t first_true(Pred pred) {
+  int64_t lo = ordinal(-1.0f), hi = ordinal(1.0f);
+  while (lo < hi) {
+    const int64_t mid = lo + (hi - lo) / 2;
+    if (pred(from_ordinal(mid)))
+      hi = mid;
+    else
+      lo = mid + 1;
+  }
+  return lo;
+}
+
+// Levels i and i + 1 differ by far more than the rounding of |u - level| on [-1, 1], so the rule's
+// choice never decreases as u grows and is fixed by the smallest u reaching each code (its thresholds).
+bool build_decision_table(int bits, NfTable* tab) {
+  const Levels lv = levels_for(bits);
+  const int n = 1 << bits;
+  int64_t thr[16];
+  for (int i = 1; i < n; ++i) thr[i] = first_true([&](float u) { return nearest_by_rule(u, lv.v, n) >= i; });
+  for (int k = 0; k <= 32; ++k) {
+    const int64_t lo = first_true([&](float u) { return cell_of(u) >= k; });
+    const int64_t hi = k == 32 ? ordinal(1.0f) : first_true([&](float u) { return cell_of(u) >= k + 1; }) - 1;
+    tab->base[k] = nearest_by_rule(from_ordinal(lo), lv.v, n);
+    tab->t[k] = std::numeric_limits<float>::infinity();
+    int inside = 0;
+    for (int i = 1; i < n; ++i)
+      if (thr[i] > lo && thr[i] <= hi) {
+        tab->t[k] = from_ordinal(thr[i]);
+        ++inside;
+      }
+    if (inside > 1) return false;
+  }
+  return true;
+}
+
+}  // namespace
+
+bool nf_decision_table(int bits, NfTable* out) {
+  static std::mutex mu;
+  static NfTable cache[5];
+  static int state[5] = {0, 0, 0, 0, 0};  // 0 not built, 1 built, -1 not representable
+  if (bits < 2 || bits > 4 || !out) return false;
+  std::lock_guard<std::mutex> lock(mu);
+  if (state[bits] == 0) state[bits] = build_decision_table(bits, &cache[bits]) ? 1 : -1;
+  if (state[bits] < 0) return false;
+  *out = cache[bits];
+  return true;
+}
+
 cudaError_t launch_quantize_nfk(const float* W, int64_t n_elems, int bits, int block, int dq_block,
                                 const qlr_qweight* out, int32_t* status, cudaStream_t st) {
   const int64_t n_blocks = n_elems / block;
-  const int64_t grid = (n_blocks + 255) / 256;
+  NfTable tab;
+  if (bits < 2 || bits > 4 || !nf_decision_table(bits, &tab)) return cudaErrorInvalidValue;
   Levels lv = levels_for(bits);
   int zc = 0;
   for (int i = 0; i < (1 << bits); ++i)
     if (lv.v[i] == 0.f) zc = i;
-  count_launch();
-  if (block == 64)
-    quantize_nfk_kernel<64><<<static_cast<unsigned>(grid), kNfThreads, 0, st>>>(
-        W, n_blocks, bits, dq_block, lv, zc, out->codes, out->c1, out->c1_fp8, out->s2, status);
-  else
-    quantize_nfk_kernel<128><<<static_cast<unsigned>(grid), kNfThreads, 0, st>>>(
-        W, n_blocks, bits, dq_block, lv, zc, out->codes, out->c1, out->c1_fp8, out->s2, status);
-  return cudaGetLastError();
+  return block == 64 ? launch_nfk_block<64>(W, n_blocks, bits, dq_block, tab, zc, out, status, st)
+                     : launch_nfk_block<128>(W, n_blocks, bits, dq_block, tab, zc, out, status, st);
 }
 
 cudaError_t launch_quantize_int4g(const float* W, int64_t N, int64_t K, int group, const qlr_qweight* out,

@@ -25,7 +25,8 @@ ERRORS = {0: "OK", -1: "ERR_ARG", -2: "ERR_SHAPE", -3: "ERR_ALIGN", -4: "ERR_UNS
           -5: "ERR_NONFINITE", -6: "ERR_TIMEOUT", -7: "ERR_CUDA", -8: "ERR_WORKSPACE"}
 
 EXPORTED = (
-    "qlr_error_string", "qlr_version", "qlr_qweight_part_bytes", "qlr_nf_levels", "qlr_quantize_nf4",
+    "qlr_error_string", "qlr_version", "qlr_qweight_part_bytes", "qlr_nf_levels", "qlr_nf_decision_table",
+    "qlr_quantize_nf4",
     "qlr_quantize_int4_group", "qlr_dequant", "qlr_qalora_merge", "qlr_forward_workspace_bytes", "qlr_forward",
     "qlr_backward_lora_workspace_bytes", "qlr_backward_lora", "qlr_backward_dx_workspace_bytes",
     "qlr_backward_dx", "qlr_swiglu_forward", "qlr_swiglu_backward", "qlr_device_sm_count", "qlr_lora_down",
@@ -194,6 +195,15 @@ def nf_levels(bits: int) -> torch.Tensor:
     out = (ctypes.c_float * (1 << bits))()
     _check(lib().qlr_nf_levels(bits, ctypes.cast(out, ctypes.c_void_p)), "qlr_nf_levels")
     return torch.tensor(list(out), dtype=torch.float32)
+
+
+def nf_decision_table(bits: int):
+    """(threshold[33], base[33]) of the NF-k quantiser's nearest-level decision (host arrays)."""
+    t = (ctypes.c_float * 33)()
+    b = (ctypes.c_int32 * 33)()
+    _check(lib().qlr_nf_decision_table(bits, ctypes.cast(t, ctypes.c_void_p), ctypes.cast(b, ctypes.c_void_p)),
+           "qlr_nf_decision_table")
+    return list(t), list(b)
 
 
 def new_status(device) -> torch.Tensor:

@@ -166,3 +166,82 @@ def test_nf_quantize_ties_bit_exact(cuda_lib, bits, block, dq):
     q = qlr.quantize_nf4(f32_dev(W), bits, block, dq)
     torch.cuda.synchronize()
     _compare_nf(q, ref)
+
+
+def _ulp_neighbours(x: np.ndarray, width: int) -> np.ndarray:
+    """x and its fp32 neighbours up to `width` ulps either side (same sign)."""
+    b = np.asarray(x, np.float32).view(np.int32).astype(np.int64)
+    out = np.concatenate([(b + d) for d in range(-width, width + 1)])
+    out = out[(out >= -2 ** 31) & (out < 2 ** 31)].astype(np.int32).view(np.float32)
+    return out[np.isfinite(out)]
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+@pytest.mark.parametrize("block", [64, 128])
+def test_nf_quantize_random_divisors_at_switch_points(cuda_lib, bits, block):
+    """Quotients fp32(w / absmax) within two ulps of every switch of the oracle's code, for absmax drawn
+    log-uniformly over [1e-4, 10] and at both ends of the quantiser's one-reciprocal-per-block division
+    (2^-64, 2^64) and past them (2^-70, 2^70, plain division): every quotient that decides a code must be
+    the correctly rounded fp32 one, as in the oracle."""
+    qlr = cuda_lib
+    sw = _nf_tie_inputs(bits)
+    rng = np.random.default_rng(100 + bits)
+    ms = list((10.0 ** rng.uniform(-4, 1, 24)).astype(np.float32))
+    ms += [np.float32(v) for v in (2.0 ** -64, 2.0 ** -64 * (1 + 2.0 ** -23), 2.0 ** 64, 2.0 ** 64 * (1 - 2.0 ** -24),
+                                   2.0 ** -70, 2.0 ** 70, 1.9999999 * 2.0 ** -64)]
+    rows = []
+    for m in ms:
+        x = _ulp_neighbours((sw.astype(np.float64) * np.float64(m)).astype(np.float32), 2)
+        x = x[np.abs(x) <= m]
+        for start in range(0, x.size, block - 1):
+            blk = np.zeros(block, np.float32)
+            seg = x[start:start + block - 1]
+            blk[0] = m
+            blk[1:1 + seg.size] = seg
+            rows.append(blk)
+    W = np.concatenate(rows)
+    W = np.concatenate([W, np.zeros((-W.size) % 256, np.float32)]).reshape(-1, 256)
+    ref = Q.quantize_nfk(W, bits, block, 256)
+    q = qlr.quantize_nf4(f32_dev(W), bits, block, 256)
+    torch.cuda.synchronize()
+    _compare_nf(q, ref)
+
+
+def test_int4_group_quantize_random_scales_at_half_steps(cuda_lib):
+    """Inputs whose fp32 quotient x / scale plus the zero point lands within an ulp of k + 1/2, for groups
+    with random ranges (log-uniform over [1e-3, 10] either side of zero, or one-sided), and a group whose
+    fp16 scale overflows: the quantiser's one-reciprocal-per-group division must give the oracle's codes."""
+    qlr = cuda_lib
+    rng = np.random.default_rng(7)
+    groups = []
+    for gi in range(96):
+        a, b = (10.0 ** rng.uniform(-3, 1, 2)).astype(np.float32)
+        lo, hi = (np.float32(-a), np.float32(b)) if gi % 3 else ((np.float32(0.0), np.float32(b)) if gi % 2
+                                                                  else (np.float32(-a), np.float32(0.0)))
+        probe = np.zeros((1, 32), np.float32)
+        probe[0, 0], probe[0, 1] = lo, hi
+        pr = Q.quantize_int4_group(probe, 32)
+        sc = np.float64(pr["scale"].reshape(-1)[0].astype(np.float32))
+        z = np.float64(pr["zero"].reshape(-1)[0].astype(np.float32))
+        if sc == 0:
+            continue
+        ks = np.arange(0, 15, dtype=np.float64)
+        x = _ulp_neighbours(((ks + 0.5 - z) * sc).astype(np.float32), 1)
+        x = x[(x >= lo) & (x <= hi)]
+        for start in range(0, x.size, 30):
+            g = np.zeros(32, np.float32)
+            g[0], g[1] = lo, hi
+            seg = x[start:start + 30]
+            g[2:2 + seg.size] = seg
+            groups.append(g)
+    big = np.zeros(32, np.float32)
+    big[0], big[1], big[2], big[3] = -2.0 ** 66, 2.0 ** 65, 3.0, -1e20
+    groups.append(big)
+    W = np.stack(groups)
+    W = np.concatenate([W, np.zeros(((-W.shape[0]) % 4, 32), np.float32)]).reshape(-1, 128)
+    ref = Q.quantize_int4_group(W, 32)
+    q = qlr.quantize_int4_group(f32_dev(W), 32)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(host_bytes(q.codes), ref["packed"])
+    np.testing.assert_array_equal(q.scale.cpu().numpy().view(np.uint16), ref["scale"].view(np.uint16))
+    np.testing.assert_array_equal(q.zero.cpu().numpy().view(np.uint16), ref["zero"].view(np.uint16))
