@@ -44,15 +44,15 @@ __device__ __forceinline__ int nf_code(float u, const float2* s_tab) {
 // NF-k blockwise quantisation (QLoRA explainer: "Background: what is quantization?",
 // "Innovation 1: 4-bit NormalFloat (NF4)", "Innovation 2: Double Quantization").
 // One CTA of 256 threads per group of 256 first-level blocks (the double-quantisation group).  A thread
-// owns 8 consecutive inputs per chunk (two 16-byte loads) and walks BLOCK / 8 chunks, two at a time with
-// the next two already in flight; the BLOCK / 8 threads of a block combine their absmax with shuffles,
+// owns 8 consecutive inputs per chunk (two 16-byte loads) and walks BLOCK / 8 chunks, one at a time with
+// the next already in flight (32 registers: eight CTAs per SM); the BLOCK / 8 threads of a block combine their absmax with shuffles,
 // and the codes of a thread leave as one 32-bit (k = 4) or 16-bit (k = 2) store, or as 3-bit planes
 // assembled over four adjacent lanes (32 codes).
 constexpr int kNfThreads = 256;
-constexpr int kNfUnroll = 2;  // chunks per thread per step
+constexpr int kNfUnroll = 1;  // chunks per thread per step
 
 template <int BLOCK, int BITS>
-__global__ void __launch_bounds__(kNfThreads) quantize_nfk_kernel(
+__global__ void __launch_bounds__(kNfThreads, 8) quantize_nfk_kernel(
     const float* __restrict__ W, int64_t n_blocks, int dq_block, const __grid_constant__ NfTable tab, int zero_code,
     uint8_t* __restrict__ codes, float* __restrict__ c1_out, uint8_t* __restrict__ c1_fp8,
     float* __restrict__ s2_out, int32_t* status) {
