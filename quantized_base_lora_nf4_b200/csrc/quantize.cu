@@ -43,24 +43,25 @@ __device__ __forceinline__ int nf_code(float u, const float2* s_tab) {
 
 // NF-k blockwise quantisation (QLoRA explainer: "Background: what is quantization?",
 // "Innovation 1: 4-bit NormalFloat (NF4)", "Innovation 2: Double Quantization").
-// One CTA of 256 threads per group of 256 first-level blocks (the double-quantisation group).  A thread
-// owns 8 consecutive inputs per chunk (two 16-byte loads) and walks BLOCK / 8 chunks, one at a time with
-// the next already in flight (32 registers: eight CTAs per SM); the BLOCK / 8 threads of a block combine their absmax with shuffles,
+// One CTA of 4 BLOCK threads per group of 256 first-level blocks (the double-quantisation group).  A
+// thread owns 8 consecutive inputs per chunk (two 16-byte loads) and walks 8 chunks, one at a time with
+// the next already in flight (32 registers: 2048 threads per SM); the BLOCK / 8 threads of a block combine their absmax with shuffles,
 // and the codes of a thread leave as one 32-bit (k = 4) or 16-bit (k = 2) store, or as 3-bit planes
 // assembled over four adjacent lanes (32 codes).
-constexpr int kNfThreads = 256;
 constexpr int kNfUnroll = 1;  // chunks per thread per step
 
 template <int BLOCK, int BITS>
-__global__ void __launch_bounds__(kNfThreads, 8) quantize_nfk_kernel(
+__global__ void __launch_bounds__(4 * BLOCK, 2048 / (4 * BLOCK)) quantize_nfk_kernel(
     const float* __restrict__ W, int64_t n_blocks, int dq_block, const __grid_constant__ NfTable tab, int zero_code,
     uint8_t* __restrict__ codes, float* __restrict__ c1_out, uint8_t* __restrict__ c1_fp8,
     float* __restrict__ s2_out, int32_t* status) {
+  constexpr int kNfThreads = 4 * BLOCK;
   constexpr int TPB = BLOCK / 8;                         // threads per block: 8 or 16
-  constexpr int NCH = 256 * BLOCK / (kNfThreads * 8);    // chunks per thread: 8 or 16
+  constexpr int NCH = 256 * BLOCK / (kNfThreads * 8);    // chunks per thread: 8
   constexpr int NIT = NCH / kNfUnroll;
   __shared__ float s_c1[256];
   __shared__ float s_red[kNfThreads / 32];
+  static_assert(kNfThreads >= 256, "one thread per first-level constant of the group");
   __shared__ float2 s_tab[33];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid < 33) s_tab[tid] = make_float2(tab.t[tid], __int_as_float(tab.base[tid]));
@@ -327,15 +328,15 @@ cudaError_t launch_nfk_block(const float* W, int64_t n_blocks, int bits, int dq_
   count_launch();
   switch (bits) {
     case 2:
-      quantize_nfk_kernel<BLOCK, 2><<<grid, kNfThreads, 0, st>>>(W, n_blocks, dq_block, tab, zc, out->codes, out->c1,
+      quantize_nfk_kernel<BLOCK, 2><<<grid, 4 * BLOCK, 0, st>>>(W, n_blocks, dq_block, tab, zc, out->codes, out->c1,
                                                                  out->c1_fp8, out->s2, status);
       break;
     case 3:
-      quantize_nfk_kernel<BLOCK, 3><<<grid, kNfThreads, 0, st>>>(W, n_blocks, dq_block, tab, zc, out->codes, out->c1,
+      quantize_nfk_kernel<BLOCK, 3><<<grid, 4 * BLOCK, 0, st>>>(W, n_blocks, dq_block, tab, zc, out->codes, out->c1,
                                                                  out->c1_fp8, out->s2, status);
       break;
     default:
-      quantize_nfk_kernel<BLOCK, 4><<<grid, kNfThreads, 0, st>>>(W, n_blocks, dq_block, tab, zc, out->codes, out->c1,
+      quantize_nfk_kernel<BLOCK, 4><<<grid, 4 * BLOCK, 0, st>>>(W, n_blocks, dq_block, tab, zc, out->codes, out->c1,
                                                                  out->c1_fp8, out->s2, status);
       break;
   }
