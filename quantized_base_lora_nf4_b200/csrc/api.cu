@@ -120,14 +120,14 @@ int check_gemm_weight(const qlr_qweight* w) {
 // Width of the packed codes: NF-k codes are k bits, INT4 group codes 4.
 int code_bits(const qlr_qweight* w) { return w->fmt == QLR_FMT_NFK ? w->bits : 4; }
 
-// The fused kernel's codes ring: a 32 KB region split into a power-of-two number (at most 8) of
-// slots of one TMA box each, so the kernel indexes it with masks and shifts.
+// The fused kernel's codes ring (kCodeRingBytes) split into a power-of-two number, at most kCodeRingSlots,
+// of slots of one TMA box each, so the kernel indexes it with masks and shifts.
 void set_code_ring(GemmParams& p, int bits, int steps_per_box, int box_bytes) {
   p.code_bits = bits;
   p.code_steps = steps_per_box;
   p.code_box_bytes = box_bytes;
-  int lg = 3;
-  while (lg > 0 && (box_bytes << lg) > 32768) --lg;
+  int lg = kCodeRingSlotsLog2;
+  while (lg > 0 && (box_bytes << lg) > kCodeRingBytes) --lg;
   p.code_slots_log2 = lg;
 }
 

@@ -60,9 +60,9 @@ template <int BN>
 struct FCfg {
   static constexpr int kA = 16384;
   static constexpr int kB = BN * 128;
-  static constexpr int kC = 4096;
+  static constexpr int kC = kCodeRingBytes / kCodeRingSlots;
   static constexpr int NSA = BN >= 256 ? 3 : 4;
-  static constexpr int NSC = 8;
+  static constexpr int NSC = kCodeRingSlots;
   static constexpr int kStaging = 4 * 32 * 32 * 4;  // per epilogue warp a 32 x 32 fp32 tile
   static constexpr int kFixed = kStaging + 2048;
   static constexpr int kBudget = 227 * 1024 - kFixed - NSA * kA - NSC * kC;
@@ -80,7 +80,7 @@ struct FCfg {
 struct alignas(8) FBars {
   uint64_t b_full[8], b_empty[8];
   uint64_t a_full[4], a_empty[4];
-  uint64_t c_full[8], c_empty[8];
+  uint64_t c_full[kCodeRingSlots], c_empty[kCodeRingSlots];
   uint64_t acc_full[2], acc_empty[2];
   uint64_t drain;
   uint32_t tmem_base;

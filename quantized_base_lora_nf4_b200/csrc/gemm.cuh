@@ -33,6 +33,14 @@ struct DqParams {
   Levels lv;
 };
 
+// The fused kernel's codes ring: kCodeRingBytes of shared memory that the host splits into a power-of-two
+// number of slots of one TMA box each, at most kCodeRingSlots (the kernel initialises one full/empty
+// barrier pair per possible slot).
+constexpr int kCodeRingBytes = 32768;
+constexpr int kCodeRingSlots = 8;
+constexpr int kCodeRingSlotsLog2 = 3;
+static_assert((1 << kCodeRingSlotsLog2) == kCodeRingSlots, "slot count is a power of two");
+
 // D[Mm, Nn] = sum_k A[Mm, k] B[k, Nn]  (+ a tail segment of extra reduction columns)
 struct GemmParams {
   int Mm, Nn;            // extents of D (MMA M side = TMEM lanes, MMA N side = TMEM columns)
