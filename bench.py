@@ -369,7 +369,7 @@ def run_ours(args, wl_name, rank, world, dev, steps, warmup, e2e_steps=None, swi
         flush_l2(flush)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
-        step(record=True)
+        step()  # no events inside: one recorded between two launches keeps the second from starting early
         e1.record()
         evs.append((e0, e1))
     torch.cuda.synchronize()
@@ -378,6 +378,15 @@ def run_ours(args, wl_name, rank, world, dev, steps, warmup, e2e_steps=None, swi
         dist.barrier()
     torch.cuda.synchronize()
     clk = clocks.stop() if clocks else None
+    # the fused kernels' own durations (roofline, step breakdown): the same number of steps again, each fused
+    # launch between an event pair on its stream
+    for _ in range(steps):
+        flush_l2(flush)
+        step(record=True)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
     ms_steps = [a.elapsed_time(b) for a, b in evs]
     ms_total = sum(ms_steps)
     fwd_ms = [a.elapsed_time(b) for a, b in fwd_ev]
