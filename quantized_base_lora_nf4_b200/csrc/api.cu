@@ -402,7 +402,7 @@ int qlr_lora_down(const qlr_qweight* w, const uint16_t* X, int64_t M, const uint
   const int64_t K = w->K;
   if (!pooled && lora_down_small_supported(M)) return cuda_rc(launch_lora_down_small(X, M, K, A, r, s, T_save, st));
   if (!pooled && skinny_supported(M, K, r))
-    return cuda_rc(launch_skinny(X, M, K, A, false, s, T_save, stat, wait_limit_cycles(), st));
+    return cuda_rc(launch_skinny(X, M, K, A, false, r, s, T_save, stat, wait_limit_cycles(), st));
   if (pooled && pooled_adapter_supported(K, w->group, r))
     return cuda_rc(launch_pooled_lora_down(X, M, K, w->group, A, r, s, T_save, st));
   // T_save = bf16(s * P(X) A^T) = bf16(s * X Aexp^T), Aexp[j, k] = A[j, k / L] / L for the pooled adapter
@@ -546,7 +546,7 @@ int run_dT(const qlr_qweight* w, const uint16_t* dY, int64_t M, const uint16_t* 
            void* workspace, int32_t* status, cudaStream_t st) {
   // dT = bf16(s dY B)
   if (skinny_supported(M, w->N, r))
-    return cuda_rc(launch_skinny(dY, M, w->N, B, true, s, dT_out, status_or_sink(status), wait_limit_cycles(), st));
+    return cuda_rc(launch_skinny(dY, M, w->N, B, true, r, s, dT_out, status_or_sink(status), wait_limit_cycles(), st));
   AdapterGemm g{A_TMA_K, B_TMA_MN, adapter_bn(r), M, w->N, dY, M, w->N, B, w->N, r};
   return run_adapter(g, r, ADAPTER_ROWS_BF16, s, 1, dT_out, r, static_cast<uint8_t*>(workspace),
                      status_or_sink(status), st);

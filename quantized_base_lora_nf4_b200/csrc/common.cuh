@@ -53,11 +53,11 @@ size_t pooled_dA_workspace_bytes(int64_t M, int64_t K, int L, int r);
 cudaError_t launch_pooled_dA(const uint16_t* X, int64_t M, int64_t K, int L, const uint16_t* dT, int r, float* dA,
                              float* part, cudaStream_t st);
 
-// The rank-64 products T = bf16(s X A^T) (A [64, K]) and dT = bf16(s dY B) (B [K, 64], w_is_k_by_64) at
-// 1024 or more tokens in one launch: clusters of 4 CTAs split K and sum their partial tiles in shared
-// memory in a fixed order (skinny.cu).  No workspace.
+// The rank-r products T = bf16(s X A^T) (A [r, K]) and dT = bf16(s dY B) (B [K, r], w_is_k_by_r), r = 16, 32
+// or 64, at 1024 or more tokens in one launch: clusters of 4 CTAs split K and sum their partial tiles in
+// shared memory in a fixed order (skinny.cu).  No workspace.
 bool skinny_supported(int64_t M, int64_t K, int r);
-cudaError_t launch_skinny(const uint16_t* X, int64_t M, int64_t K, const uint16_t* W, bool w_is_k_by_64, float s,
+cudaError_t launch_skinny(const uint16_t* X, int64_t M, int64_t K, const uint16_t* W, bool w_is_k_by_r, int r, float s,
                           uint16_t* out, int32_t* status, long long wait_cycles, cudaStream_t st);
 
 // T = bf16(s X A^T) for 1..16 tokens without pooling: one fixed-order reduction kernel, no workspace.

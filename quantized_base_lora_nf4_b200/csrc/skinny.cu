@@ -1,13 +1,13 @@
-// The rank-64 adapter products at many tokens in one launch (QLoRA explainer, "Background: how LoRA
-// works": the adapter's down-projection; its gradient dT = s dY B for the backward):
-//     OUT[m, j] = bf16( s * sum_k X[m, k] W(k, j) ),   X [M, K] bf16 row-major, j < 64,
-// with W(k, j) = A[j, k] (A [64, K] row-major: T_save = bf16(s X A^T)) or W(k, j) = B[k, j] (B [K, 64]
+// The adapter products of rank r = 16, 32 or 64 at many tokens in one launch (QLoRA explainer,
+// "Background: how LoRA works": the adapter's down-projection; its gradient dT = s dY B for the backward):
+//     OUT[m, j] = bf16( s * sum_k X[m, k] W(k, j) ),   X [M, K] bf16 row-major, j < r,
+// with W(k, j) = A[j, k] (A [r, K] row-major: T_save = bf16(s X A^T)) or W(k, j) = B[k, j] (B [K, r]
 // row-major: dT = bf16(s dY B)).
 //
 // The reduction is long (K = 4096 .. 11008) and the output narrow, so a launch must split K to keep
 // every SM streaming.  Here a cluster of 4 CTAs owns 64 tokens, each CTA a quarter of K: a TMA producer
-// warp streams [64 tokens x 64 k] tiles of X and [64 x 64] tiles of W into an 8-stage ring, four warps
-// multiply them with mma.sync (16 tokens x 64 outputs each, fp32 accumulate), and the four fp32
+// warp streams [64 tokens x 64 k] tiles of X and [r x 64 k] tiles of W into an 8-stage ring, four warps
+// multiply them with mma.sync (16 tokens x r outputs each, fp32 accumulate), and the four fp32
 // partial tiles are summed in shared memory across the cluster (CTA c sums rows 16c .. 16c+15 over the
 // ranks in order 0..3, a fixed order), scaled and written as bf16.  No partial sums reach global memory
 // and no second launch is needed.
@@ -26,7 +26,7 @@ constexpr int kSkCluster = 4;                    // CTAs per cluster (quarters o
 constexpr int kSkRows = 64;                      // tokens per cluster
 constexpr int kSkStages = 8;
 constexpr int kSkTile = 64 * 128;                // one [64 x 64] bf16 tile, 128-byte rows
-constexpr int kSkStage = 2 * kSkTile;            // X tile + W tile
+constexpr int kSkStage = 2 * kSkTile;            // X tile + W tile (r x 64 bf16, at most as large)
 constexpr int kSkPartStride = 72;                // fp32 row stride of the partial tile (bank spread)
 constexpr int kSkPartBytes = kSkRows * kSkPartStride * 4;
 constexpr int kSkThreads = 5 * 32;               // 4 MMA warps + 1 TMA warp
@@ -62,14 +62,17 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
-// byte offset of 16-byte chunk `ch` of row `row` in a tile written by TMA with the 128-byte swizzle
-__device__ __forceinline__ uint32_t sw128(int row, int ch) {
-  return static_cast<uint32_t>(row * 128 + ((ch ^ (row & 7)) << 4));
+// byte offset of 16-byte chunk `ch` of row `row` in a tile of RB-byte rows written by TMA with the RB-byte
+// swizzle (RB = 128, 64 or 32): the chunk bits of the offset are XORed with the bits from 7 up
+template <int RB>
+__device__ __forceinline__ uint32_t swz(int row, int ch) {
+  const int off = row * RB + ch * 16;
+  return static_cast<uint32_t>(off ^ (((off >> 7) & (RB / 16 - 1)) << 4));
 }
 
-// TRANS_W: W is B [K, 64] (a tile holds 64 k rows of 64 outputs) rather than A [64, K] (64 output rows of
-// 64 k).
-template <bool TRANS_W>
+// TRANS_W: W is B [K, R] (a tile holds 64 k rows of R outputs, 2R-byte rows) rather than A [R, K] (R output
+// rows of 64 k).
+template <bool TRANS_W, int R>
 __global__ void __launch_bounds__(kSkThreads, 1) skinny_kernel(const __grid_constant__ SkinnyParams p,
                                                                const __grid_constant__ CUtensorMap tm_x,
                                                                const __grid_constant__ CUtensorMap tm_w) {
@@ -105,9 +108,9 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_kernel(const __grid_cons
   pdl_wait();
   __syncthreads();
 
-  float acc[8][4];
+  float acc[R / 8][4];
 #pragma unroll
-  for (int n = 0; n < 8; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+  for (int n = 0; n < R / 8; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
 
   if (warp == 4) {
     // ------------------------------------------------------------------ TMA producer
@@ -118,7 +121,7 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_kernel(const __grid_cons
         if (!mbar_wait(&bars->empty[st], ((s / kSkStages) & 1) ^ 1, abort_flag, p.wait_cycles)) break;
         uint8_t* dst = ring + st * kSkStage;
         const int32_t k = static_cast<int32_t>(k_begin + 64 * ((s + rot) % nsteps));
-        mbar_arrive_expect_tx(&bars->full[st], kSkStage);
+        mbar_arrive_expect_tx(&bars->full[st], kSkTile + 128 * R);
         tma_load_2d(dst, &tm_x, k, static_cast<int32_t>(m0), &bars->full[st]);
         if (TRANS_W)
           tma_load_2d(dst + kSkTile, &tm_w, 0, k, &bars->full[st]);
@@ -143,16 +146,16 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_kernel(const __grid_cons
       for (int kk = 0; kk < 4; ++kk) {
         uint32_t a[4];
         const int ar = 16 * warp + (lane & 15);
-        ldsm_x4(xt + sw128(ar, 2 * kk + (lane >> 4)), a);
+        ldsm_x4(xt + swz<128>(ar, 2 * kk + (lane >> 4)), a);
 #pragma unroll
-        for (int np = 0; np < 4; ++np) {  // output tiles 2 np, 2 np + 1 (8 outputs each)
+        for (int np = 0; np < R / 16; ++np) {  // output tiles 2 np, 2 np + 1 (8 outputs each)
           uint32_t b[4];
           if (TRANS_W) {  // tile rows are k: transpose while loading
             const int kr = 16 * kk + (lane & 7) + ((q8 & 1) << 3);
-            ldsm_x4_t(wt + sw128(kr, 2 * np + (q8 >> 1)), b);
+            ldsm_x4_t(wt + swz<2 * R>(kr, 2 * np + (q8 >> 1)), b);
           } else {        // tile rows are outputs j
             const int jr = 16 * np + (lane & 7) + ((q8 >> 1) << 3);
-            ldsm_x4(wt + sw128(jr, 2 * kk + (q8 & 1)), b);
+            ldsm_x4(wt + swz<128>(jr, 2 * kk + (q8 & 1)), b);
           }
           mma_16816(acc[2 * np], a, b[0], b[1]);
           mma_16816(acc[2 * np + 1], a, b[2], b[3]);
@@ -163,17 +166,17 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_kernel(const __grid_cons
     }
     // this CTA's partial tile: rows g, g + 8 of the warp's 16, columns 8 n + 2 t, + 1
 #pragma unroll
-    for (int n = 0; n < 8; ++n) {
+    for (int n = 0; n < R / 8; ++n) {
       float* r0 = part + (16 * warp + g) * kSkPartStride + 8 * n + 2 * t;
       *reinterpret_cast<float2*>(r0) = make_float2(acc[n][0], acc[n][1]);
       *reinterpret_cast<float2*>(r0 + 8 * kSkPartStride) = make_float2(acc[n][2], acc[n][3]);
     }
   }
   cluster_sync_all();  // every partial tile of the cluster written
-  if (warp < 4) {
+  if (threadIdx.x < 2 * R) {
     // rank c sums rows 16 c .. 16 c + 15 over the four partial tiles in rank order: 8 outputs a thread
-    const int row = 16 * static_cast<int>(rank) + (threadIdx.x >> 3);
-    const int col = (threadIdx.x & 7) * 8;
+    const int row = 16 * static_cast<int>(rank) + static_cast<int>(threadIdx.x) / (R / 8);
+    const int col = (static_cast<int>(threadIdx.x) % (R / 8)) * 8;
     const uint32_t local = smem_u32(part + row * kSkPartStride + col);
     float sum[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -190,17 +193,17 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_kernel(const __grid_cons
       o.y = pack_bf16x2_rn(__fmul_rn(p.s, sum[2]), __fmul_rn(p.s, sum[3]));
       o.z = pack_bf16x2_rn(__fmul_rn(p.s, sum[4]), __fmul_rn(p.s, sum[5]));
       o.w = pack_bf16x2_rn(__fmul_rn(p.s, sum[6]), __fmul_rn(p.s, sum[7]));
-      *reinterpret_cast<uint4*>(p.out + m * 64 + col) = o;
+      *reinterpret_cast<uint4*>(p.out + m * R + col) = o;
     }
   }
   cluster_sync_all();  // no CTA leaves while another still reads its partial tile
   if (threadIdx.x == 0 && bars->abort_flag) report(p.status, QLR_ERR_TIMEOUT);
 }
 
-template <bool TRANS_W>
+template <bool TRANS_W, int R>
 cudaError_t launch_skinny_variant(const SkinnyParams& p, const CUtensorMap& tx, const CUtensorMap& tw, int grid,
                                   cudaStream_t st) {
-  auto kern = skinny_kernel<TRANS_W>;
+  auto kern = skinny_kernel<TRANS_W, R>;
   const cudaError_t e = ensure_max_dynamic_smem(kern, kSkSmem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -223,13 +226,15 @@ cudaError_t launch_skinny_variant(const SkinnyParams& p, const CUtensorMap& tx, 
 
 }  // namespace
 
-bool skinny_supported(int64_t M, int64_t K, int r) { return r == 64 && M >= 1024 && K % 64 == 0; }
+bool skinny_supported(int64_t M, int64_t K, int r) {
+  return (r == 16 || r == 32 || r == 64) && M >= 1024 && K % 64 == 0;
+}
 
-cudaError_t launch_skinny(const uint16_t* X, int64_t M, int64_t K, const uint16_t* W, bool w_is_k_by_64, float s,
+cudaError_t launch_skinny(const uint16_t* X, int64_t M, int64_t K, const uint16_t* W, bool w_is_k_by_r, int r, float s,
                           uint16_t* out, int32_t* status, long long wait_cycles, cudaStream_t st) {
   CUtensorMap tx, tw;
   if (make_tmap(&tx, X, 2, M, K, kSkRows, 64, 128)) return cudaErrorInvalidValue;
-  if (w_is_k_by_64 ? make_tmap(&tw, W, 2, K, 64, 64, 64, 128) : make_tmap(&tw, W, 2, 64, K, 64, 64, 128))
+  if (w_is_k_by_r ? make_tmap(&tw, W, 2, K, r, 64, r, 2 * r) : make_tmap(&tw, W, 2, r, K, r, 64, 128))
     return cudaErrorInvalidValue;
   SkinnyParams p;
   p.M = M;
@@ -240,8 +245,15 @@ cudaError_t launch_skinny(const uint16_t* X, int64_t M, int64_t K, const uint16_
   p.status = status;
   p.wait_cycles = wait_cycles;
   const int grid = static_cast<int>((M + kSkRows - 1) / kSkRows) * kSkCluster;
-  return w_is_k_by_64 ? launch_skinny_variant<true>(p, tx, tw, grid, st)
-                      : launch_skinny_variant<false>(p, tx, tw, grid, st);
+  switch (r) {
+    case 16: return w_is_k_by_r ? launch_skinny_variant<true, 16>(p, tx, tw, grid, st)
+                                : launch_skinny_variant<false, 16>(p, tx, tw, grid, st);
+    case 32: return w_is_k_by_r ? launch_skinny_variant<true, 32>(p, tx, tw, grid, st)
+                                : launch_skinny_variant<false, 32>(p, tx, tw, grid, st);
+    case 64: return w_is_k_by_r ? launch_skinny_variant<true, 64>(p, tx, tw, grid, st)
+                                : launch_skinny_variant<false, 64>(p, tx, tw, grid, st);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace qlr
