@@ -249,7 +249,9 @@ QLR_API int qlr_forward(const qlr_qweight* w, const uint16_t* X, int64_t M, cons
 /* The two stages of qlr_forward, callable separately (same arguments and buffers):
  *   qlr_lora_down     T_save = bf16(s * P(X) A^T)      (split-K tensor-core GEMM + fixed-order sum; for
  *                     1..16 tokens without pooling, and for the pooled adapter, one fixed-order
- *                     reduction kernel straight from X and no workspace)
+ *                     reduction kernel straight from X and no workspace; for r in {16, 32, 64} at 1024
+ *                     or more tokens without pooling, one launch of 4-CTA clusters that split K and sum
+ *                     their partials in shared memory in a fixed order, no workspace)
  *   qlr_forward_base  Y = bf16(X dequant(W)^T + T_save B^T)   (the fused dequant + tcgen05 kernel)
  * qlr_lora_down uses the workspace of qlr_forward_workspace_bytes; qlr_forward_base needs none. */
 QLR_API int qlr_lora_down(const qlr_qweight* w, const uint16_t* X, int64_t M, const uint16_t* A, int r, float s,
