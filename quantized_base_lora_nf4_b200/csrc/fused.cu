@@ -35,6 +35,10 @@ constexpr int kThreadsFused = 480;
 // so the dequantisers' integer work does not delay the next MMAs.  With BN-token tiles the
 // dequantisation per MMA doubles and the eight dequantiser warps are spread two per scheduler instead.
 constexpr int kIssuerWarp = 1;
+// Warps in a dequantiser group (128 tile rows) and in the epilogue (four TMEM lane quadrants).  Each of
+// these warps signals its part of a stage or tile with one barrier arrival from lane 0 after a warp
+// sync: 32 arrivals at one shared-memory address would be serialised by the memory pipe.
+constexpr int kGroupWarps = 4;
 template <bool PAIR>
 struct Roles {
   static constexpr int kActWarp = PAIR ? 9 : 0;
@@ -146,16 +150,16 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
       mbar_init(&bars->b_empty[s], 1);
     }
     for (int s = 0; s < NSA; ++s) {
-      mbar_init(&bars->a_full[s], 128);
+      mbar_init(&bars->a_full[s], kGroupWarps);
       mbar_init(&bars->a_empty[s], 1);
     }
     for (int s = 0; s < NSC; ++s) {
       mbar_init(&bars->c_full[s], 1);
-      mbar_init(&bars->c_empty[s], 128 * p.code_steps);  // every step of a box is one dequantiser group
+      mbar_init(&bars->c_empty[s], kGroupWarps * p.code_steps);  // every step of a box is one dequantiser group
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&bars->acc_full[a], 1);
-      mbar_init(&bars->acc_empty[a], 128);
+      mbar_init(&bars->acc_empty[a], kGroupWarps);
     }
     mbar_init(&bars->drain, 1);
     bars->abort_flag = 0;
@@ -348,7 +352,8 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
           eng::store_chunk_f32_t<EPI>(v, stgf, lane, n0 + c * 32, m0 + q * 32, p);
       }
       tc_fence_before();
-      mbar_arrive(&bars->acc_empty[acc]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->acc_empty[acc]);
     }
   } else {
     // ------------------------------------------------------------------ dequantisers (warps 6..13)
@@ -414,13 +419,14 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
       const eng::DqConst nxt = have_next ? prefetch() : eng::DqConst{0u, 0u};
 
       const int sa = c_j % NSA;
-      if (!mbar_wait(&bars->a_empty[sa], ((c_j / NSA) & 1) ^ 1, abort_flag, p.wait_cycles)) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->a_empty[sa], ((c_j / NSA) & 1) ^ 1, abort_flag, p.wait_cycles)))
+        break;
       uint8_t* st_a = ring_a + sa * C::kA;
       if (c_ks < nmain) {
         const int kb = p.code_bits, lg = p.code_slots_log2;
         const uint32_t box = p.code_steps == 2 ? c_jc >> 1 : c_jc, sub = p.code_steps == 2 ? (c_jc & 1) : 0;
         const int sc = static_cast<int>(box & ((1u << lg) - 1u));
-        if (!mbar_wait(&bars->c_full[sc], (box >> lg) & 1, abort_flag, p.wait_cycles)) break;
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars->c_full[sc], (box >> lg) & 1, abort_flag, p.wait_cycles))) break;
         const uint8_t* st_c = ring_c + sc * p.code_box_bytes;
         int64_t row, col;
         bool valid;
@@ -433,7 +439,8 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
           eng::dequant_row64(p.dq, st_c + nr * 16 * kb + h * 8 * kb, kb, cur, valid, st_a + h * 8192 + nr * 128,
                              nr & 7);
         }
-        mbar_arrive(&bars->c_empty[sc]);
+        __syncwarp();  // the warp's code reads are done
+        if (lane == 0) mbar_arrive(&bars->c_empty[sc]);
       } else {
         const int kt = (c_ks - nmain) * 64;
         if (!MN) {  // B_lora[m0 + t, kt .. kt + 63]
@@ -450,8 +457,9 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
             copy_row64(src, row < p.tail_a_rows, c_m0 + 64 * h, p.tail_a_cols, st_a + h * 8192 + nr * 128, nr & 7);
         }
       }
-      fence_proxy_async_smem();
-      mbar_arrive(&bars->a_full[sa]);
+      fence_proxy_async_smem();  // each thread's tile stores, before the MMA reads them
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->a_full[sa]);
       cur = nxt;
       have = have_next;
     }
