@@ -55,6 +55,33 @@ __device__ __forceinline__ uint4 lut8(const Lut& t, uint32_t w) {
   return r;
 }
 
+// The first eight entries of a table, for codes below 8 (2- and 3-bit codes unpacked to 4-bit fields):
+// each 4-bit field is itself a byte-permute selector (its top bit, the sign-replicate flag, is clear),
+// so one permute per byte plane and the two interleaves give 4 codes.
+struct Lut8 {
+  uint32_t l0, l1, h0, h1;
+};
+
+__device__ __forceinline__ Lut8 make_lut8(const float (&v)[8]) {
+  uint32_t p[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) p[j] = pack_bf16x2_rn(v[2 * j], v[2 * j + 1]);
+  return Lut8{prmt(p[0], p[1], 0x6420), prmt(p[2], p[3], 0x6420), prmt(p[0], p[1], 0x7531),
+              prmt(p[2], p[3], 0x7531)};
+}
+
+__device__ __forceinline__ uint4 lut8_small(const Lut8& t, uint32_t w) {
+  uint4 r;
+  const uint32_t lo0 = prmt(t.l0, t.l1, w), hi0 = prmt(t.h0, t.h1, w);
+  const uint32_t w1 = w >> 16;
+  const uint32_t lo1 = prmt(t.l0, t.l1, w1), hi1 = prmt(t.h0, t.h1, w1);
+  r.x = prmt(lo0, hi0, 0x5140);
+  r.y = prmt(lo0, hi0, 0x7362);
+  r.z = prmt(lo1, hi1, 0x5140);
+  r.w = prmt(lo1, hi1, 0x7362);
+  return r;
+}
+
 // Per-thread scale data of one 64-code run, loaded one stage ahead of its use so the global-memory
 // latency overlaps the dequantisation of the previous stage.
 //   NF with double quantisation: a = E4M3 byte of the block, b = bits of its fp32 second-level constant;
@@ -92,6 +119,16 @@ __device__ __forceinline__ Lut nf_lut_c(const DqParams& dq, const DqConst& c) {
 #pragma unroll
   for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(dq.lv.v[i], scale);
   return make_lut(v);
+}
+
+// The 2^bits <= 8 levels of a 2- or 3-bit NF block (entries past the last level are never selected).
+__device__ __forceinline__ Lut8 nf_lut8_c(const DqParams& dq, const DqConst& c) {
+  const float scale = dq.dq_block ? __fmul_rn(e4m3_to_f32(static_cast<uint8_t>(c.a)), __uint_as_float(c.b))
+                                  : __uint_as_float(c.a);
+  float v[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(dq.lv.v[i], scale);
+  return make_lut8(v);
 }
 
 __device__ __forceinline__ Lut int4_lut_c(uint32_t sc_bits16, uint32_t z_bits16) {
@@ -152,7 +189,9 @@ __device__ __forceinline__ void load_codes64(const uint8_t* src, int bits, uint3
 
 // Dequantise 64 consecutive codes (one run of a row of W, `bits` wide, its scale data in `c`) into
 // the eight 16-byte chunks of one 128-byte swizzled shared-memory row at `dst_row` (`sw` = row index
-// for the swizzle).
+// for the swizzle).  SMALL: the weight is 2- or 3-bit NF, looked up in the table's first eight entries
+// (a separate instantiation, so the 4-bit and INT4 code paths stay as compact as before).
+template <bool SMALL>
 __device__ __forceinline__ void dequant_row64(const DqParams& dq, const uint8_t* codes_smem, int bits, const DqConst& c,
                                               bool valid, uint8_t* dst_row, int sw) {
   if (!valid) {
@@ -162,6 +201,12 @@ __device__ __forceinline__ void dequant_row64(const DqParams& dq, const uint8_t*
   }
   uint32_t w[8];
   load_codes64(codes_smem, bits, w);
+  if constexpr (SMALL) {
+    const Lut8 t = nf_lut8_c(dq, c);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) *reinterpret_cast<uint4*>(dst_row + ((k ^ sw) << 4)) = lut8_small(t, w[k]);
+    return;
+  }
   if (dq.fmt == QLR_FMT_NFK) {
     const Lut t = nf_lut_c(dq, c);
 #pragma unroll

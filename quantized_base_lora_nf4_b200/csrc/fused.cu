@@ -122,7 +122,8 @@ __device__ __forceinline__ void copy_row64_pooled(const uint16_t* src_row, bool 
 // PAIR: one tile covers 2 x BN tokens with both TMEM accumulators, so every dequantised weight
 // stage feeds twice the MMA work (the epilogue then does not overlap the next tile's main loop).
 // EPI: EPI_STORE (with a run-time accumulate flag), EPI_SWIGLU_FWD or EPI_SWIGLU_BWD (see GemmParams).
-template <int A_SRC, int BN, bool PAIR, int EPI>
+// SMALL: the weight is 2- or 3-bit NF (the dequantisers' eight-entry lookup).
+template <int A_SRC, int BN, bool PAIR, int EPI, bool SMALL>
 __global__ void __launch_bounds__(kThreadsFused, 1)
     fused_kernel(const __grid_constant__ GemmParams p, const __grid_constant__ GemmMaps maps) {
   using C = FCfg<BN>;
@@ -432,11 +433,11 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
         bool valid;
         run_of(c_m0, c_ks * 64, row, col, valid);
         if (!MN) {  // row t: 8 kb bytes per step, code_steps steps per box row
-          eng::dequant_row64(p.dq, st_c + t * 8 * kb * p.code_steps + sub * 8 * kb, kb, cur, valid, st_a + t * 128,
+          eng::dequant_row64<SMALL>(p.dq, st_c + t * 8 * kb * p.code_steps + sub * 8 * kb, kb, cur, valid, st_a + t * 128,
                              t & 7);
         } else {    // reduction row nr: 16 kb bytes (128 codes), half h
           const int nr = t & 63, h = t >> 6;
-          eng::dequant_row64(p.dq, st_c + nr * 16 * kb + h * 8 * kb, kb, cur, valid, st_a + h * 8192 + nr * 128,
+          eng::dequant_row64<SMALL>(p.dq, st_c + nr * 16 * kb + h * 8 * kb, kb, cur, valid, st_a + h * 8192 + nr * 128,
                              nr & 7);
         }
         __syncwarp();  // the warp's code reads are done
@@ -475,10 +476,10 @@ __global__ void __launch_bounds__(kThreadsFused, 1)
   if (threadIdx.x == 0 && bars->abort_flag) report(p.status, QLR_ERR_TIMEOUT);
 }
 
-template <int A_SRC, int BN, bool PAIR, int EPI>
+template <int A_SRC, int BN, bool PAIR, int EPI, bool SMALL>
 cudaError_t launch_fused_variant(const GemmParams& p, const GemmMaps& maps, cudaStream_t st) {
   using C = FCfg<BN>;
-  auto kern = fused_kernel<A_SRC, BN, PAIR, EPI>;
+  auto kern = fused_kernel<A_SRC, BN, PAIR, EPI, SMALL>;
   const cudaError_t attr_err = ensure_max_dynamic_smem(kern, C::kSmem + 1024);
   if (attr_err != cudaSuccess) return attr_err;
   const int items = p.n_items;
@@ -489,26 +490,33 @@ cudaError_t launch_fused_variant(const GemmParams& p, const GemmMaps& maps, cuda
 }  // namespace
 
 namespace {
-template <int A_SRC, int EPI>
+template <int A_SRC, int EPI, bool SMALL>
 cudaError_t launch_fused_epi(int bn, const GemmParams& p, const GemmMaps& maps, cudaStream_t st) {
-  if (bn == 512) return launch_fused_variant<A_SRC, 256, true, EPI>(p, maps, st);
-  if (bn == 256) return launch_fused_variant<A_SRC, 256, false, EPI>(p, maps, st);
-  if (bn == 64) return launch_fused_variant<A_SRC, 64, false, EPI>(p, maps, st);
+  if (bn == 512) return launch_fused_variant<A_SRC, 256, true, EPI, SMALL>(p, maps, st);
+  if (bn == 256) return launch_fused_variant<A_SRC, 256, false, EPI, SMALL>(p, maps, st);
+  if (bn == 64) return launch_fused_variant<A_SRC, 64, false, EPI, SMALL>(p, maps, st);
   return cudaErrorNotSupported;
 }
 }  // namespace
 
 // bn = tokens per tile: 512 (paired 256-column accumulators), 256 or 64; the epilogue mode is p.epi (the
 // SwiGLU forward only with the forward, the SwiGLU backward only with the input gradient).
+// 2- and 3-bit NF weights with the plain epilogue take the eight-entry lookup instantiation, every other
+// case the general one.
 cudaError_t launch_fused(int a_src, int bn, const GemmParams& p, const GemmMaps& maps, cudaStream_t st) {
   if (p.splits != 1) return cudaErrorNotSupported;
+  const bool small = p.dq.fmt == QLR_FMT_NFK && p.code_bits < 4;
   if (a_src == A_DQ_K) {
-    if (p.epi == EPI_STORE) return launch_fused_epi<A_DQ_K, EPI_STORE>(bn, p, maps, st);
-    if (p.epi == EPI_SWIGLU_FWD) return launch_fused_epi<A_DQ_K, EPI_SWIGLU_FWD>(bn, p, maps, st);
+    if (p.epi == EPI_STORE)
+      return small ? launch_fused_epi<A_DQ_K, EPI_STORE, true>(bn, p, maps, st)
+                   : launch_fused_epi<A_DQ_K, EPI_STORE, false>(bn, p, maps, st);
+    if (p.epi == EPI_SWIGLU_FWD) return launch_fused_epi<A_DQ_K, EPI_SWIGLU_FWD, false>(bn, p, maps, st);
   }
   if (a_src == A_DQ_MN) {
-    if (p.epi == EPI_STORE) return launch_fused_epi<A_DQ_MN, EPI_STORE>(bn, p, maps, st);
-    if (p.epi == EPI_SWIGLU_BWD) return launch_fused_epi<A_DQ_MN, EPI_SWIGLU_BWD>(bn, p, maps, st);
+    if (p.epi == EPI_STORE)
+      return small ? launch_fused_epi<A_DQ_MN, EPI_STORE, true>(bn, p, maps, st)
+                   : launch_fused_epi<A_DQ_MN, EPI_STORE, false>(bn, p, maps, st);
+    if (p.epi == EPI_SWIGLU_BWD) return launch_fused_epi<A_DQ_MN, EPI_SWIGLU_BWD, false>(bn, p, maps, st);
   }
   return cudaErrorNotSupported;
 }
