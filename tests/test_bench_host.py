@@ -2,6 +2,7 @@
 kernel source it was captured on is unchanged and every launch asked for was captured, the measured peaks
 are preferred to the fallback, and the CPU baseline times the oracle with fp32 contractions."""
 import json
+import os
 
 import bench
 from synth import workload
@@ -36,6 +37,18 @@ def test_traffic_keys_name_shape_format_and_tokens():
     assert k.startswith("fwd:4096x4096:nf") and k.endswith(":r64:M2048")
     q = workload("qalora").linears[0]
     assert bench.traffic_key("dx", q, 2048) == "dx:4096x4096:int4g32:r16:M2048"
+
+
+def test_committed_capture_covers_every_fused_launch_of_the_step_workloads():
+    """The committed capture has a key for the forward and the input gradient of every linear of the three
+    step workloads (the stack, the QA-LoRA layer, the MLP block), so roofline.traffic is reported for each
+    while the capture matches the kernel source."""
+    with open(os.path.join(bench.ROOT, "profiles", "fused_traffic.json")) as f:
+        have = set(json.load(f)["bytes_per_launch"])
+    for name, M in (("lqlora", 2048), ("qalora", 2048), ("mlp7b", 4096)):
+        for spec in workload(name).linears:
+            for kind in ("fwd", "dx"):
+                assert bench.traffic_key(kind, spec, M) in have, (name, kind, spec.name)
 
 
 def test_measured_peaks_preferred(tmp_path, monkeypatch):
